@@ -1,0 +1,269 @@
+"""Seeded synthetic workloads for paged decode attention.
+
+This module is the ONLY thing the CUDA path and the CPU oracle share.  It
+draws inputs -- shapes, N(0,1) values rounded to bf16 by torch, shuffled
+physical block ids, context lengths, slot ids of the appended tokens -- and
+holds none of the method's arithmetic: no attention, no quantisation, no
+gather.  (Slot ids and table rows are plain bookkeeping: logical block i of a
+sequence sits in physical block table[i], token t in slot table[t//bs]*bs + t%bs.)
+
+Workloads (shaped like the pages' Llama-3-8B examples; names say what they are):
+
+=====================  ==========================================================
+tiny_gqa2_d64          2 seqs, ctx 37 and 80 cached (+1 appended each), 4 q / 2 kv
+                       heads, d 64, bs 16, pool of 16 blocks in seeded random order
+llama3_8b_b64          64 seqs, 32 q / 8 kv heads, d 128, bf16, bs 16,
+                       ctx ~ U{512..4096} (incl. the appended token), pool 1.1x demand
+long_context_b8        8 seqs, 32 / 8 heads, d 128, bf16, bs 16, ctx ~ U{32768..131072},
+                       split-context partitions of 512 tokens
+shared_prefix_4x8      4 prompts x 2048 tokens, each shared by 8 samples through
+                       identical physical ids; private tails ~ U{0..256}
+fp8_mha_b32_bs{16,32,64}  32 seqs, 32 q / 32 kv heads, d 128, E4M3 cache with a
+                       per-tensor fp32 scale max|x|/448, ctx 4096
+=====================  ==========================================================
+
+Values: q, K, V ~ N(0, 1) drawn in fp32 by ``torch.Generator(device).manual_seed(seed)``
+and rounded to bf16 by torch.  Cache slots no sequence owns (the tail of a
+partially filled last block, and every block no table references) hold a NaN
+sentinel, so any read of them into a result shows up.  Table entries past a
+sequence's last block are -1.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+from typing import Optional
+
+import torch
+
+BF16_NAN = 0x7FC1          # bf16 quiet NaN with a payload: the "never read this" sentinel
+E4M3_NAN = 0x7F            # E4M3 NaN code
+
+CONFIGS = {
+    "tiny_gqa2_d64": dict(B=2, h_q=4, h_kv=2, d=64, bs=16, cache="bf16", ctx_cached=(37, 80),
+                          num_blocks=16, partition=0),
+    "llama3_8b_b64": dict(B=64, h_q=32, h_kv=8, d=128, bs=16, cache="bf16", ctx_range=(512, 4096),
+                          pool_factor=1.1, partition=512),
+    "long_context_b8": dict(B=8, h_q=32, h_kv=8, d=128, bs=16, cache="bf16",
+                            ctx_range=(32768, 131072), pool_factor=1.0, partition=512),
+    "shared_prefix_4x8": dict(prompts=4, samples=8, prompt_len=2048, tail_range=(0, 256), h_q=32,
+                              h_kv=8, d=128, bs=16, cache="bf16", partition=512),
+    "fp8_mha_b32_bs16": dict(B=32, h_q=32, h_kv=32, d=128, bs=16, cache="e4m3", ctx_fixed=4096,
+                             pool_factor=1.0, partition=512),
+    "fp8_mha_b32_bs32": dict(B=32, h_q=32, h_kv=32, d=128, bs=32, cache="e4m3", ctx_fixed=4096,
+                             pool_factor=1.0, partition=512),
+    "fp8_mha_b32_bs64": dict(B=32, h_q=32, h_kv=32, d=128, bs=64, cache="e4m3", ctx_fixed=4096,
+                             pool_factor=1.0, partition=512),
+}
+
+
+@dataclass
+class DecodeCase:
+    """One decode step of a batch: caches hold every token but the last of each sequence;
+    ``key_new``/``value_new`` are the appended tokens and ``slot_mapping`` their slots."""
+    name: str
+    B: int
+    h_q: int
+    h_kv: int
+    d: int
+    bs: int
+    num_blocks: int
+    cache: str                      # "bf16" or "e4m3"
+    partition: int
+    scale: float
+    q: torch.Tensor                 # bf16 [B, h_q, d]
+    key_new: torch.Tensor           # bf16 [B, h_kv, d]
+    value_new: torch.Tensor         # bf16 [B, h_kv, d]
+    slot_mapping: torch.Tensor      # int64 [B]
+    block_tables: torch.Tensor      # int32 [B, max_blocks]
+    context_lens: torch.Tensor      # int32 [B], including the appended token
+    # bf16 caches: filled directly [NB, h_kv, bs, d]; e4m3 caches: None (each side fills its
+    # own from fill_rows / fill_slots with its own quantiser)
+    k_cache: Optional[torch.Tensor] = None
+    v_cache: Optional[torch.Tensor] = None
+    fill_k_rows: Optional[torch.Tensor] = None   # bf16 [n_fill, h_kv, d]
+    fill_v_rows: Optional[torch.Tensor] = None
+    fill_slots: Optional[torch.Tensor] = None    # int64 [n_fill]
+    k_scale: float = 1.0
+    v_scale: float = 1.0
+    meta: dict = field(default_factory=dict)
+
+    @property
+    def max_context_len(self) -> int:
+        return int(self.context_lens.max().item()) if self.B else 0
+
+    @property
+    def elem_bytes(self) -> int:
+        return 1 if self.cache == "e4m3" else 2
+
+    def kv_bytes(self) -> int:
+        """K+V bytes the step must read: sum of ctx * h_kv * d * elem * 2."""
+        return int(self.context_lens.to(torch.int64).sum().item()) * self.h_kv * self.d * self.elem_bytes * 2
+
+
+def _gen(seed: int, device) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return g
+
+
+def _randn_bf16(shape, g, device) -> torch.Tensor:
+    return torch.randn(shape, generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+
+
+def _cpu_gen(seed: int) -> torch.Generator:
+    g = torch.Generator()
+    g.manual_seed(seed)
+    return g
+
+
+def _tables_from_order(order: list, blocks_per_seq: list, max_blocks: int) -> torch.Tensor:
+    """Hand consecutive ids of ``order`` to the sequences in turn; -1 pads each row."""
+    tab = torch.full((len(blocks_per_seq), max_blocks), -1, dtype=torch.int32)
+    pos = 0
+    for s, n in enumerate(blocks_per_seq):
+        tab[s, :n] = torch.tensor(order[pos:pos + n], dtype=torch.int32)
+        pos += n
+    return tab
+
+
+def _owned_slot_mask(tables: torch.Tensor, cached: torch.Tensor, num_blocks: int, bs: int) -> torch.Tensor:
+    """bool [num_blocks, bs]: True where a cached (pre-append) token lives."""
+    mask = torch.zeros(num_blocks, bs, dtype=torch.bool)
+    for s in range(tables.shape[0]):
+        n = int(cached[s])
+        full, rem = divmod(n, bs)
+        ids = tables[s, :full].to(torch.int64)
+        mask[ids] = True
+        if rem:
+            mask[int(tables[s, full]), :rem] = True
+    return mask
+
+
+def make_case(name: str, seed: int = 0, device="cpu", **over) -> DecodeCase:
+    """Build one workload.  ``over`` replaces any config entry (e.g. B=4 for a reduced case)."""
+    if name not in CONFIGS:
+        raise KeyError(name)
+    cfg = dict(CONFIGS[name])
+    cfg.update(over)
+    device = torch.device(device)
+    gc = _cpu_gen(seed)                    # structure (lengths, block order) always from the CPU stream
+
+    if name == "shared_prefix_4x8":
+        return _make_shared_prefix(name, cfg, seed, device, gc)
+
+    B, h_q, h_kv, d, bs = cfg["B"], cfg["h_q"], cfg["h_kv"], cfg["d"], cfg["bs"]
+    if "ctx_cached" in cfg:
+        cached = torch.tensor(cfg["ctx_cached"][:B], dtype=torch.int64)
+    elif "ctx_fixed" in cfg:
+        cached = torch.full((B,), cfg["ctx_fixed"] - 1, dtype=torch.int64)
+    else:
+        lo, hi = cfg["ctx_range"]
+        cached = torch.randint(lo, hi + 1, (B,), generator=gc, dtype=torch.int64) - 1
+    ctx = cached + 1
+    blocks_per_seq = [int(-(-int(c) // bs)) for c in ctx]
+    demand = sum(blocks_per_seq)
+    if "num_blocks" in cfg:
+        nb = cfg["num_blocks"]
+    else:
+        nb = int(math.ceil(cfg.get("pool_factor", 1.0) * demand))
+    if nb < demand:
+        raise ValueError("pool of %d blocks cannot hold %d" % (nb, demand))
+    max_blocks = max(blocks_per_seq) if blocks_per_seq else 1
+    order = torch.randperm(nb, generator=gc).tolist()
+    tables = _tables_from_order(order, blocks_per_seq, max_blocks)
+    slots = torch.tensor([int(tables[s, int(cached[s]) // bs]) * bs + int(cached[s]) % bs
+                          for s in range(B)], dtype=torch.int64)
+
+    g = _gen(seed, device)
+    q = _randn_bf16((B, h_q, d), g, device)
+    k_new = _randn_bf16((B, h_kv, d), g, device)
+    v_new = _randn_bf16((B, h_kv, d), g, device)
+    owned = _owned_slot_mask(tables, cached, nb, bs)
+
+    case = DecodeCase(name=name, B=B, h_q=h_q, h_kv=h_kv, d=d, bs=bs, num_blocks=nb, cache=cfg["cache"],
+                      partition=cfg["partition"], scale=1.0 / math.sqrt(d), q=q, key_new=k_new,
+                      value_new=v_new, slot_mapping=slots.to(device), block_tables=tables.to(device),
+                      context_lens=ctx.to(torch.int32).to(device),
+                      meta=dict(seed=seed, cached=cached.tolist()))
+    pool_k = _randn_bf16((nb, h_kv, bs, d), g, device)
+    pool_v = _randn_bf16((nb, h_kv, bs, d), g, device)
+    hole = (~owned).to(device)[:, None, :, None].expand(nb, h_kv, bs, d)
+    if cfg["cache"] == "bf16":
+        nan = torch.tensor(BF16_NAN, dtype=torch.int16).view(torch.bfloat16).to(device)
+        case.k_cache = torch.where(hole, nan, pool_k)
+        case.v_cache = torch.where(hole, nan, pool_v)
+    else:
+        # E4M3: each side quantises the owned rows itself (pool layout -> rows + slot ids).
+        ids = owned.reshape(-1).nonzero().flatten()                 # slot ids of owned tokens
+        blk, off = ids // bs, ids % bs
+        kr = pool_k.permute(0, 2, 1, 3)[blk.to(device), off.to(device)]   # [n, h_kv, d]
+        vr = pool_v.permute(0, 2, 1, 3)[blk.to(device), off.to(device)]
+        case.fill_k_rows, case.fill_v_rows = kr.contiguous(), vr.contiguous()
+        case.fill_slots = ids.to(torch.int64).to(device)
+        # per-tensor scale over every K (resp. V) value of the workload, appended tokens included
+        kmax = torch.maximum(kr.float().abs().max(), k_new.float().abs().max())
+        vmax = torch.maximum(vr.float().abs().max(), v_new.float().abs().max())
+        case.k_scale = float((kmax / 448.0).item())
+        case.v_scale = float((vmax / 448.0).item())
+    return case
+
+
+def empty_e4m3_pool(case: DecodeCase, device=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """Two uint8 pools [NB, h_kv, bs, d] filled with the E4M3 NaN sentinel."""
+    device = device if device is not None else case.q.device
+    shape = (case.num_blocks, case.h_kv, case.bs, case.d)
+    return (torch.full(shape, E4M3_NAN, dtype=torch.uint8, device=device),
+            torch.full(shape, E4M3_NAN, dtype=torch.uint8, device=device))
+
+
+def _make_shared_prefix(name, cfg, seed, device, gc) -> DecodeCase:
+    """P prompts of L tokens, S samples each; the samples' tables repeat the prompt's physical
+    ids (refcount S), then list private tail blocks.  L is block aligned, so tails start in
+    fresh blocks and the appended token lands in a private block."""
+    P, S, L = cfg["prompts"], cfg["samples"], cfg["prompt_len"]
+    h_q, h_kv, d, bs = cfg["h_q"], cfg["h_kv"], cfg["d"], cfg["bs"]
+    B = P * S
+    lo, hi = cfg["tail_range"]
+    tails = torch.randint(lo, hi + 1, (B,), generator=gc, dtype=torch.int64)
+    cached = L + tails                       # prompt + generated tail, before this step
+    ctx = cached + 1
+    pblocks = -(-L // bs)
+    private = [int(-(-int(c) // bs)) - pblocks for c in ctx]
+    nb = P * pblocks + sum(private)
+    order = torch.randperm(nb, generator=gc).tolist()
+    max_blocks = pblocks + max(private)
+    tables = torch.full((B, max_blocks), -1, dtype=torch.int32)
+    pos = P * pblocks
+    for p in range(P):
+        pids = torch.tensor(order[p * pblocks:(p + 1) * pblocks], dtype=torch.int32)
+        for j in range(S):
+            s = p * S + j
+            tables[s, :pblocks] = pids
+            n = private[s]
+            tables[s, pblocks:pblocks + n] = torch.tensor(order[pos:pos + n], dtype=torch.int32)
+            pos += n
+    slots = torch.tensor([int(tables[s, int(cached[s]) // bs]) * bs + int(cached[s]) % bs
+                          for s in range(B)], dtype=torch.int64)
+    owned = _owned_slot_mask(tables, cached, nb, bs)
+    g = _gen(seed, device)
+    q = _randn_bf16((B, h_q, d), g, device)
+    k_new = _randn_bf16((B, h_kv, d), g, device)
+    v_new = _randn_bf16((B, h_kv, d), g, device)
+    pool_k = _randn_bf16((nb, h_kv, bs, d), g, device)
+    pool_v = _randn_bf16((nb, h_kv, bs, d), g, device)
+    hole = (~owned).to(device)[:, None, :, None].expand(nb, h_kv, bs, d)
+    nan = torch.tensor(BF16_NAN, dtype=torch.int16).view(torch.bfloat16).to(device)
+    return DecodeCase(name=name, B=B, h_q=h_q, h_kv=h_kv, d=d, bs=bs, num_blocks=nb, cache="bf16",
+                      partition=cfg["partition"], scale=1.0 / math.sqrt(d), q=q, key_new=k_new,
+                      value_new=v_new, slot_mapping=slots.to(device), block_tables=tables.to(device),
+                      context_lens=ctx.to(torch.int32).to(device),
+                      k_cache=torch.where(hole, nan, pool_k), v_cache=torch.where(hole, nan, pool_v),
+                      meta=dict(seed=seed, cached=cached.tolist(), prompts=P, samples=S,
+                                prompt_blocks=pblocks, unique_tokens=P * L + int(tails.sum()) + B))
+
+
+def random_rows(n: int, h_kv: int, d: int, seed: int, device="cpu") -> tuple[torch.Tensor, torch.Tensor]:
+    """K and V rows ~ N(0,1) in bf16, [n, h_kv, d] each (for cache-write cases)."""
+    g = _gen(seed, torch.device(device))
+    return _randn_bf16((n, h_kv, d), g, device), _randn_bf16((n, h_kv, d), g, device)
