@@ -1,0 +1,449 @@
+#!/usr/bin/env python
+"""Benchmark of one paged decode step (cache write of the appended tokens + split-context
+decode attention + partition merge) on the llama3_8b_b64 workload: 64 sequences, 32 query /
+8 KV heads, head_dim 128, bf16 KV in 16-token blocks drawn shuffled from a pool sized to
+1.1x demand, contexts ~ U{512..4096}.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints ONE JSON line (rank 0).  `value` is KV GB/s of the whole job (algorithmic K+V bytes
+the step must read / device time of the step, CUDA events, inputs resident in HBM, L2
+flushed between steps).  `e2e` is the same metric through the binding's public calls with
+pinned host inputs copied in and the output copied back inside the timed region.
+`--impl reference` times the CPU oracle (the plain fp64 C implementation) on a bounded
+sample of the same workload, on the host cores.
+
+Multi-GPU (torchrun): weak scaling -- every rank runs its own batch of the same shape; the
+units are independent, so no collective touches the data path.  The step time is the max
+over ranks (device events), `value` the sum of all ranks' bytes over that time.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime as _dt
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "paged decode attention KV GB/s & % of B200 HBM peak; decode tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SOURCES = [os.path.join(ROOT, "paged_kv_cache_428_b200", "csrc", f) for f in ("decode.cuh", "common.cuh")]
+TRAFFIC_SUMMARY = os.path.join(ROOT, "profiles", "ncu_decode_partition_llama3_8b_b64.md")
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama3_8b_b64")
+    ap.add_argument("--partition", type=int, default=None, help="tokens per split-context partition")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args(argv)
+
+
+# ---------------------------------------------------------------------------------------- ranks
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world: int, backend: str):
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=_dt.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(values, world: int, device):
+    """Element-wise max over ranks (timing only; never on the data path)."""
+    import torch
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def sum_over_ranks(values, world: int, device):
+    import torch
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return t.tolist()
+
+
+def shard_seeds(seed: int, world: int):
+    """Each rank draws its own batch of the workload shape (weak scaling)."""
+    return [seed + 1000 * r for r in range(world)]
+
+
+# ------------------------------------------------------------------------------------- metrics
+def kv_bytes(case) -> int:
+    return case.kv_bytes()
+
+
+def partition_kernel_bytes(case) -> int:
+    """Algorithmic bytes of the partition pass: K+V of every context token (ctx*h_kv*d*b*2),
+    q (B*h_q*d*2), the block-table entries used (4 per block) and context_lens (4 per seq).
+    Split-context partials are implementation overhead and are not counted."""
+    ctx = case.context_lens.to("cpu").tolist()
+    blocks = sum(-(-c // case.bs) for c in ctx)
+    return kv_bytes(case) + case.B * case.h_q * case.d * 2 + 4 * blocks + 4 * case.B
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic_per_launch():
+    """DRAM bytes (read + write) of one partition-kernel launch from the committed ncu summary,
+    or None when the summary is missing or the kernel source changed since it was taken."""
+    if not os.path.exists(TRAFFIC_SUMMARY):
+        return None
+    text = open(TRAFFIC_SUMMARY).read()
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9]+)", text)
+    h = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
+    if not m or not h or h.group(1) != kernel_source_hash():
+        return None
+    return int(m.group(1))
+
+
+# -------------------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clock, power and throttle reasons in the background."""
+    QUERY = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", "clocks_%d.csv" % os.getpid())
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", gpu_id, "--query-gpu=" + self.QUERY,
+                                          "--format=csv,noheader,nounits", "-lms", "20"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self, t0: float, t1: float):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "note": "nvidia-smi unavailable"}
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                ts = _dt.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append((ts, float(parts[2]), float(parts[3]), parts[4], parts[6:10]))
+            except ValueError:
+                continue
+        inside = [r for r in rows if t0 <= r[0] <= t1]
+        window = "timed region"
+        if not inside and rows:                          # very short timed region: nearest samples
+            inside = sorted(rows, key=lambda r: min(abs(r[0] - t0), abs(r[0] - t1)))[:3]
+            window = "nearest to timed region"
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in inside for i in range(4) if r[4][i].lower().startswith("active")})
+        pw = [float(r[3]) for r in inside if re.match(r"^[0-9.]+$", r[3])]
+        return {"sm_mhz": statistics.median([r[1] for r in inside]) if inside else None,
+                "sm_max_mhz": max(r[2] for r in inside) if inside else None,
+                "reasons": reasons, "samples": len(inside), "window": window,
+                "power_w_max": max(pw) if pw else None}
+
+
+# ---------------------------------------------------------------------------------- our arm
+def run_ours(args):
+    import torch
+    import workloads
+    import paged_kv_cache_428_b200 as pa
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = init_dist(world, "nccl")
+    seed = shard_seeds(args.seed, world)[rank]
+    case = workloads.make_case(args.workload, seed, device=dev)
+    if case.cache == "e4m3":
+        raise SystemExit("bench.py times the bf16 workloads; E4M3 runs go through tests")
+    P = case.partition if args.partition is None else args.partition
+    B, h_q, d = case.B, case.h_q, case.d
+    mcl = case.max_context_len
+    kc, vc = case.k_cache, case.v_cache
+    q, k_new, v_new = case.q, case.key_new, case.value_new
+    slots, tables, ctx = case.slot_mapping, case.block_tables, case.context_lens
+    out = torch.empty((B, h_q, d), dtype=torch.bfloat16, device=dev)
+    ws = pa.make_workspace(B, h_q, d, mcl, P, dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(evs=None):
+        if evs:
+            evs[0].record(stream)
+        pa.pa_reshape_and_cache(k_new, v_new, kc, vc, slots, stream=stream)
+        if evs:
+            evs[1].record(stream)
+        pa.pa_decode_partitions(out, q, kc, vc, tables, ctx, mcl, case.scale, P, workspace=ws, stream=stream)
+        if evs:
+            evs[2].record(stream)
+        pa.pa_decode_merge(out, ctx, mcl, P, ws, stream=stream)
+        if evs:
+            evs[3].record(stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            flush.zero_()
+            step()
+    torch.cuda.synchronize(dev)
+
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+    time.sleep(0.3)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    t0 = time.time()
+    with torch.cuda.stream(stream):
+        for i in range(args.steps):
+            flush.zero_()                               # outside the events: L2 starts cold
+            step(evs[i])
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    t1 = time.time()
+    time.sleep(0.1)
+    sampler.stop()
+    clocks = sampler.summary(t0, t1)
+
+    step_ms = sum(e[0].elapsed_time(e[3]) for e in evs)
+    write_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
+    part_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
+    merge_ms = sum(e[2].elapsed_time(e[3]) for e in evs)
+
+    # end to end through the public calls: pinned host inputs in, result out, every step
+    e2e = None
+    if not args.no_e2e:
+        host = {n: t.cpu().pin_memory() for n, t in
+                (("q", q), ("k_new", k_new), ("v_new", v_new), ("slots", slots), ("tables", tables), ("ctx", ctx))}
+        dbuf = {n: torch.empty_like(t, device=dev) for n, t in host.items()}
+        out_host = torch.empty((B, h_q, d), dtype=torch.bfloat16).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = out_host.numel() * out_host.element_size()
+
+        def e2e_step():
+            for n in host:
+                dbuf[n].copy_(host[n], non_blocking=True)
+            pa.pa_reshape_and_cache(dbuf["k_new"], dbuf["v_new"], kc, vc, dbuf["slots"], stream=stream)
+            pa.pa_decode(out, dbuf["q"], kc, vc, dbuf["tables"], dbuf["ctx"], mcl, case.scale, P, workspace=ws,
+                         stream=stream)
+            out_host.copy_(out, non_blocking=True)
+
+        with torch.cuda.stream(stream):
+            for _ in range(args.warmup):
+                flush.zero_()
+                e2e_step()
+        torch.cuda.synchronize(dev)
+        eev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        with torch.cuda.stream(stream):
+            for i in range(args.steps):
+                flush.zero_()
+                eev[i][0].record(stream)
+                e2e_step()
+                eev[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = sum(a.elapsed_time(b) for a, b in eev)
+        e2e = {"ms": e2e_ms, "h2d": h2d, "d2h": d2h}
+
+    errs = pa.pa_device_errors(clear=True)
+    if errs:
+        raise SystemExit("device error bits 0x%x during the benchmark" % errs)
+
+    my_bytes = kv_bytes(case)
+    mx = max_over_ranks([step_ms, part_ms, merge_ms, write_ms, e2e["ms"] if e2e else 0.0], world, dev)
+    tot_bytes, tot_seqs = sum_over_ranks([float(my_bytes), float(B)], world, dev)
+    step_ms, part_ms, merge_ms, write_ms, e2e_ms = mx
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return None
+
+    K = args.steps
+    per_step_s = step_ms / 1e3 / K
+    value = tot_bytes / per_step_s / 1e9
+    peak, peak_kind = measured_peaks()
+    part_bytes = partition_kernel_bytes(case)
+    achieved = part_bytes / (part_ms / 1e3 / K) / 1e9
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(step_ms / K, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "num_seqs": B, "h_q": h_q, "h_kv": case.h_kv, "head_dim": d,
+                   "block_size": case.bs, "ctx": "U{512..4096} incl. appended token", "partition": P,
+                   "num_blocks": case.num_blocks, "kv_bytes_per_step_per_gpu": my_bytes,
+                   "step": "reshape_and_cache(64 new tokens) + decode partitions + merge",
+                   "l2": "flushed between steps (2x L2 write, outside the events)",
+                   "parallelism": "replicas (weak scaling, no collective)" if world > 1 else "single GPU"},
+        "tokens_per_s": round(tot_seqs / per_step_s, 1),
+        "pct_of_hbm_peak": round(value / world / peak, 4),
+        "pct_of_nominal_8tbs": round(value / world / 8000.0, 4),
+        "kernels_ms_per_step": {"reshape_and_cache": round(write_ms / K, 5),
+                                "decode_partitions": round(part_ms / K, 5),
+                                "decode_merge": round(merge_ms / K, 5)},
+        "roofline": {"bound": "hbm", "kernel": "paged_decode_partition_kernel", "achieved": round(achieved, 1),
+                     "peak": peak, "peak_kind": peak_kind + " (hbm_gbs copy bandwidth)", "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": ncu_traffic_per_launch(),
+                     "algorithmic_bytes_per_launch": part_bytes},
+        "gpu_launches": 3 * K,
+        "clocks": clocks,
+    }
+    if e2e:
+        line["e2e"] = {"value": round(tot_bytes / (e2e_ms / 1e3 / K) / 1e9, 2), "unit": "GB/s",
+                       "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                       "ms_per_step": round(e2e_ms / K, 5)}
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(case)
+    if world > 1:
+        dist.destroy_process_group()
+    return line
+
+
+def cpu_baseline(case):
+    """The oracle as it stands, single-threaded, on the host: the whole step (cache write of the
+    appended tokens and every (sequence, query head) row of the decode), once."""
+    import numpy as np
+    import torch
+    import oracle
+    orc = oracle.load()
+    u16 = lambda t: t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+    kc, vc = u16(case.k_cache).copy(), u16(case.v_cache).copy()
+    q, kn, vn = u16(case.q), u16(case.key_new), u16(case.value_new)
+    tab, ctx, sl = case.block_tables.cpu().numpy(), case.context_lens.cpu().numpy(), case.slot_mapping.cpu().numpy()
+    t0 = time.perf_counter()
+    orc.reshape_and_cache(kn, vn, kc, vc, sl, h_kv=case.h_kv, d=case.d, bs=case.bs, num_blocks=case.num_blocks)
+    orc.paged_decode(q, kc, vc, tab, ctx, h_kv=case.h_kv, bs=case.bs, scale=case.scale)
+    dt = time.perf_counter() - t0
+    return {"value": round(kv_bytes(case) / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "seconds": round(dt, 2), "host_cpus": os.cpu_count(),
+            "sample": "one full step of the workload (cache write of %d tokens + all %d x %d decode rows), "
+                      "single-threaded fp64 C" % (case.B, case.B, case.h_q)}
+
+
+# ---------------------------------------------------------------------------- reference arm
+def run_reference(args):
+    """The CPU oracle on the host cores, on a bounded sample of the same workload per step."""
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return None
+    import numpy as np
+    import torch
+    import oracle
+    import workloads
+    orc = oracle.load()
+    case = workloads.make_case(args.workload, args.seed)
+    u16 = lambda t: t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+    kc, vc = u16(case.k_cache).copy(), u16(case.v_cache).copy()
+    q, kn, vn = u16(case.q), u16(case.key_new), u16(case.value_new)
+    tab, ctx, sl = case.block_tables.numpy(), case.context_lens.numpy(), case.slot_mapping.numpy()
+    orc.reshape_and_cache(kn, vn, kc, vc, sl, h_kv=case.h_kv, d=case.d, bs=case.bs, num_blocks=case.num_blocks)
+    g = case.h_q // case.h_kv
+    all_rows = [(s, h) for s in range(case.B) for h in range(case.h_q)]
+    kw = dict(h_kv=case.h_kv, bs=case.bs, scale=case.scale)
+    t = time.perf_counter()
+    orc.paged_decode_rows(all_rows[:4], q, kc, vc, tab, ctx, **kw)
+    per_row = (time.perf_counter() - t) / 4
+    budget = 90.0 / max(1, args.steps + args.warmup)              # whole run within a few minutes
+    n_rows = int(max(1, min(len(all_rows), budget / max(per_row, 1e-6))))
+    pos = 0
+    row_bytes = lambda r: int(ctx[r[0]]) * case.d * 2 * 2 / g      # 1/g of the KV head's bytes
+
+    def take():
+        nonlocal pos
+        rows = [all_rows[(pos + i) % len(all_rows)] for i in range(n_rows)]
+        pos = (pos + n_rows) % len(all_rows)
+        return rows
+
+    for _ in range(args.warmup):
+        orc.paged_decode_rows(take(), q, kc, vc, tab, ctx, **kw)
+    tot_s, tot_b = 0.0, 0.0
+    for _ in range(args.steps):
+        rows = take()
+        t = time.perf_counter()
+        orc.paged_decode_rows(rows, q, kc, vc, tab, ctx, **kw)
+        tot_s += time.perf_counter() - t
+        tot_b += sum(row_bytes(r) for r in rows)
+    value = tot_b / tot_s / 1e9
+    sample = "%d of %d (sequence, query head) decode rows per step, rotating through the batch" % (n_rows, len(all_rows))
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 5), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(tot_s / args.steps * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "num_seqs": case.B, "h_q": case.h_q, "h_kv": case.h_kv,
+                       "head_dim": case.d, "block_size": case.bs, "ctx": "U{512..4096} incl. appended token"},
+            "cpu_baseline": {"value": round(value, 5), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 5), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    line = run_reference(args) if args.impl == "reference" else run_ours(args)
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

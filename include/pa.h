@@ -1,0 +1,214 @@
+/*
+ * pa.h -- C ABI of the B200 paged-KV decode library (libpa.so).
+ *
+ * Paged KV cache: the K and V of every sequence live in fixed-size physical
+ * blocks of a shared pool; a per-sequence block table maps logical block i to
+ * a physical block id, so a sequence's cache need not be contiguous.
+ * Sources (web pages), cited by title and section:
+ *   "深度解构 LLM 推理优化：从 KV Cache 冗余到 PagedAttention 内存分页映射"
+ *       section 2.1 (block table), 2.2 (on-demand allocation from a global
+ *       free pool), 2.3 (copy-on-write for shared prompts), 3.2 (FP8 KV)
+ *   "现代 AI 的“推理加速之谜”：从 KV Cache 到 PagedAttention 的演进"
+ *       section 1 (Attention(Q,K,V) = softmax(QK^T / sqrt(d_k)) V; only the
+ *       new token's Q, K, V are computed each step), section 3.A (GQA)
+ *   "KVCache技术背景与核心挑战 / PageAttention内存管理机制" (intelliparadigm)
+ *       sections 2.1-2.2 (blocks with reference counts), 3.1 (copy-on-write)
+ *   "vLLM 推理原理 从 KV Cache 到分页与连续批处理"
+ *       section "PagedAttention 怎样整理这些缓存" (logical blocks -> physical
+ *       blocks 2, 5, 1; the last block may be partly filled)
+ *
+ * Conventions for every call below
+ *   - Device pointers are owned by the caller (e.g. allocated through
+ *     PyTorch).  The library allocates no device memory: pa_decode takes a
+ *     caller workspace sized by pa_decode_workspace_size.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Device calls only enqueue work; none synchronises.
+ *   - Return value: PA_OK (0) or a negative PA_ERR_* code; nothing is
+ *     launched when an argument check fails.  No exception crosses the ABI.
+ *   - Cache layout: k_cache and v_cache are [num_blocks][h_kv][block_size]
+ *     [head_dim], row-major; each (block, head) tile is one contiguous span
+ *     of block_size*head_dim elements.  Elements are bf16 (PA_CACHE_BF16) or
+ *     OCP FP8 E4M3 bytes (PA_CACHE_E4M3) dequantised as code * scale with one
+ *     fp32 scale per tensor.
+ *   - Supported shapes: head_dim in {64, 128}; block_size in {16, 32, 64};
+ *     h_q / h_kv in {1, 2, 4, 8}.  Query head h reads KV head
+ *     h / (h_q / h_kv) (contiguous groups).
+ *   - Device-side guards: an out-of-range slot, block id or block pair is
+ *     never dereferenced; the kernel skips it and records a bit in the
+ *     device error word (pa_device_errors).  Every wait inside a kernel is
+ *     bounded; a wait that runs out records PA_DEVERR_TIMEOUT.
+ */
+#ifndef PA_H
+#define PA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------ */
+#define PA_OK               0
+#define PA_ERR_INVALID_ARG (-1)   /* null pointer, bad size, h_q % h_kv != 0, bad dtype ... */
+#define PA_ERR_UNSUPPORTED (-2)   /* shape outside the supported set */
+#define PA_ERR_WORKSPACE   (-3)   /* workspace missing or too small */
+#define PA_ERR_OOM         (-4)   /* allocator: free pool cannot satisfy the request */
+#define PA_ERR_CUDA        (-5)   /* a CUDA call or launch failed */
+#define PA_ERR_NOT_FOUND   (-6)   /* allocator: unknown sequence id */
+
+/* device error word bits (pa_device_errors) */
+#define PA_DEVERR_BAD_SLOT  0x1u  /* a slot id outside the pool was skipped */
+#define PA_DEVERR_BAD_BLOCK 0x2u  /* a block-table entry outside the pool (or row) was skipped */
+#define PA_DEVERR_BAD_PAIR  0x4u  /* a copy pair outside the pool was skipped */
+#define PA_DEVERR_TIMEOUT   0x8u  /* a bounded in-kernel wait ran out */
+
+typedef enum { PA_CACHE_BF16 = 0, PA_CACHE_E4M3 = 1 } pa_cache_dtype;
+
+/* Human-readable text of a status code (static storage). */
+const char *pa_status_str(int status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int pa_version(void);
+
+/* KV bytes per cached token: 2 (K and V) x layers x h_kv x head_dim x
+ * elem_bytes ("深度解构…" section 1.1, per-token memory equation; "vLLM 推理原理…"
+ * M_KV estimate).  Host only. */
+size_t pa_kv_bytes_per_token(int layers, int h_kv, int head_dim, int elem_bytes);
+
+/* ---- cache write --------------------------------------------------------
+ * Store the step's new K and V rows in their physical slots: for token t and
+ * KV head h, cache[slot/bs][h][slot%bs][:] = row[t][h][:]
+ * ("现代 AI…" section 1: each step computes only the new token's K, V and
+ * keeps them; "vLLM 推理原理…" section "KV Cache 缓存的究竟是什么").
+ *   key, value     device bf16; row t, head h at key + t*key_stride + h*head_dim
+ *                  (key_stride/value_stride in elements; 0 = packed h_kv*head_dim)
+ *   k_cache/v_cache device, layout above, of cache_dtype
+ *   slot_mapping   device int64 [num_tokens]; slot = block*block_size + offset;
+ *                  a negative slot skips the token (padding); a slot past the
+ *                  pool is skipped and flags PA_DEVERR_BAD_SLOT
+ *   cache_dtype    PA_CACHE_BF16: bits are copied unchanged.
+ *                  PA_CACHE_E4M3: code = RNE-satfinite(x / scale) with an IEEE
+ *                  fp32 division ("深度解构…" section 3.2, FP8 KV cache)
+ *   k_scale/v_scale per-tensor fp32 scales (E4M3 only; must be > 0 and finite)
+ * Bit-exact by construction: no arithmetic other than the quantisation. */
+int pa_reshape_and_cache(const void *key, const void *value, int64_t key_stride, int64_t value_stride,
+                         void *k_cache, void *v_cache, const int64_t *slot_mapping, int num_tokens,
+                         int h_kv, int head_dim, int block_size, int num_blocks,
+                         int cache_dtype, float k_scale, float v_scale, void *stream);
+
+/* ---- decode attention ----------------------------------------------------
+ * One decode step: for sequence s and query head h,
+ *   out[s][h] = softmax(scale * q[s][h] . K_s^T) . V_s
+ * over the first context_lens[s] tokens of sequence s, token t read from
+ * physical block block_tables[s][t / bs] at offset t % bs
+ * ("现代 AI…" section 1, attention formula; "深度解构…" section 2.1 and
+ * "vLLM 推理原理…" section "PagedAttention 怎样整理这些缓存", block table).
+ * context_lens[s] includes the token written this step; 0 gives a zero row.
+ *
+ * Long contexts are split into partitions of partition_size tokens; each
+ * partition keeps its own running max, sum and unnormalised output and a
+ * second pass merges them (split-context decode).  partition_size = 0 means
+ * one partition per sequence; otherwise it must be a multiple of block_size.
+ *   out            device bf16 [num_seqs][h_q][head_dim] (RNE of the fp32 result)
+ *   q              device bf16 [num_seqs][h_q][head_dim]
+ *   block_tables   device int32 [num_seqs][max_blocks_per_seq]; entries past
+ *                  ceil(ctx/bs) are never read
+ *   context_lens   device int32 [num_seqs]
+ *   max_context_len host-known upper bound of context_lens; it only sizes the
+ *                  grid (no device->host read).  A longer context is still
+ *                  computed correctly: its last partition grows.
+ *   workspace      device, >= pa_decode_workspace_size(...) bytes, 16-byte
+ *                  aligned; holds fp32 partials; may be NULL when that size is 0
+ * Accuracy: fp32 accumulation; vs an fp64 evaluation of the same formula,
+ * max|err| <= 2e-2 and <= 1e-2 * max|ref| for bf16 caches, <= 6e-2 for E4M3. */
+size_t pa_decode_workspace_size(int num_seqs, int h_q, int head_dim, int max_context_len,
+                                int partition_size);
+
+int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
+              const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
+              int num_seqs, int max_context_len, int h_q, int h_kv, int head_dim, int block_size,
+              int num_blocks, float scale, int cache_dtype, float k_scale, float v_scale,
+              int partition_size, void *workspace, size_t workspace_bytes, void *stream);
+
+/* The two passes of pa_decode as separate launches (same arguments), so that
+ * each can be timed on its own: pa_decode == pa_decode_partitions followed by
+ * pa_decode_merge on the same stream.  Sequences that fit one partition are
+ * finished by the first pass; the merge pass combines the others. */
+int pa_decode_partitions(void *out, const void *q, const void *k_cache, const void *v_cache,
+                         const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
+                         int num_seqs, int max_context_len, int h_q, int h_kv, int head_dim,
+                         int block_size, int num_blocks, float scale, int cache_dtype, float k_scale,
+                         float v_scale, int partition_size, void *workspace, size_t workspace_bytes,
+                         void *stream);
+
+int pa_decode_merge(void *out, const int32_t *context_lens, int num_seqs, int max_context_len, int h_q,
+                    int head_dim, int partition_size, const void *workspace, size_t workspace_bytes,
+                    void *stream);
+
+/* ---- copy-on-write block copy ---------------------------------------------
+ * For every pair (src, dst) and every layer: cache[dst] = cache[src], byte
+ * for byte, for K and for V ("深度解构…" section 2.3; intelliparadigm section
+ * 3.1: copy the shared block, then remap the writer's table).
+ *   k_caches/v_caches host arrays of num_layers device pointers (<= 256)
+ *   block_pairs     device int64 [num_pairs][2] = (src, dst); a pair outside
+ *                   [0, num_blocks) is skipped and flags PA_DEVERR_BAD_PAIR
+ *   block_bytes     bytes of one physical block of one layer
+ *                   (h_kv*block_size*head_dim*elem); a multiple of 16 */
+int pa_copy_blocks(void *const *k_caches, void *const *v_caches, int num_layers,
+                   const int64_t *block_pairs, int num_pairs, size_t block_bytes, int num_blocks,
+                   void *stream);
+
+/* ---- device error word ------------------------------------------------------
+ * Read (and optionally clear) the error bits the kernels recorded on the
+ * current device.  SYNCHRONISES the device first.  Diagnostic use only. */
+int pa_device_errors(unsigned int *flags, int clear);
+
+/* ---- host-side validation (optional, before a launch) -------------------------
+ * Host copies of the tables / slots: PA_OK or PA_ERR_INVALID_ARG. */
+int pa_validate_block_tables(const int32_t *block_tables, int max_blocks_per_seq,
+                             const int32_t *context_lens, int num_seqs, int block_size, int num_blocks);
+int pa_validate_slots(const int64_t *slot_mapping, int num_tokens, int block_size, int num_blocks);
+
+/* ---- host block allocator -----------------------------------------------------
+ * A global free pool of num_blocks physical blocks with a reference count per
+ * block; sequences own block lists ("深度解构…" sections 2.1-2.3;
+ * intelliparadigm sections 2.1, 2.2, 3.1; "vLLM 推理原理…" generation flow:
+ * release a finished request's blocks).  Policy: LIFO free pool, initial
+ * order a Fisher-Yates shuffle by SplitMix64(seed) (seed 0 = identity); a
+ * block is taken only when the previous one is full; fork shares all blocks
+ * (refcount + 1); the first write into a partly filled block whose refcount
+ * is > 1 takes a fresh block, reports (old, new) for pa_copy_blocks and
+ * drops the old block's count (the last holder writes in place); freeing a
+ * sequence returns blocks whose count reaches 0, last block first.
+ * Failures leave the state unchanged.  Not thread-safe: one caller at a time. */
+typedef struct pa_alloc pa_alloc;
+
+pa_alloc *pa_alloc_create(int num_blocks, int block_size, uint64_t seed);   /* NULL on bad args */
+void      pa_alloc_destroy(pa_alloc *a);
+int  pa_alloc_new_seq(pa_alloc *a, int64_t *seq_id);
+/* One token: its slot, and (cow_src, cow_dst) = (-1, -1) unless a copy is needed. */
+int  pa_alloc_append_slot(pa_alloc *a, int64_t seq, int64_t *slot, int64_t *cow_src, int64_t *cow_dst);
+/* n tokens (prefill-style growth); slots may be NULL, else n entries.  At most one
+ * copy can be needed (the first, partly filled block). */
+int  pa_alloc_append_n(pa_alloc *a, int64_t seq, int n, int64_t *slots, int64_t *cow_src, int64_t *cow_dst);
+/* One token for each of n sequences, in order (a decode step).  slots: n entries;
+ * cow_pairs: room for 2*n int64; *num_cow receives the number of pairs.  All or nothing. */
+int  pa_alloc_append_batch(pa_alloc *a, const int64_t *seqs, int n, int64_t *slots,
+                           int64_t *cow_pairs, int *num_cow);
+int  pa_alloc_fork(pa_alloc *a, int64_t parent, int64_t *child);
+int  pa_alloc_free_seq(pa_alloc *a, int64_t seq);
+/* Host rows [num_seqs][max_blocks] (unused entries -1) and lengths. */
+int  pa_alloc_block_table(const pa_alloc *a, const int64_t *seqs, int num_seqs, int32_t *table,
+                          int max_blocks, int32_t *context_lens);
+int  pa_alloc_seq_len(const pa_alloc *a, int64_t seq, int64_t *len);
+int  pa_alloc_stats(const pa_alloc *a, int *free_blocks, int *used_blocks, int *shared_blocks,
+                    int64_t *frag_tokens);
+/* Reference count of a block (>= 0), or PA_ERR_INVALID_ARG. */
+int  pa_alloc_refcount(const pa_alloc *a, int block);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H */

@@ -1,0 +1,368 @@
+"""B200-native paged-KV decode attention: Python binding of libpa.so (include/pa.h).
+
+The binding only marshals arguments: it checks dtypes, shapes, devices and
+contiguity of torch tensors, passes raw pointers and the current CUDA stream
+to the C ABI, and raises :class:`PagedKVError` on a non-zero status.  Every
+step of the computation runs in the library's CUDA kernels; there is no CPU
+path.  Importing this package fails if libpa.so has not been built
+(``python paged_kv_cache_428_b200/build.py``).
+
+Functions keep the C names:
+
+* :func:`pa_reshape_and_cache` -- write the step's new K/V rows into their slots
+* :func:`pa_decode` -- split-context decode attention through the block table
+  (= :func:`pa_decode_partitions` + :func:`pa_decode_merge`)
+* :func:`pa_copy_blocks` -- copy-on-write block copy over all layers
+* :class:`BlockAllocator` -- the host block allocator (free pool, refcounts,
+  fork, copy-on-write decisions) that builds block tables and slot ids
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+from pathlib import Path
+from typing import Optional, Sequence
+
+import torch
+
+_PKG = Path(__file__).resolve().parent
+LIB_PATH = _PKG / "libpa.so"
+
+PA_CACHE_BF16 = 0
+PA_CACHE_E4M3 = 1
+PA_DEVERR_BAD_SLOT = 0x1
+PA_DEVERR_BAD_BLOCK = 0x2
+PA_DEVERR_BAD_PAIR = 0x4
+PA_DEVERR_TIMEOUT = 0x8
+
+STATUS = {0: "PA_OK", -1: "PA_ERR_INVALID_ARG", -2: "PA_ERR_UNSUPPORTED", -3: "PA_ERR_WORKSPACE",
+          -4: "PA_ERR_OOM", -5: "PA_ERR_CUDA", -6: "PA_ERR_NOT_FOUND"}
+
+
+class PagedKVError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__("%s: %s (%s)" % (what, STATUS.get(status, status), _lib.pa_status_str(status).decode()))
+
+
+def _load() -> ctypes.CDLL:
+    if not LIB_PATH.exists():
+        raise ImportError("libpa.so is not built; run `python paged_kv_cache_428_b200/build.py` "
+                          "(there is no fallback implementation)")
+    L = ctypes.CDLL(str(LIB_PATH))
+    vp, i32, i64, f32, sz, u64 = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float,
+                                  ctypes.c_size_t, ctypes.c_uint64)
+    P64 = ctypes.POINTER(ctypes.c_int64)
+    P32 = ctypes.POINTER(ctypes.c_int32)
+    PI = ctypes.POINTER(ctypes.c_int)
+    sig = {
+        "pa_status_str": (ctypes.c_char_p, [i32]),
+        "pa_version": (i32, []),
+        "pa_kv_bytes_per_token": (sz, [i32, i32, i32, i32]),
+        "pa_reshape_and_cache": (i32, [vp, vp, i64, i64, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, f32, vp]),
+        "pa_decode_workspace_size": (sz, [i32, i32, i32, i32, i32]),
+        "pa_decode": (i32, [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32, i32, i32, f32, i32, f32, f32,
+                            i32, vp, sz, vp]),
+        "pa_decode_partitions": (i32, [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32, i32, i32, f32, i32,
+                                       f32, f32, i32, vp, sz, vp]),
+        "pa_decode_merge": (i32, [vp, vp, i32, i32, i32, i32, i32, vp, sz, vp]),
+        "pa_copy_blocks": (i32, [vp, vp, i32, vp, i32, sz, i32, vp]),
+        "pa_device_errors": (i32, [ctypes.POINTER(ctypes.c_uint), i32]),
+        "pa_validate_block_tables": (i32, [vp, i32, vp, i32, i32, i32]),
+        "pa_validate_slots": (i32, [vp, i32, i32, i32]),
+        "pa_alloc_create": (vp, [i32, i32, u64]),
+        "pa_alloc_destroy": (None, [vp]),
+        "pa_alloc_new_seq": (i32, [vp, P64]),
+        "pa_alloc_append_slot": (i32, [vp, i64, P64, P64, P64]),
+        "pa_alloc_append_n": (i32, [vp, i64, i32, vp, P64, P64]),
+        "pa_alloc_append_batch": (i32, [vp, vp, i32, vp, vp, PI]),
+        "pa_alloc_fork": (i32, [vp, i64, P64]),
+        "pa_alloc_free_seq": (i32, [vp, i64]),
+        "pa_alloc_block_table": (i32, [vp, vp, i32, vp, i32, vp]),
+        "pa_alloc_seq_len": (i32, [vp, i64, P64]),
+        "pa_alloc_stats": (i32, [vp, PI, PI, PI, P64]),
+        "pa_alloc_refcount": (i32, [vp, i32]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    return L
+
+
+_lib = _load()
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libpa.so (ctypes handle)."""
+    return _lib
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != 0:
+        raise PagedKVError(rc, what)
+
+
+def _stream_ptr(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _need(t: torch.Tensor, name: str, dtypes, ndim: Optional[int] = None, cuda: bool = True) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s must be a torch.Tensor" % name)
+    if t.dtype not in dtypes:
+        raise TypeError("%s: dtype %s, expected one of %s" % (name, t.dtype, dtypes))
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError("%s: expected %d dims, got shape %s" % (name, ndim, tuple(t.shape)))
+    if cuda and not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+
+
+def cache_dtype_code(cache: torch.Tensor) -> int:
+    if cache.dtype == torch.bfloat16:
+        return PA_CACHE_BF16
+    if cache.dtype in (torch.uint8, torch.float8_e4m3fn):
+        return PA_CACHE_E4M3
+    raise TypeError("cache dtype must be bfloat16, uint8 or float8_e4m3fn (E4M3 codes), got %s" % cache.dtype)
+
+
+# ----------------------------------------------------------------------------------------------
+def pa_kv_bytes_per_token(layers: int, h_kv: int, head_dim: int, elem_bytes: int) -> int:
+    return int(_lib.pa_kv_bytes_per_token(layers, h_kv, head_dim, elem_bytes))
+
+
+def pa_version() -> int:
+    return int(_lib.pa_version())
+
+
+def pa_status_str(status: int) -> str:
+    return _lib.pa_status_str(status).decode()
+
+
+def pa_reshape_and_cache(key: torch.Tensor, value: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                         slot_mapping: torch.Tensor, k_scale: float = 1.0, v_scale: float = 1.0,
+                         stream=None) -> None:
+    """key/value bf16 [T, h_kv, d] (rows may be strided in dim 0); caches [NB, h_kv, bs, d]."""
+    for t, n in ((key, "key"), (value, "value")):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or t.dim() != 3 or t.stride(2) != 1 or t.stride(1) != t.shape[2]:
+            raise ValueError("%s must be a CUDA bf16 [T, h_kv, d] tensor with packed heads" % n)
+    _need(k_cache, "k_cache", (torch.bfloat16, torch.uint8, torch.float8_e4m3fn), 4)
+    _need(v_cache, "v_cache", (k_cache.dtype,), 4)
+    _need(slot_mapping, "slot_mapping", (torch.int64,), 1)
+    T, h_kv, d = key.shape
+    NB, h2, bs, d2 = k_cache.shape
+    if h2 != h_kv or d2 != d or tuple(v_cache.shape) != tuple(k_cache.shape) or value.shape != key.shape \
+            or slot_mapping.shape[0] != T:
+        raise ValueError("shape mismatch between key/value, caches and slot_mapping")
+    rc = _lib.pa_reshape_and_cache(key.data_ptr(), value.data_ptr(), key.stride(0), value.stride(0),
+                                   k_cache.data_ptr(), v_cache.data_ptr(), slot_mapping.data_ptr(), T, h_kv, d, bs,
+                                   NB, cache_dtype_code(k_cache), float(k_scale), float(v_scale),
+                                   _stream_ptr(stream))
+    _check(rc, "pa_reshape_and_cache")
+
+
+def pa_decode_workspace_size(num_seqs: int, h_q: int, head_dim: int, max_context_len: int,
+                             partition_size: int) -> int:
+    return int(_lib.pa_decode_workspace_size(num_seqs, h_q, head_dim, max_context_len, partition_size))
+
+
+def make_workspace(num_seqs: int, h_q: int, head_dim: int, max_context_len: int, partition_size: int,
+                   device="cuda") -> torch.Tensor:
+    """A caller-owned workspace of the size pa_decode needs (uint8, possibly empty)."""
+    n = pa_decode_workspace_size(num_seqs, h_q, head_dim, max_context_len, partition_size)
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=device)
+
+
+def _decode_args(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len, scale, partition_size,
+                 k_scale, v_scale, workspace):
+    _need(out, "out", (torch.bfloat16,), 3)
+    _need(q, "q", (torch.bfloat16,), 3)
+    _need(k_cache, "k_cache", (torch.bfloat16, torch.uint8, torch.float8_e4m3fn), 4)
+    _need(v_cache, "v_cache", (k_cache.dtype,), 4)
+    _need(block_tables, "block_tables", (torch.int32,), 2)
+    _need(context_lens, "context_lens", (torch.int32,), 1)
+    B, h_q, d = q.shape
+    NB, h_kv, bs, d2 = k_cache.shape
+    if tuple(out.shape) != (B, h_q, d) or d2 != d or tuple(v_cache.shape) != tuple(k_cache.shape) \
+            or block_tables.shape[0] != B or context_lens.shape[0] != B:
+        raise ValueError("shape mismatch between out, q, caches, block_tables and context_lens")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    ws_ptr, ws_bytes = 0, 0
+    if workspace is not None:
+        _need(workspace, "workspace", (torch.uint8,), 1)
+        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel()
+    return (out.data_ptr(), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_tables.data_ptr(),
+            block_tables.shape[1], context_lens.data_ptr(), B, int(max_context_len), h_q, h_kv, d, bs, NB,
+            float(scale), cache_dtype_code(k_cache), float(k_scale), float(v_scale), int(partition_size),
+            ws_ptr, ws_bytes)
+
+
+def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len: int, scale: float = None,
+              partition_size: int = 512, k_scale: float = 1.0, v_scale: float = 1.0,
+              workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """out[s, h] = softmax(scale * q[s, h] . K^T) . V over the paged cache; returns out."""
+    if workspace is None:
+        workspace = make_workspace(q.shape[0], q.shape[1], q.shape[2], max_context_len, partition_size, q.device)
+    args = _decode_args(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len, scale,
+                        partition_size, k_scale, v_scale, workspace)
+    _check(_lib.pa_decode(*args, _stream_ptr(stream)), "pa_decode")
+    return out
+
+
+def pa_decode_partitions(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len: int,
+                         scale: float = None, partition_size: int = 512, k_scale: float = 1.0,
+                         v_scale: float = 1.0, workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+    args = _decode_args(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len, scale,
+                        partition_size, k_scale, v_scale, workspace)
+    _check(_lib.pa_decode_partitions(*args, _stream_ptr(stream)), "pa_decode_partitions")
+
+
+def pa_decode_merge(out, context_lens, max_context_len: int, partition_size: int,
+                    workspace: Optional[torch.Tensor], stream=None) -> None:
+    _need(out, "out", (torch.bfloat16,), 3)
+    _need(context_lens, "context_lens", (torch.int32,), 1)
+    B, h_q, d = out.shape
+    ws_ptr, ws_bytes = (workspace.data_ptr(), workspace.numel()) if workspace is not None else (0, 0)
+    _check(_lib.pa_decode_merge(out.data_ptr(), context_lens.data_ptr(), B, int(max_context_len), h_q, d,
+                                int(partition_size), ws_ptr, ws_bytes, _stream_ptr(stream)), "pa_decode_merge")
+
+
+def pa_copy_blocks(k_caches: Sequence[torch.Tensor], v_caches: Sequence[torch.Tensor], block_pairs: torch.Tensor,
+                   stream=None) -> None:
+    """block_pairs int64 [n, 2] (src, dst) on the device; every layer's K and V block is copied."""
+    if len(k_caches) != len(v_caches) or len(k_caches) == 0:
+        raise ValueError("need the same, non-zero number of K and V caches")
+    ref = k_caches[0]
+    for t in list(k_caches) + list(v_caches):
+        _need(t, "cache", (ref.dtype,), 4)
+        if tuple(t.shape) != tuple(ref.shape):
+            raise ValueError("all caches must have the same shape")
+    _need(block_pairs, "block_pairs", (torch.int64,), 2)
+    if block_pairs.shape[1] != 2:
+        raise ValueError("block_pairs must be [n, 2]")
+    L = len(k_caches)
+    kp = (ctypes.c_void_p * L)(*[t.data_ptr() for t in k_caches])
+    vp = (ctypes.c_void_p * L)(*[t.data_ptr() for t in v_caches])
+    block_bytes = ref[0].numel() * ref.element_size()
+    _check(_lib.pa_copy_blocks(ctypes.cast(kp, ctypes.c_void_p), ctypes.cast(vp, ctypes.c_void_p), L,
+                               block_pairs.data_ptr(), block_pairs.shape[0], block_bytes, ref.shape[0],
+                               _stream_ptr(stream)), "pa_copy_blocks")
+
+
+def pa_device_errors(clear: bool = True) -> int:
+    """Error bits the kernels recorded on the current device (synchronises the device)."""
+    v = ctypes.c_uint(0)
+    _check(_lib.pa_device_errors(ctypes.byref(v), int(clear)), "pa_device_errors")
+    return int(v.value)
+
+
+def pa_validate_block_tables(block_tables: torch.Tensor, context_lens: torch.Tensor, block_size: int,
+                             num_blocks: int) -> int:
+    """Host copies (CPU int32 tensors); returns the status code."""
+    bt = block_tables.to("cpu", torch.int32).contiguous()
+    cl = context_lens.to("cpu", torch.int32).contiguous()
+    return int(_lib.pa_validate_block_tables(bt.data_ptr(), bt.shape[1], cl.data_ptr(), bt.shape[0], block_size,
+                                             num_blocks))
+
+
+def pa_validate_slots(slot_mapping: torch.Tensor, block_size: int, num_blocks: int) -> int:
+    sm = slot_mapping.to("cpu", torch.int64).contiguous()
+    return int(_lib.pa_validate_slots(sm.data_ptr(), sm.numel(), block_size, num_blocks))
+
+
+# ----------------------------------------------------------------------------------------------
+class BlockAllocator:
+    """Host block allocator (pa_alloc_* in pa.h): global free pool, per-block refcounts,
+    per-sequence block lists, fork, copy-on-write decisions, release."""
+
+    def __init__(self, num_blocks: int, block_size: int, seed: int = 0):
+        self._h = _lib.pa_alloc_create(num_blocks, block_size, seed)
+        if not self._h:
+            raise PagedKVError(-1, "pa_alloc_create")
+        self.num_blocks = num_blocks
+        self.block_size = block_size
+
+    def close(self) -> None:
+        if self._h:
+            _lib.pa_alloc_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def new_seq(self) -> int:
+        sid = ctypes.c_int64()
+        _check(_lib.pa_alloc_new_seq(self._h, ctypes.byref(sid)), "pa_alloc_new_seq")
+        return sid.value
+
+    def append_slot(self, seq: int):
+        """Returns (slot, (cow_src, cow_dst)); (-1, -1) when no copy is needed."""
+        slot, s, d = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
+        _check(_lib.pa_alloc_append_slot(self._h, seq, ctypes.byref(slot), ctypes.byref(s), ctypes.byref(d)),
+               "pa_alloc_append_slot")
+        return slot.value, (s.value, d.value)
+
+    def append_n(self, seq: int, n: int):
+        slots = (ctypes.c_int64 * max(n, 1))()
+        s, d = ctypes.c_int64(), ctypes.c_int64()
+        _check(_lib.pa_alloc_append_n(self._h, seq, n, ctypes.cast(slots, ctypes.c_void_p), ctypes.byref(s),
+                                      ctypes.byref(d)), "pa_alloc_append_n")
+        return list(slots)[:n], (s.value, d.value)
+
+    def append_batch(self, seqs: Sequence[int]):
+        """One token for each sequence (a decode step): (slots, [(src, dst), ...])."""
+        n = len(seqs)
+        sq = (ctypes.c_int64 * max(n, 1))(*seqs)
+        slots = (ctypes.c_int64 * max(n, 1))()
+        pairs = (ctypes.c_int64 * max(2 * n, 2))()
+        ncow = ctypes.c_int()
+        _check(_lib.pa_alloc_append_batch(self._h, ctypes.cast(sq, ctypes.c_void_p), n,
+                                          ctypes.cast(slots, ctypes.c_void_p), ctypes.cast(pairs, ctypes.c_void_p),
+                                          ctypes.byref(ncow)), "pa_alloc_append_batch")
+        return list(slots)[:n], [(pairs[2 * i], pairs[2 * i + 1]) for i in range(ncow.value)]
+
+    def fork(self, parent: int) -> int:
+        c = ctypes.c_int64()
+        _check(_lib.pa_alloc_fork(self._h, parent, ctypes.byref(c)), "pa_alloc_fork")
+        return c.value
+
+    def free_seq(self, seq: int) -> None:
+        _check(_lib.pa_alloc_free_seq(self._h, seq), "pa_alloc_free_seq")
+
+    def block_table(self, seqs: Sequence[int], max_blocks: int):
+        """(table int32 [n, max_blocks] with -1 padding, context_lens int32 [n]) as CPU tensors."""
+        n = len(seqs)
+        sq = torch.tensor(list(seqs), dtype=torch.int64)
+        table = torch.empty((n, max_blocks), dtype=torch.int32)
+        lens = torch.empty((n,), dtype=torch.int32)
+        _check(_lib.pa_alloc_block_table(self._h, sq.data_ptr(), n, table.data_ptr(), max_blocks, lens.data_ptr()),
+               "pa_alloc_block_table")
+        return table, lens
+
+    def seq_len(self, seq: int) -> int:
+        n = ctypes.c_int64()
+        _check(_lib.pa_alloc_seq_len(self._h, seq, ctypes.byref(n)), "pa_alloc_seq_len")
+        return n.value
+
+    def stats(self) -> dict:
+        f, u, s = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+        fr = ctypes.c_int64()
+        _check(_lib.pa_alloc_stats(self._h, ctypes.byref(f), ctypes.byref(u), ctypes.byref(s), ctypes.byref(fr)),
+               "pa_alloc_stats")
+        return {"free": f.value, "used": u.value, "shared": s.value, "frag_tokens": fr.value}
+
+    def refcount(self, block: int) -> int:
+        rc = _lib.pa_alloc_refcount(self._h, block)
+        if rc < 0:
+            raise PagedKVError(rc, "pa_alloc_refcount")
+        return rc

@@ -1,0 +1,306 @@
+// pa_lib.cu -- C-ABI entry points of the device calls (argument checks, dispatch, launch).
+// All device code of the library is in this one translation unit.
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+
+#include "common.cuh"
+#include "cache_ops.cuh"
+#include "decode.cuh"
+
+using namespace pa;
+
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int launch_status()
+{
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+bool supported_head_dim(int d) { return d == 64 || d == 128; }
+bool supported_block_size(int bs) { return bs == 16 || bs == 32 || bs == 64; }
+bool supported_group(int g) { return g == 1 || g == 2 || g == 4 || g == 8; }
+
+int grid_partitions(int max_context_len, int partition_size)
+{
+    if (partition_size <= 0) return 1;
+    const long long n = ((long long)max_context_len + partition_size - 1) / partition_size;
+    return n < 1 ? 1 : static_cast<int>(n);
+}
+
+size_t ml_bytes(int num_seqs, int h_q, int p_max)
+{
+    const size_t b = (size_t)num_seqs * h_q * p_max * 2 * sizeof(float);
+    return (b + 255) / 256 * 256;
+}
+
+// ---------------------------------------------------------------------------------------
+template <int D, int BS, int G, bool FP8>
+int launch_partition(const DecodeParams &prm, int num_seqs, cudaStream_t st)
+{
+    using C = DecodeConfig<D, BS, G, FP8>;
+    static std::atomic<unsigned long long> smem_set{0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (!(smem_set.load(std::memory_order_acquire) & bit)) {
+        if (cudaFuncSetAttribute(paged_decode_partition_kernel<D, BS, G, FP8>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
+            return PA_ERR_CUDA;
+        smem_set.fetch_or(bit, std::memory_order_release);
+    }
+    const dim3 grid(prm.p_max, prm.h_kv, num_seqs);
+    paged_decode_partition_kernel<D, BS, G, FP8><<<grid, C::THREADS, C::SMEM, st>>>(prm);
+    return launch_status();
+}
+
+template <int D, int BS, bool FP8>
+int dispatch_group(int g, const DecodeParams &prm, int n, cudaStream_t st)
+{
+    switch (g) {
+    case 1: return launch_partition<D, BS, 1, FP8>(prm, n, st);
+    case 2: return launch_partition<D, BS, 2, FP8>(prm, n, st);
+    case 4: return launch_partition<D, BS, 4, FP8>(prm, n, st);
+    case 8: return launch_partition<D, BS, 8, FP8>(prm, n, st);
+    default: return PA_ERR_UNSUPPORTED;
+    }
+}
+
+template <int D, bool FP8>
+int dispatch_block(int bs, int g, const DecodeParams &prm, int n, cudaStream_t st)
+{
+    switch (bs) {
+    case 16: return dispatch_group<D, 16, FP8>(g, prm, n, st);
+    case 32: return dispatch_group<D, 32, FP8>(g, prm, n, st);
+    case 64: return dispatch_group<D, 64, FP8>(g, prm, n, st);
+    default: return PA_ERR_UNSUPPORTED;
+    }
+}
+
+int dispatch_partition(int d, int bs, int g, bool fp8, const DecodeParams &prm, int n, cudaStream_t st)
+{
+    if (d == 64) return fp8 ? dispatch_block<64, true>(bs, g, prm, n, st) : dispatch_block<64, false>(bs, g, prm, n, st);
+    if (d == 128) return fp8 ? dispatch_block<128, true>(bs, g, prm, n, st) : dispatch_block<128, false>(bs, g, prm, n, st);
+    return PA_ERR_UNSUPPORTED;
+}
+
+// Shared argument checks of the decode calls.  Returns PA_OK and fills `prm`.
+int prepare_decode(DecodeParams &prm, void *out, const void *q, const void *k_cache, const void *v_cache,
+                   const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
+                   int num_seqs, int max_context_len, int h_q, int h_kv, int head_dim, int block_size,
+                   int num_blocks, float scale, int cache_dtype, float k_scale, float v_scale,
+                   int partition_size, void *workspace, size_t workspace_bytes)
+{
+    if (num_seqs < 0 || max_context_len < 0 || h_q <= 0 || h_kv <= 0 || num_blocks <= 0 ||
+        max_blocks_per_seq <= 0 || partition_size < 0)
+        return PA_ERR_INVALID_ARG;
+    if (h_q % h_kv != 0) return PA_ERR_INVALID_ARG;
+    if (cache_dtype != PA_CACHE_BF16 && cache_dtype != PA_CACHE_E4M3) return PA_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
+    if (cache_dtype == PA_CACHE_E4M3 &&
+        !(std::isfinite(k_scale) && std::isfinite(v_scale) && k_scale > 0.f && v_scale > 0.f))
+        return PA_ERR_INVALID_ARG;
+    if (!supported_head_dim(head_dim) || !supported_block_size(block_size) || !supported_group(h_q / h_kv))
+        return PA_ERR_UNSUPPORTED;
+    if (partition_size > 0 && partition_size % block_size != 0) return PA_ERR_INVALID_ARG;
+    if (h_kv > 65535 || num_seqs > 65535) return PA_ERR_UNSUPPORTED;
+    if (num_seqs > 0) {
+        if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PA_ERR_INVALID_ARG;
+        if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+            return PA_ERR_INVALID_ARG;
+    }
+    const int p_max = grid_partitions(max_context_len, partition_size);
+    const size_t need = pa_decode_workspace_size(num_seqs, h_q, head_dim, max_context_len, partition_size);
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)))
+        return PA_ERR_WORKSPACE;
+
+    prm.out = static_cast<__nv_bfloat16 *>(out);
+    prm.q = static_cast<const __nv_bfloat16 *>(q);
+    prm.k_cache = static_cast<const uint8_t *>(k_cache);
+    prm.v_cache = static_cast<const uint8_t *>(v_cache);
+    prm.block_tables = block_tables;
+    prm.context_lens = context_lens;
+    prm.ws_ml = need > 0 ? static_cast<float *>(workspace) : nullptr;
+    prm.ws_o = need > 0 ? reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
+                                                    ml_bytes(num_seqs, h_q, p_max))
+                        : nullptr;
+    prm.max_blocks_per_seq = max_blocks_per_seq;
+    prm.h_q = h_q;
+    prm.h_kv = h_kv;
+    prm.num_blocks = num_blocks;
+    prm.partition_size = need > 0 ? partition_size : 0;
+    prm.p_max = need > 0 ? p_max : 1;
+    const float ks = cache_dtype == PA_CACHE_E4M3 ? k_scale : 1.f;
+    prm.qk_scale = scale * kLog2e * ks;
+    prm.v_scale = cache_dtype == PA_CACHE_E4M3 ? v_scale : 1.f;
+    return PA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t pa_decode_workspace_size(int num_seqs, int h_q, int head_dim, int max_context_len, int partition_size)
+{
+    if (num_seqs <= 0 || h_q <= 0 || head_dim <= 0 || partition_size <= 0) return 0;
+    const int p_max = grid_partitions(max_context_len, partition_size);
+    if (p_max <= 1) return 0;
+    return ml_bytes(num_seqs, h_q, p_max) + (size_t)num_seqs * h_q * p_max * head_dim * sizeof(float);
+}
+
+int pa_decode_partitions(void *out, const void *q, const void *k_cache, const void *v_cache,
+                         const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
+                         int num_seqs, int max_context_len, int h_q, int h_kv, int head_dim, int block_size,
+                         int num_blocks, float scale, int cache_dtype, float k_scale, float v_scale,
+                         int partition_size, void *workspace, size_t workspace_bytes, void *stream)
+{
+    DecodeParams prm{};
+    int rc = prepare_decode(prm, out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                            num_seqs, max_context_len, h_q, h_kv, head_dim, block_size, num_blocks, scale,
+                            cache_dtype, k_scale, v_scale, partition_size, workspace, workspace_bytes);
+    if (rc != PA_OK || num_seqs == 0) return rc;
+    return dispatch_partition(head_dim, block_size, h_q / h_kv, cache_dtype == PA_CACHE_E4M3, prm, num_seqs,
+                              static_cast<cudaStream_t>(stream));
+}
+
+int pa_decode_merge(void *out, const int32_t *context_lens, int num_seqs, int max_context_len, int h_q,
+                    int head_dim, int partition_size, const void *workspace, size_t workspace_bytes,
+                    void *stream)
+{
+    if (num_seqs < 0 || h_q <= 0 || max_context_len < 0 || partition_size < 0) return PA_ERR_INVALID_ARG;
+    if (!supported_head_dim(head_dim)) return PA_ERR_UNSUPPORTED;
+    if (num_seqs > 65535 || h_q > 65535) return PA_ERR_UNSUPPORTED;
+    const size_t need = pa_decode_workspace_size(num_seqs, h_q, head_dim, max_context_len, partition_size);
+    if (need == 0 || num_seqs == 0) return PA_OK;                 // single partition: nothing to merge
+    if (!out || !context_lens) return PA_ERR_INVALID_ARG;
+    if (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)) return PA_ERR_WORKSPACE;
+    const int p_max = grid_partitions(max_context_len, partition_size);
+    MergeParams mp{};
+    mp.out = static_cast<__nv_bfloat16 *>(out);
+    mp.context_lens = context_lens;
+    mp.ws_ml = static_cast<const float *>(workspace);
+    mp.ws_o = reinterpret_cast<const float *>(static_cast<const uint8_t *>(workspace) + ml_bytes(num_seqs, h_q, p_max));
+    mp.h_q = h_q;
+    mp.partition_size = partition_size;
+    mp.p_max = p_max;
+    const dim3 grid(h_q, num_seqs);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (head_dim == 64)
+        paged_decode_merge_kernel<64><<<grid, 128, 0, st>>>(mp);
+    else
+        paged_decode_merge_kernel<128><<<grid, 128, 0, st>>>(mp);
+    return launch_status();
+}
+
+int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
+              int max_blocks_per_seq, const int32_t *context_lens, int num_seqs, int max_context_len, int h_q,
+              int h_kv, int head_dim, int block_size, int num_blocks, float scale, int cache_dtype,
+              float k_scale, float v_scale, int partition_size, void *workspace, size_t workspace_bytes,
+              void *stream)
+{
+    int rc = pa_decode_partitions(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                                  num_seqs, max_context_len, h_q, h_kv, head_dim, block_size, num_blocks, scale,
+                                  cache_dtype, k_scale, v_scale, partition_size, workspace, workspace_bytes,
+                                  stream);
+    if (rc != PA_OK) return rc;
+    return pa_decode_merge(out, context_lens, num_seqs, max_context_len, h_q, head_dim, partition_size,
+                           workspace, workspace_bytes, stream);
+}
+
+int pa_reshape_and_cache(const void *key, const void *value, int64_t key_stride, int64_t value_stride,
+                         void *k_cache, void *v_cache, const int64_t *slot_mapping, int num_tokens, int h_kv,
+                         int head_dim, int block_size, int num_blocks, int cache_dtype, float k_scale,
+                         float v_scale, void *stream)
+{
+    if (num_tokens < 0 || h_kv <= 0 || num_blocks <= 0) return PA_ERR_INVALID_ARG;
+    if (cache_dtype != PA_CACHE_BF16 && cache_dtype != PA_CACHE_E4M3) return PA_ERR_INVALID_ARG;
+    if (!supported_head_dim(head_dim) || !supported_block_size(block_size)) return PA_ERR_UNSUPPORTED;
+    const int64_t row = (int64_t)h_kv * head_dim;
+    if (key_stride == 0) key_stride = row;
+    if (value_stride == 0) value_stride = row;
+    if (key_stride < row || value_stride < row || key_stride % 8 != 0 || value_stride % 8 != 0)
+        return PA_ERR_INVALID_ARG;
+    if (cache_dtype == PA_CACHE_E4M3 &&
+        !(std::isfinite(k_scale) && std::isfinite(v_scale) && k_scale > 0.f && v_scale > 0.f))
+        return PA_ERR_INVALID_ARG;
+    if (num_tokens == 0) return PA_OK;
+    if (!key || !value || !k_cache || !v_cache || !slot_mapping) return PA_ERR_INVALID_ARG;
+    if (!aligned16(key) || !aligned16(value) || !aligned16(k_cache) || !aligned16(v_cache))
+        return PA_ERR_INVALID_ARG;
+
+    CacheWriteParams p{};
+    p.key = static_cast<const __nv_bfloat16 *>(key);
+    p.value = static_cast<const __nv_bfloat16 *>(value);
+    p.key_stride = key_stride;
+    p.value_stride = value_stride;
+    p.k_cache = static_cast<uint8_t *>(k_cache);
+    p.v_cache = static_cast<uint8_t *>(v_cache);
+    p.slot_mapping = slot_mapping;
+    p.num_tokens = num_tokens;
+    p.h_kv = h_kv;
+    p.block_size = block_size;
+    p.num_slots = (long long)num_blocks * block_size;
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
+    const long long threads = (long long)num_tokens * h_kv * 2 * (head_dim / 8);
+    const long long blocks = (threads + 255) / 256;
+    if (blocks > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const bool fp8 = cache_dtype == PA_CACHE_E4M3;
+    if (head_dim == 64) {
+        if (fp8) reshape_and_cache_e4m3_kernel<64><<<(unsigned)blocks, 256, 0, st>>>(p);
+        else     reshape_and_cache_bf16_kernel<64><<<(unsigned)blocks, 256, 0, st>>>(p);
+    } else {
+        if (fp8) reshape_and_cache_e4m3_kernel<128><<<(unsigned)blocks, 256, 0, st>>>(p);
+        else     reshape_and_cache_bf16_kernel<128><<<(unsigned)blocks, 256, 0, st>>>(p);
+    }
+    return launch_status();
+}
+
+int pa_copy_blocks(void *const *k_caches, void *const *v_caches, int num_layers, const int64_t *block_pairs,
+                   int num_pairs, size_t block_bytes, int num_blocks, void *stream)
+{
+    if (num_layers < 0 || num_pairs < 0 || num_blocks <= 0) return PA_ERR_INVALID_ARG;
+    if (block_bytes == 0 || block_bytes % 16 != 0) return PA_ERR_INVALID_ARG;
+    if (num_layers == 0 || num_pairs == 0) return PA_OK;
+    if (!k_caches || !v_caches || !block_pairs) return PA_ERR_INVALID_ARG;
+    for (int l = 0; l < num_layers; ++l)
+        if (!k_caches[l] || !v_caches[l] || !aligned16(k_caches[l]) || !aligned16(v_caches[l]))
+            return PA_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    for (int l0 = 0; l0 < num_layers; l0 += kMaxLayersPerLaunch) {
+        const int nl = num_layers - l0 < kMaxLayersPerLaunch ? num_layers - l0 : kMaxLayersPerLaunch;
+        CopyBlocksParams p{};
+        for (int l = 0; l < nl; ++l) {
+            p.k[l] = static_cast<uint8_t *>(k_caches[l0 + l]);
+            p.v[l] = static_cast<uint8_t *>(v_caches[l0 + l]);
+        }
+        p.pairs = block_pairs;
+        p.block_bytes = static_cast<long long>(block_bytes);
+        p.num_blocks = num_blocks;
+        copy_blocks_kernel<<<dim3(num_pairs, nl, 2), 256, 0, st>>>(p);
+        const int rc = launch_status();
+        if (rc != PA_OK) return rc;
+    }
+    return PA_OK;
+}
+
+int pa_device_errors(unsigned int *flags, int clear)
+{
+    if (!flags) return PA_ERR_INVALID_ARG;
+    if (cudaDeviceSynchronize() != cudaSuccess) return PA_ERR_CUDA;
+    unsigned int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_errors, sizeof(v)) != cudaSuccess) return PA_ERR_CUDA;
+    *flags = v;
+    if (clear) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(g_device_errors, &zero, sizeof(zero)) != cudaSuccess) return PA_ERR_CUDA;
+    }
+    return PA_OK;
+}
+
+}  // extern "C"

@@ -1,3 +1,4 @@
+import importlib.util
 import os
 import sys
 
@@ -6,6 +7,17 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
+
+
+def _build_library_if_stale():
+    """Compile libpa.so (nvcc, sm_100a) when a source is newer than the library."""
+    spec = importlib.util.spec_from_file_location("_pa_build", os.path.join(ROOT, "paged_kv_cache_428_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
+
+
+_build_library_if_stale()
 
 
 def pytest_configure(config):

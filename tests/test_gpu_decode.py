@@ -1,0 +1,258 @@
+"""GPU decode attention against the fp64 oracle, on every workload shape, plus the
+invariants the method fixes (through the C ABI)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import workloads
+import paged_kv_cache_428_b200 as pa
+from paritylib import (check_close, gpu_fill_e4m3, gpu_step, oracle_caches, oracle_out, u16, u8)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _full_parity(orc, case, rows=None, seqs=None, **kw):
+    out, kc, vc = gpu_step(case, **kw)
+    torch.cuda.synchronize()
+    okc, ovc = oracle_caches(case, orc, seqs=seqs)
+    if seqs is None:                                       # the step's cache writes are bit-exact
+        conv = u8 if case.cache == "e4m3" else u16
+        assert np.array_equal(conv(kc), okc) and np.array_equal(conv(vc), ovc)
+    ref = oracle_out(case, orc, okc, ovc, rows)
+    got = out if rows is None else torch.stack([out[s, h] for s, h in rows])
+    return check_close(got, ref, case.cache == "e4m3", case.name)
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_tiny_gqa2_d64(orc, seed):
+    case = workloads.make_case("tiny_gqa2_d64", seed)
+    _full_parity(orc, case)
+    # decode before the append too (contexts 37 and 80), and with split partitions
+    case_b = workloads.make_case("tiny_gqa2_d64", seed)
+    case_b.context_lens = torch.tensor(case_b.meta["cached"], dtype=torch.int32)
+    case_b.slot_mapping = torch.full_like(case_b.slot_mapping, -1)
+    _full_parity(orc, case_b)
+    _full_parity(orc, case, partition_size=16)
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_llama3_8b_b64_full(orc, seed):
+    """The benchmarked workload at full size, in the launch configuration bench.py times."""
+    case = workloads.make_case("llama3_8b_b64", seed, device=DEV)
+    _full_parity(orc, case)
+
+
+def test_long_context_b8_sampled(orc):
+    case = workloads.make_case("long_context_b8", 0, device=DEV)
+    rows = [(s, h) for s in (0, 5) for h in (0, 3, 4, 17, 31)] + [(7, 8), (2, 30)]
+    _full_parity(orc, case, rows=rows)
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_long_context_reduced_all_rows(orc, seed):
+    case = workloads.make_case("long_context_b8", seed, B=2, ctx_range=(20000, 40000))
+    _full_parity(orc, case)
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_shared_prefix_4x8(orc, seed):
+    case = workloads.make_case("shared_prefix_4x8", seed, device=DEV)
+    _full_parity(orc, case)
+
+
+@pytest.mark.parametrize("bs", [16, 32, 64])
+def test_fp8_mha_b32_sampled_full_size(orc, bs):
+    case = workloads.make_case("fp8_mha_b32_bs%d" % bs, 0, device=DEV)
+    seqs = {0, 13, 31}
+    rows = [(s, h) for s in sorted(seqs) for h in (0, 7, 19, 31)]
+    _full_parity(orc, case, rows=rows, seqs=seqs)
+
+
+@pytest.mark.parametrize("bs", [16, 32, 64])
+@pytest.mark.parametrize("seed", [1, 2])
+def test_fp8_mha_reduced_all_rows(orc, bs, seed):
+    case = workloads.make_case("fp8_mha_b32_bs%d" % bs, seed, B=3, ctx_fixed=1000)
+    _full_parity(orc, case)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("bs", [16, 32, 64])
+@pytest.mark.parametrize("g", [1, 2, 4, 8])
+@pytest.mark.parametrize("cache", ["bf16", "e4m3"])
+def test_every_kernel_variant(orc, d, bs, g, cache):
+    """Small ragged cases over the whole supported shape grid (each template instance)."""
+    h_kv = 2
+    case = workloads.make_case("llama3_8b_b64", 7 * d + bs + g, B=5, h_q=h_kv * g, h_kv=h_kv, d=d, bs=bs,
+                               ctx_range=(1, 700), pool_factor=1.3, partition=128 if bs <= 64 else 0)
+    if cache == "e4m3":
+        case = _as_e4m3(case)
+    _full_parity(orc, case)
+    _full_parity(orc, case, partition_size=0)
+
+
+def _as_e4m3(case):
+    """Turn a bf16 case into an E4M3 one: the same rows become fill rows."""
+    nb, bs = case.num_blocks, case.bs
+    kc, vc = case.k_cache, case.v_cache
+    owned = ~torch.isnan(kc.float()).all(dim=3).all(dim=1)            # [nb, bs]
+    ids = owned.reshape(-1).nonzero().flatten()
+    blk, off = ids // bs, ids % bs
+    case.fill_k_rows = kc.permute(0, 2, 1, 3)[blk, off].contiguous()
+    case.fill_v_rows = vc.permute(0, 2, 1, 3)[blk, off].contiguous()
+    case.fill_slots = ids.to(torch.int64)
+    kmax = max(float(case.fill_k_rows.float().abs().max()), float(case.key_new.float().abs().max()))
+    vmax = max(float(case.fill_v_rows.float().abs().max()), float(case.value_new.float().abs().max()))
+    case.k_scale = float(torch.tensor(kmax / 448.0, dtype=torch.float32))
+    case.v_scale = float(torch.tensor(vmax / 448.0, dtype=torch.float32))
+    case.cache = "e4m3"
+    case.k_cache = case.v_cache = None
+    return case
+
+
+# ---------------------------------------------------------------- invariants and special cases
+
+def _decode(case, kc, vc, tables=None, P=None, ctx=None, mcl=None):
+    out = torch.empty((case.B, case.h_q, case.d), dtype=torch.bfloat16, device=DEV)
+    tab = (case.block_tables if tables is None else tables).to(DEV)
+    cl = (case.context_lens if ctx is None else ctx).to(DEV)
+    pa.pa_decode(out, case.q.to(DEV), kc, vc, tab, cl, case.max_context_len if mcl is None else mcl, case.scale,
+                 case.partition if P is None else P, case.k_scale, case.v_scale)
+    torch.cuda.synchronize()
+    return out
+
+
+def test_permutation_invariance_bitwise():
+    case = workloads.make_case("llama3_8b_b64", 4, device=DEV, B=16)
+    kc, vc = case.k_cache, case.v_cache
+    out1 = _decode(case, kc, vc)
+    perm = torch.randperm(case.num_blocks, generator=torch.Generator().manual_seed(1)).to(DEV)
+    kc2, vc2 = torch.empty_like(kc), torch.empty_like(vc)
+    kc2[perm], vc2[perm] = kc, vc
+    tab = case.block_tables
+    tab2 = torch.where(tab >= 0, perm[tab.clamp(min=0).long()].to(torch.int32), tab)
+    out2 = _decode(case, kc2, vc2, tables=tab2)
+    assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
+
+
+def test_contiguous_physical_blocks_give_the_same_bits():
+    """Identity placement (logical block i in physical block i of each row) vs the shuffled
+    pool: the result does not depend on where blocks live."""
+    case = workloads.make_case("llama3_8b_b64", 6, device=DEV, B=8)
+    out1 = _decode(case, case.k_cache, case.v_cache)
+    tab = case.block_tables.cpu()
+    nblk = [-(-int(c) // case.bs) for c in case.context_lens.cpu()]
+    order = [b for s in range(case.B) for b in tab[s, :nblk[s]].tolist()]
+    kc2 = torch.empty_like(case.k_cache)
+    vc2 = torch.empty_like(case.v_cache)
+    src = torch.tensor(order, device=DEV)
+    kc2[: len(order)], vc2[: len(order)] = case.k_cache[src], case.v_cache[src]
+    tab2 = torch.full_like(tab, -1)
+    pos = 0
+    for s in range(case.B):
+        tab2[s, :nblk[s]] = torch.arange(pos, pos + nblk[s], dtype=torch.int32)
+        pos += nblk[s]
+    out2 = _decode(case, kc2, vc2, tables=tab2)
+    assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
+
+
+def test_shared_vs_privately_copied_prefix_bitwise():
+    """Samples reading one refcounted prefix vs samples whose prefix blocks were copied
+    with pa_copy_blocks into private blocks: identical blocks and identical outputs."""
+    case = workloads.make_case("shared_prefix_4x8", 1, device=DEV)
+    kc, vc = case.k_cache, case.v_cache
+    out_shared = _decode(case, kc, vc)
+    pb = case.meta["prompt_blocks"]
+    S = case.meta["samples"]
+    tab = case.block_tables.cpu().clone()
+    extra = (S - 1) * case.meta["prompts"] * pb
+    nb2 = case.num_blocks + extra
+    kc2 = torch.cat([kc, torch.empty((extra,) + tuple(kc.shape[1:]), dtype=kc.dtype, device=DEV)])
+    vc2 = torch.cat([vc, torch.empty((extra,) + tuple(vc.shape[1:]), dtype=vc.dtype, device=DEV)])
+    nxt = case.num_blocks
+    pairs = []
+    for s in range(case.B):
+        if s % S == 0:
+            continue                                     # the first sample keeps the originals
+        for i in range(pb):
+            pairs.append((int(tab[s, i]), nxt))
+            tab[s, i] = nxt
+            nxt += 1
+    pa.pa_copy_blocks([kc2], [vc2], torch.tensor(pairs, dtype=torch.int64, device=DEV))
+    for a, b in pairs[:50]:
+        assert torch.equal(kc2[a].view(torch.int16), kc2[b].view(torch.int16))
+    case.num_blocks = nb2
+    out_private = _decode(case, kc2, vc2, tables=tab)
+    assert torch.equal(out_shared.view(torch.int16), out_private.view(torch.int16))
+
+
+def test_split_vs_unsplit_agree():
+    case = workloads.make_case("llama3_8b_b64", 2, device=DEV, B=24)
+    ref = _decode(case, case.k_cache, case.v_cache, P=0).float()
+    for P in (16, 64, 256, 512, 2048):
+        got = _decode(case, case.k_cache, case.v_cache, P=P).float()
+        # fp32 reassociation only: within one bf16 rounding step of each other
+        tol = 2.0 ** -8 * torch.maximum(ref.abs(), got.abs()) + 1e-6
+        assert ((got - ref).abs() <= tol).all(), P
+
+
+def test_context_hint_smaller_than_real_context(orc):
+    """max_context_len only sizes the grid: a longer context is still attended in full."""
+    case = workloads.make_case("llama3_8b_b64", 3, B=6, ctx_range=(700, 3000))
+    out, kc, vc = gpu_step(case, max_context_len=600)
+    okc, ovc = oracle_caches(case, orc)
+    check_close(out, oracle_out(case, orc, okc, ovc), False, "short hint")
+
+
+def test_single_token_context_returns_v0_exactly():
+    case = workloads.make_case("tiny_gqa2_d64", 0, device=DEV)
+    ctx = torch.tensor([1, 1], dtype=torch.int32)
+    out = _decode(case, case.k_cache, case.v_cache, ctx=ctx, P=0)
+    tab = case.block_tables.cpu()
+    g = case.h_q // case.h_kv
+    for s in range(case.B):
+        for h in range(case.h_q):
+            v0 = case.v_cache[int(tab[s, 0]), h // g, 0]
+            assert torch.equal(out[s, h].view(torch.int16), v0.view(torch.int16))
+
+
+def test_zero_query_gives_mean_of_v(orc):
+    case = workloads.make_case("llama3_8b_b64", 8, B=4)
+    case.q = torch.zeros_like(case.q)
+    out, kc, vc = gpu_step(case)
+    okc, ovc = oracle_caches(case, orc)
+    ref = oracle_out(case, orc, okc, ovc)
+    check_close(out, ref, False, "q=0")
+
+
+def test_empty_context_gives_zeros():
+    case = workloads.make_case("llama3_8b_b64", 9, device=DEV, B=4)
+    ctx = case.context_lens.clone()
+    ctx[1] = 0
+    ctx[3] = 0
+    out = _decode(case, case.k_cache, case.v_cache, ctx=ctx)
+    assert torch.count_nonzero(out[1].float()) == 0 and torch.count_nonzero(out[3].float()) == 0
+    assert torch.isfinite(out.float()).all()
+
+
+def test_bad_block_id_is_skipped_and_flagged():
+    case = workloads.make_case("llama3_8b_b64", 10, device=DEV, B=3)
+    tab = case.block_tables.clone()
+    tab[1, 2] = case.num_blocks + 7                          # outside the pool
+    pa.pa_device_errors(clear=True)
+    out = _decode(case, case.k_cache, case.v_cache, tables=tab)
+    assert pa.pa_device_errors(clear=True) & pa.PA_DEVERR_BAD_BLOCK
+    assert torch.isnan(out[1].float()).all()                  # the damaged sequence is poisoned
+    ok = _decode(case, case.k_cache, case.v_cache)
+    assert torch.equal(out[0].view(torch.int16), ok[0].view(torch.int16))
+    assert torch.equal(out[2].view(torch.int16), ok[2].view(torch.int16))
+    assert pa.pa_device_errors(clear=True) == 0
+
+
+def test_sentinel_slots_never_reach_the_result():
+    """Unowned slots hold NaN; outputs stay finite for every partition size."""
+    case = workloads.make_case("llama3_8b_b64", 12, device=DEV, B=8)
+    for P in (0, 16, 512):
+        assert torch.isfinite(_decode(case, case.k_cache, case.v_cache, P=P).float()).all()
