@@ -246,11 +246,13 @@ def run_ours(args):
         dist.barrier()
     torch.cuda.synchronize(dev)
     t0 = time.time()
+    torch.cuda.nvtx.range_push("timed")
     with torch.cuda.stream(stream):
         for i in range(args.steps):
             flush.zero_()                               # outside the events: L2 starts cold
             step(evs[i])
     torch.cuda.synchronize(dev)
+    torch.cuda.nvtx.range_pop()
     if world > 1:
         dist.barrier()
     t1 = time.time()
@@ -290,6 +292,7 @@ def run_ours(args):
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize(dev)
+        torch.cuda.nvtx.range_push("timed_e2e")
         with torch.cuda.stream(stream):
             for i in range(args.steps):
                 flush.zero_()
@@ -297,6 +300,7 @@ def run_ours(args):
                 e2e_step()
                 eev[i][1].record(stream)
         torch.cuda.synchronize(dev)
+        torch.cuda.nvtx.range_pop()
         e2e_ms = sum(a.elapsed_time(b) for a, b in eev)
         e2e = {"ms": e2e_ms, "h2d": h2d, "d2h": d2h}
 

@@ -142,6 +142,46 @@ struct DecodeConfig {
     static constexpr int SMEM = OFF_PBUF + NW * PBUF_FLOATS * 4;
 };
 
+// Merge the per-warp online-softmax states of one CTA and write the result: the final bf16
+// row when the sequence has a single partition, else this partition's (m, l, o) partial.
+// Shared memory holds cm[NW][G] (running max, log2 domain), cl[NW][G] (running sum) and
+// co[NW][G][D] (unnormalised output); a warp that saw no token has m = -inf, l = 0, o = 0.
+template <int NW, int G, int D>
+__device__ __forceinline__ void cta_combine_and_write(const DecodeParams &p, const float *cm, int part, int n_part,
+                                                      int kvh, int seq, bool failed)
+{
+    const float *cl = cm + NW * G;
+    const float *co = cl + NW * G;
+    for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
+        const int h = idx / D, dd = idx % D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) M = fmaxf(M, cm[w * G + h]);
+        float L = 0.f, O = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < NW; ++w) {
+                const float sc = exp2f(cm[w * G + h] - M);
+                L += cl[w * G + h] * sc;
+                O += co[(w * G + h) * D + dd] * sc;
+            }
+        }
+        const size_t qrow = (size_t)seq * p.h_q + (size_t)kvh * G + h;
+        if (n_part == 1) {
+            float r = L > 0.f ? (O / L) * p.v_scale : 0.f;
+            if (failed) r = __int_as_float(0x7fc00000);
+            p.out[qrow * D + dd] = __float2bfloat16_rn(r);
+        } else {
+            const size_t prow = qrow * p.p_max + part;
+            p.ws_o[prow * D + dd] = failed ? __int_as_float(0x7fc00000) : O * p.v_scale;
+            if (dd == 0) {
+                p.ws_ml[prow * 2] = M;
+                p.ws_ml[prow * 2 + 1] = failed ? __int_as_float(0x7fc00000) : L;
+            }
+        }
+    }
+}
+
 template <int D, int BS, int G, bool FP8>
 __device__ __forceinline__ void load_row_chunk(const uint8_t *p, float2 (&out)[16 / (FP8 ? 1 : 2) / 2])
 {
@@ -471,35 +511,7 @@ __global__ void __launch_bounds__(DecodeConfig<D, BS, G, FP8>::THREADS)
                 *reinterpret_cast<float2 *>(co + ((size_t)(warp * G + h) * D) + lane * S::DPL + 2 * e) = o[h][e];
     }
     __syncthreads();
-    const bool failed = (*abort_flag != 0) || (*bad_flag != 0);
-    for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
-        const int h = idx / D, dd = idx % D;
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < NW; ++w) M = fmaxf(M, cm[w * G + h]);
-        float L = 0.f, O = 0.f;
-        if (M != -INFINITY) {
-#pragma unroll
-            for (int w = 0; w < NW; ++w) {
-                const float sc = exp2f(cm[w * G + h] - M);
-                L += cl[w * G + h] * sc;
-                O += co[(w * G + h) * D + dd] * sc;
-            }
-        }
-        const size_t qrow = (size_t)seq * p.h_q + (size_t)kvh * G + h;
-        if (n_part == 1) {
-            float r = L > 0.f ? (O / L) * p.v_scale : 0.f;
-            if (failed) r = __int_as_float(0x7fc00000);
-            p.out[qrow * D + dd] = __float2bfloat16_rn(r);
-        } else {
-            const size_t prow = qrow * p.p_max + part;
-            p.ws_o[prow * D + dd] = failed ? __int_as_float(0x7fc00000) : O * p.v_scale;
-            if (dd == 0) {
-                p.ws_ml[prow * 2] = M;
-                p.ws_ml[prow * 2 + 1] = failed ? __int_as_float(0x7fc00000) : L;
-            }
-        }
-    }
+    cta_combine_and_write<NW, G, D>(p, cm, part, n_part, kvh, seq, (*abort_flag != 0) || (*bad_flag != 0));
 }
 
 // ---- pass 2: merge the partitions of each (sequence, query head) ------------------------

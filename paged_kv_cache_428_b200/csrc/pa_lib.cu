@@ -3,10 +3,13 @@
 #include <atomic>
 #include <cmath>
 #include <cstdint>
+#include <cstdlib>
+#include <cstring>
 
 #include "common.cuh"
 #include "cache_ops.cuh"
 #include "decode.cuh"
+#include "decode_mma.cuh"
 
 using namespace pa;
 
@@ -58,9 +61,88 @@ int launch_partition(const DecodeParams &prm, int num_seqs, cudaStream_t st)
     return launch_status();
 }
 
+// ---- tensor maps of the bf16 caches (2-D: rows of head_dim elements, 128B swizzle) -----
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled()
+{
+    static EncodeTiledFn fn = []() -> EncodeTiledFn {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        return reinterpret_cast<EncodeTiledFn>(ptr);
+    }();
+    return fn;
+}
+
+// The cache viewed as [num_blocks * h_kv * block_size rows][head_dim] bf16; a box is 64
+// elements (128 bytes) by block_size rows, swizzled in 128-byte atoms.
+int make_cache_map(CUtensorMap *map, const void *cache, int num_blocks, int h_kv, int block_size, int head_dim)
+{
+    EncodeTiledFn enc = encode_tiled();
+    if (!enc) return PA_ERR_CUDA;
+    const cuuint64_t dims[2] = {(cuuint64_t)head_dim, (cuuint64_t)num_blocks * h_kv * block_size};
+    const cuuint64_t strides[1] = {(cuuint64_t)head_dim * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)block_size};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(cache), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? PA_OK : PA_ERR_CUDA;
+}
+
+template <int D, int BS, int G>
+int launch_partition_mma(const DecodeParams &prm, int num_seqs, cudaStream_t st)
+{
+    using C = MmaDecodeConfig<D, BS, G>;
+    static std::atomic<unsigned long long> smem_set{0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (!(smem_set.load(std::memory_order_acquire) & bit)) {
+        if (cudaFuncSetAttribute(paged_decode_partition_mma_kernel<D, BS, G>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
+            return PA_ERR_CUDA;
+        smem_set.fetch_or(bit, std::memory_order_release);
+    }
+    CUtensorMap mk, mv;
+    int rc = make_cache_map(&mk, prm.k_cache, prm.num_blocks, prm.h_kv, BS, D);
+    if (rc == PA_OK) rc = make_cache_map(&mv, prm.v_cache, prm.num_blocks, prm.h_kv, BS, D);
+    if (rc != PA_OK) return rc;
+    const dim3 grid(prm.p_max, prm.h_kv, num_seqs);
+    paged_decode_partition_mma_kernel<D, BS, G><<<grid, C::THREADS, C::SMEM, st>>>(prm, mk, mv);
+    return launch_status();
+}
+
+// bf16 caches run on the tensor cores; PA_DECODE_BF16_CUDA_CORES=1 selects the CUDA-core
+// kernel instead (kept for A/B measurements; read once per process).
+bool bf16_on_cuda_cores()
+{
+    static const bool v = [] {
+        const char *e = std::getenv("PA_DECODE_BF16_CUDA_CORES");
+        return e != nullptr && std::strcmp(e, "1") == 0;
+    }();
+    return v;
+}
+
 template <int D, int BS, bool FP8>
 int dispatch_group(int g, const DecodeParams &prm, int n, cudaStream_t st)
 {
+    if constexpr (!FP8) {
+        if (!bf16_on_cuda_cores()) {
+            switch (g) {
+            case 1: return launch_partition_mma<D, BS, 1>(prm, n, st);
+            case 2: return launch_partition_mma<D, BS, 2>(prm, n, st);
+            case 4: return launch_partition_mma<D, BS, 4>(prm, n, st);
+            case 8: return launch_partition_mma<D, BS, 8>(prm, n, st);
+            default: return PA_ERR_UNSUPPORTED;
+            }
+        }
+    }
     switch (g) {
     case 1: return launch_partition<D, BS, 1, FP8>(prm, n, st);
     case 2: return launch_partition<D, BS, 2, FP8>(prm, n, st);

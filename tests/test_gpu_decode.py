@@ -114,6 +114,14 @@ def _as_e4m3(case):
 
 # ---------------------------------------------------------------- invariants and special cases
 
+def _with_appended(case):
+    """Write the case's appended tokens into its (device) caches, in place, so that every
+    slot below the context length holds data; returns the case."""
+    pa.pa_reshape_and_cache(case.key_new.to(DEV), case.value_new.to(DEV), case.k_cache, case.v_cache,
+                            case.slot_mapping.to(DEV))
+    return case
+
+
 def _decode(case, kc, vc, tables=None, P=None, ctx=None, mcl=None):
     out = torch.empty((case.B, case.h_q, case.d), dtype=torch.bfloat16, device=DEV)
     tab = (case.block_tables if tables is None else tables).to(DEV)
@@ -125,7 +133,7 @@ def _decode(case, kc, vc, tables=None, P=None, ctx=None, mcl=None):
 
 
 def test_permutation_invariance_bitwise():
-    case = workloads.make_case("llama3_8b_b64", 4, device=DEV, B=16)
+    case = _with_appended(workloads.make_case("llama3_8b_b64", 4, device=DEV, B=16))
     kc, vc = case.k_cache, case.v_cache
     out1 = _decode(case, kc, vc)
     perm = torch.randperm(case.num_blocks, generator=torch.Generator().manual_seed(1)).to(DEV)
@@ -134,13 +142,14 @@ def test_permutation_invariance_bitwise():
     tab = case.block_tables
     tab2 = torch.where(tab >= 0, perm[tab.clamp(min=0).long()].to(torch.int32), tab)
     out2 = _decode(case, kc2, vc2, tables=tab2)
+    assert torch.isfinite(out1.float()).all()
     assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
 
 
 def test_contiguous_physical_blocks_give_the_same_bits():
     """Identity placement (logical block i in physical block i of each row) vs the shuffled
     pool: the result does not depend on where blocks live."""
-    case = workloads.make_case("llama3_8b_b64", 6, device=DEV, B=8)
+    case = _with_appended(workloads.make_case("llama3_8b_b64", 6, device=DEV, B=8))
     out1 = _decode(case, case.k_cache, case.v_cache)
     tab = case.block_tables.cpu()
     nblk = [-(-int(c) // case.bs) for c in case.context_lens.cpu()]
@@ -155,13 +164,14 @@ def test_contiguous_physical_blocks_give_the_same_bits():
         tab2[s, :nblk[s]] = torch.arange(pos, pos + nblk[s], dtype=torch.int32)
         pos += nblk[s]
     out2 = _decode(case, kc2, vc2, tables=tab2)
+    assert torch.isfinite(out1.float()).all()
     assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
 
 
 def test_shared_vs_privately_copied_prefix_bitwise():
     """Samples reading one refcounted prefix vs samples whose prefix blocks were copied
     with pa_copy_blocks into private blocks: identical blocks and identical outputs."""
-    case = workloads.make_case("shared_prefix_4x8", 1, device=DEV)
+    case = _with_appended(workloads.make_case("shared_prefix_4x8", 1, device=DEV))
     kc, vc = case.k_cache, case.v_cache
     out_shared = _decode(case, kc, vc)
     pb = case.meta["prompt_blocks"]
@@ -185,17 +195,41 @@ def test_shared_vs_privately_copied_prefix_bitwise():
         assert torch.equal(kc2[a].view(torch.int16), kc2[b].view(torch.int16))
     case.num_blocks = nb2
     out_private = _decode(case, kc2, vc2, tables=tab)
+    assert torch.isfinite(out_shared.float()).all()
     assert torch.equal(out_shared.view(torch.int16), out_private.view(torch.int16))
 
 
+def _mean_abs_v_under_softmax(case, kc, vc):
+    """sum_t p_t |V_t| / sum_t p_t per (sequence, query head, dim), by plain torch on the
+    gathered rows: the scale of the error that rounding the probabilities to bf16 can cause."""
+    g = case.h_q // case.h_kv
+    out = torch.empty((case.B, case.h_q, case.d), dtype=torch.float32, device=DEV)
+    tab = case.block_tables.to(DEV).long()
+    for s in range(case.B):
+        n = int(case.context_lens[s])
+        blocks = tab[s, : -(-n // case.bs)]
+        K = kc[blocks].permute(0, 2, 1, 3).reshape(-1, case.h_kv, case.d)[:n].float()   # [n, h_kv, d]
+        V = vc[blocks].permute(0, 2, 1, 3).reshape(-1, case.h_kv, case.d)[:n].float()
+        q = case.q[s].to(DEV).float().view(case.h_kv, g, case.d)
+        logits = torch.einsum("hgd,nhd->hgn", q, K) * case.scale
+        w = torch.softmax(logits, dim=-1)
+        out[s] = torch.einsum("hgn,nhd->hgd", w, V.abs()).reshape(case.h_q, case.d)
+    return out
+
+
 def test_split_vs_unsplit_agree():
-    case = workloads.make_case("llama3_8b_b64", 2, device=DEV, B=24)
+    """Different partition sizes evaluate the same sums in a different order and round the
+    probabilities to bf16 (for p.V on the tensor cores) against different running maxima,
+    so results may differ by one output ulp plus 2 * 2^-9 * sum_t p_t |V_t| / sum_t p_t."""
+    case = _with_appended(workloads.make_case("llama3_8b_b64", 2, device=DEV, B=24))
     ref = _decode(case, case.k_cache, case.v_cache, P=0).float()
+    wbar = _mean_abs_v_under_softmax(case, case.k_cache, case.v_cache)
     for P in (16, 64, 256, 512, 2048):
         got = _decode(case, case.k_cache, case.v_cache, P=P).float()
-        # fp32 reassociation only: within one bf16 rounding step of each other
-        tol = 2.0 ** -8 * torch.maximum(ref.abs(), got.abs()) + 1e-6
-        assert ((got - ref).abs() <= tol).all(), P
+        assert torch.isfinite(got).all()
+        tol = 2.0 ** -7 * torch.maximum(ref.abs(), got.abs()) + 2.0 ** -8 * wbar + 1e-6
+        excess = ((got - ref).abs() - tol).max().item()
+        assert excess <= 0, (P, excess)
 
 
 def test_context_hint_smaller_than_real_context(orc):
@@ -228,7 +262,7 @@ def test_zero_query_gives_mean_of_v(orc):
 
 
 def test_empty_context_gives_zeros():
-    case = workloads.make_case("llama3_8b_b64", 9, device=DEV, B=4)
+    case = _with_appended(workloads.make_case("llama3_8b_b64", 9, device=DEV, B=4))
     ctx = case.context_lens.clone()
     ctx[1] = 0
     ctx[3] = 0
@@ -238,7 +272,7 @@ def test_empty_context_gives_zeros():
 
 
 def test_bad_block_id_is_skipped_and_flagged():
-    case = workloads.make_case("llama3_8b_b64", 10, device=DEV, B=3)
+    case = _with_appended(workloads.make_case("llama3_8b_b64", 10, device=DEV, B=3))
     tab = case.block_tables.clone()
     tab[1, 2] = case.num_blocks + 7                          # outside the pool
     pa.pa_device_errors(clear=True)
@@ -253,6 +287,6 @@ def test_bad_block_id_is_skipped_and_flagged():
 
 def test_sentinel_slots_never_reach_the_result():
     """Unowned slots hold NaN; outputs stay finite for every partition size."""
-    case = workloads.make_case("llama3_8b_b64", 12, device=DEV, B=8)
+    case = _with_appended(workloads.make_case("llama3_8b_b64", 12, device=DEV, B=8))
     for P in (0, 16, 512):
         assert torch.isfinite(_decode(case, case.k_cache, case.v_cache, P=P).float()).all()
