@@ -146,6 +146,32 @@ int pa_decode_merge(void *out, const int32_t *context_lens, int num_seqs, int ma
                     int head_dim, int partition_size, const void *workspace, size_t workspace_bytes,
                     void *stream);
 
+/* ---- decode without any allocation (static scratch) ---------------------------
+ * The pages have no counterpart for this call; it exists for callers that cannot
+ * allocate device memory at the point where they run a decode step: code inside an
+ * inference engine's enqueue callback (plugins must not call cudaMalloc there, because it
+ * can synchronise the device and is not allowed while the engine records work), hosts with
+ * a fixed memory budget, and runtimes whose allocator belongs to someone else.
+ * Same arguments and result as pa_decode, minus the workspace: the split-context partials
+ * go to one library-owned array of PA_STATIC_WS_BYTES in device global memory.  Every GPU
+ * on which the library's device code is loaded holds that array until the process exits.
+ *   - Returns PA_ERR_WORKSPACE, launching nothing, when pa_decode_workspace_size(...) for
+ *     the arguments exceeds PA_STATIC_WS_BYTES (e.g. use a larger partition_size, or
+ *     pa_decode with a caller workspace).
+ *   - The first call on a device looks up the array's device address (once per device, with
+ *     that device current); make that first call before any stream capture.
+ *   - All calls share the one array and it keeps the previous call's contents (nothing in it
+ *     needs to start at zero).  Calls that can overlap on the GPU -- on different streams
+ *     without ordering between them -- race on it and must not be issued that way.
+ *   - Calls no cudaMalloc, cudaFree or allocating library routine. */
+#define PA_STATIC_WS_BYTES (16u * 1024u * 1024u)
+
+int pa_decode_static_ws(void *out, const void *q, const void *k_cache, const void *v_cache,
+                        const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
+                        int num_seqs, int max_context_len, int h_q, int h_kv, int head_dim, int block_size,
+                        int num_blocks, float scale, int cache_dtype, float k_scale, float v_scale,
+                        int partition_size, void *stream);
+
 /* ---- copy-on-write block copy ---------------------------------------------
  * For every pair (src, dst) and every layer: cache[dst] = cache[src], byte
  * for byte, for K and for V ("深度解构…" section 2.3; intelliparadigm section

@@ -66,6 +66,8 @@ def _load() -> ctypes.CDLL:
         "pa_decode_partitions": (i32, [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32, i32, i32, f32, i32,
                                        f32, f32, i32, vp, sz, vp]),
         "pa_decode_merge": (i32, [vp, vp, i32, i32, i32, i32, i32, vp, sz, vp]),
+        "pa_decode_static_ws": (i32, [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32, i32, i32, f32, i32,
+                                      f32, f32, i32, vp]),
         "pa_copy_blocks": (i32, [vp, vp, i32, vp, i32, sz, i32, vp]),
         "pa_device_errors": (i32, [ctypes.POINTER(ctypes.c_uint), i32]),
         "pa_validate_block_tables": (i32, [vp, i32, vp, i32, i32, i32]),
@@ -232,6 +234,22 @@ def pa_decode_merge(out, context_lens, max_context_len: int, partition_size: int
     ws_ptr, ws_bytes = (workspace.data_ptr(), workspace.numel()) if workspace is not None else (0, 0)
     _check(_lib.pa_decode_merge(out.data_ptr(), context_lens.data_ptr(), B, int(max_context_len), h_q, d,
                                 int(partition_size), ws_ptr, ws_bytes, _stream_ptr(stream)), "pa_decode_merge")
+
+
+PA_STATIC_WS_BYTES = 16 * 1024 * 1024
+
+
+def pa_decode_static_ws(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len: int,
+                        scale: float = None, partition_size: int = 512, k_scale: float = 1.0, v_scale: float = 1.0,
+                        stream=None) -> torch.Tensor:
+    """pa_decode without a workspace argument and without any allocation: the partials go to
+    the library's static per-device array (PA_STATIC_WS_BYTES).  For callers that may not
+    allocate device memory where they run.  Calls that can overlap on the GPU race on that
+    array; a request needing more scratch than the array raises PagedKVError (workspace)."""
+    args = _decode_args(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len, scale,
+                        partition_size, k_scale, v_scale, None)
+    _check(_lib.pa_decode_static_ws(*args[:-2], _stream_ptr(stream)), "pa_decode_static_ws")
+    return out
 
 
 def pa_copy_blocks(k_caches: Sequence[torch.Tensor], v_caches: Sequence[torch.Tensor], block_pairs: torch.Tensor,

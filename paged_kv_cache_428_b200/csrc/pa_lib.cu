@@ -224,7 +224,54 @@ int prepare_decode(DecodeParams &prm, void *out, const void *q, const void *k_ca
 
 }  // namespace
 
+// Scratch of pa_decode_static_ws: one array per device in global memory (no allocation).
+// Host code must not use this symbol as an address: its device address comes from
+// cudaGetSymbolAddress, looked up once per device with that device current.
+static __device__ __align__(256) unsigned char g_pa_static_ws[PA_STATIC_WS_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::atomic<void *> g_static_ws_addr[kMaxDevices];
+
+// Device address of g_pa_static_ws on the current device (set up on first use).
+int static_ws_address(void **addr)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return PA_ERR_UNSUPPORTED;
+    void *p = g_static_ws_addr[dev].load(std::memory_order_acquire);
+    if (p == nullptr) {
+        if (cudaGetSymbolAddress(&p, g_pa_static_ws) != cudaSuccess || p == nullptr) return PA_ERR_CUDA;
+        g_static_ws_addr[dev].store(p, std::memory_order_release);
+    }
+    *addr = p;
+    return PA_OK;
+}
+
+}  // namespace
+
 extern "C" {
+
+int pa_decode_static_ws(void *out, const void *q, const void *k_cache, const void *v_cache,
+                        const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
+                        int num_seqs, int max_context_len, int h_q, int h_kv, int head_dim, int block_size,
+                        int num_blocks, float scale, int cache_dtype, float k_scale, float v_scale,
+                        int partition_size, void *stream)
+{
+    if (num_seqs < 0 || h_q <= 0 || head_dim <= 0 || max_context_len < 0 || partition_size < 0)
+        return PA_ERR_INVALID_ARG;
+    const size_t need = pa_decode_workspace_size(num_seqs, h_q, head_dim, max_context_len, partition_size);
+    if (need > PA_STATIC_WS_BYTES) return PA_ERR_WORKSPACE;           // beyond the static array
+    void *ws = nullptr;
+    if (need > 0) {
+        const int rc = static_ws_address(&ws);
+        if (rc != PA_OK) return rc;
+    }
+    return pa_decode(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                     max_context_len, h_q, h_kv, head_dim, block_size, num_blocks, scale, cache_dtype, k_scale,
+                     v_scale, partition_size, ws, need > 0 ? (size_t)PA_STATIC_WS_BYTES : 0, stream);
+}
 
 size_t pa_decode_workspace_size(int num_seqs, int h_q, int head_dim, int max_context_len, int partition_size)
 {
