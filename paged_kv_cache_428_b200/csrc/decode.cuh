@@ -131,7 +131,10 @@ struct DecodeConfig {
     using S = DecodeShape<D, BS, G, FP8>;
     static constexpr int NW = 4;                                   // consumer warps
     static constexpr int THREADS = (NW + 1) * 32;                  // + producer warp
-    static constexpr int STAGES = cmax(NW, cmin(16, 98304 / (2 * S::TILE)));
+    // a multiple of NW (see MmaDecodeConfig: parity waits are safe only when block i and
+    // block i - STAGES, which share a stage, belong to the same consumer warp)
+    static constexpr int STAGES = cmax(NW, cmin(16, 98304 / (2 * S::TILE)) / NW * NW);
+    static_assert(STAGES % NW == 0, "stage ring must be a multiple of the consumer warps");
     static constexpr int STAGE_BYTES = STAGES * 2 * S::TILE;
     static constexpr int PBUF_FLOATS = ((S::SUBT * G + G) + 3) / 4 * 4;   // per warp
     static constexpr int COMBINE_BYTES = NW * G * (D + 2) * 4;

@@ -30,15 +30,20 @@
 
 namespace pa {
 
-template <int D, int BS, int G>
+// NW_ consumer warps; RING_ bytes of shared memory for the stage ring (at least NW_ stages).
+template <int D, int BS, int G, int NW_ = 4, int RING_ = 65536>
 struct MmaDecodeConfig {
-    static constexpr int NW = 4;                          // consumer warps
+    static constexpr int NW = NW_;                        // consumer warps
     static constexpr int THREADS = (NW + 1) * 32;         // + producer warp
     static constexpr int HALVES = D / 64;                 // 128-byte column halves of a row
     static constexpr int HALF_BYTES = BS * 128;           // one TMA box (1024-byte multiple)
     static constexpr int TILE = HALVES * HALF_BYTES;      // K (or V) tile of one block
     static constexpr int STAGE_BYTES = 2 * TILE;
-    static constexpr int STAGES = cmax(NW, cmin(16, 65536 / STAGE_BYTES));
+    // A multiple of NW: consumer warp w takes blocks i = w (mod NW), and block i reuses the
+    // stage of block i - STAGES.  Only when that earlier block belongs to the same warp is
+    // the stage's full barrier guaranteed to have finished the previous phase before the
+    // warp waits on it; otherwise a parity wait could pass one phase early.
+    static constexpr int STAGES = cmax(NW, cmin(32, RING_ / STAGE_BYTES) / NW * NW);
     static constexpr int KS = D / 16;                     // k-steps of q.K
     static constexpr int MT = D / 16;                     // m-tiles of O^T (16 head dims each)
     static constexpr int NSUB = BS / 16;
@@ -53,6 +58,7 @@ struct MmaDecodeConfig {
     static_assert(BS % 16 == 0, "block size");
     static_assert(G <= 8, "group");
     static_assert(HALF_BYTES % 1024 == 0, "swizzle atoms");
+    static_assert(STAGES % NW == 0, "stage ring must be a multiple of the consumer warps");
 };
 
 // Byte offset of 16-byte chunk `chunk` (0..7) of row `row` inside a 128B-swizzled box.
@@ -61,12 +67,12 @@ __device__ __forceinline__ uint32_t swz128(int row, int chunk)
     return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
-template <int D, int BS, int G>
-__global__ void __launch_bounds__(MmaDecodeConfig<D, BS, G>::THREADS)
+template <int D, int BS, int G, int NW_ = 4, int RING_ = 65536>
+__global__ void __launch_bounds__(MmaDecodeConfig<D, BS, G, NW_, RING_>::THREADS)
     paged_decode_partition_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
                                       const __grid_constant__ CUtensorMap tmap_v)
 {
-    using C = MmaDecodeConfig<D, BS, G>;
+    using C = MmaDecodeConfig<D, BS, G, NW_, RING_>;
     constexpr int NW = C::NW, STAGES = C::STAGES;
     constexpr unsigned FULL = 0xffffffffu;
 
