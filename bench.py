@@ -37,7 +37,8 @@ if ROOT not in sys.path:
 
 METRIC = "paged decode attention KV GB/s & % of B200 HBM peak; decode tokens/s"
 FALLBACK_HBM_GBS = 6650.0
-KERNEL_SOURCES = [os.path.join(ROOT, "paged_kv_cache_428_b200", "csrc", f) for f in ("decode.cuh", "common.cuh")]
+KERNEL_SOURCES = [os.path.join(ROOT, "paged_kv_cache_428_b200", "csrc", f)
+                  for f in ("common.cuh", "decode.cuh", "decode_mma.cuh")]
 TRAFFIC_SUMMARY = os.path.join(ROOT, "profiles", "ncu_decode_partition_llama3_8b_b64.md")
 
 
@@ -219,18 +220,42 @@ def run_ours(args):
     flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
     stream = torch.cuda.Stream(device=dev)
 
+    # argument checks once; the timed loop calls the C ABI directly (which still validates),
+    # so that the host stays ahead of the GPU
+    L = pa.lib()
+    sp = stream.cuda_stream
+    rargs = pa.reshape_call_args(k_new, v_new, kc, vc, slots)
+    dargs = pa.decode_call_args(out, q, kc, vc, tables, ctx, mcl, case.scale, P, workspace=ws)
+    margs = pa.merge_call_args(out, ctx, mcl, P, ws)
+
     def step(evs=None):
         if evs:
             evs[0].record(stream)
-        pa.pa_reshape_and_cache(k_new, v_new, kc, vc, slots, stream=stream)
+        rc = L.pa_reshape_and_cache(*rargs, sp)
+        rc |= L.pa_decode_partitions(*dargs, sp)
+        rc |= L.pa_decode_merge(*margs, sp)
         if evs:
             evs[1].record(stream)
-        pa.pa_decode_partitions(out, q, kc, vc, tables, ctx, mcl, case.scale, P, workspace=ws, stream=stream)
-        if evs:
-            evs[2].record(stream)
-        pa.pa_decode_merge(out, ctx, mcl, P, ws, stream=stream)
-        if evs:
-            evs[3].record(stream)
+        if rc:
+            raise SystemExit("library call failed: %d" % rc)
+
+    def timed(body, n_ev, nvtx):
+        """Run `body` for args.steps steps, L2 flushed before each (outside the events);
+        returns the summed event intervals (ms).  Barrier + synchronize on both sides."""
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        torch.cuda.nvtx.range_push(nvtx)
+        with torch.cuda.stream(stream):
+            for i in range(args.steps):
+                flush.zero_()
+                body(evs[i])
+        torch.cuda.synchronize(dev)
+        torch.cuda.nvtx.range_pop()
+        if world > 1:
+            dist.barrier()
+        return [sum(e[k].elapsed_time(e[k + 1]) for e in evs) for k in range(n_ev - 1)]
 
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
@@ -241,47 +266,59 @@ def run_ours(args):
     uuid = str(torch.cuda.get_device_properties(dev).uuid)
     sampler = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
     time.sleep(0.3)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
     t0 = time.time()
-    torch.cuda.nvtx.range_push("timed")
-    with torch.cuda.stream(stream):
-        for i in range(args.steps):
-            flush.zero_()                               # outside the events: L2 starts cold
-            step(evs[i])
-    torch.cuda.synchronize(dev)
-    torch.cuda.nvtx.range_pop()
-    if world > 1:
-        dist.barrier()
+    # the timed region: K whole steps, each bracketed by two events
+    step_ms = timed(step, 2, "timed")[0]
     t1 = time.time()
+
+    # each kernel alone over K launches (for the roofline and the per-kernel split); an event
+    # pair itself reads about 2.7 us on this GPU, so these per-kernel times are slight overestimates
+    def only(fn, args_):
+        def body(evs):
+            evs[0].record(stream)
+            rc = fn(*args_, sp)
+            evs[1].record(stream)
+            if rc:
+                raise SystemExit("library call failed: %d" % rc)
+        return body
+    write_ms = timed(only(L.pa_reshape_and_cache, rargs), 2, "kernel_write")[0]
+    part_ms = timed(only(L.pa_decode_partitions, dargs), 2, "kernel_decode")[0]
+    t2 = time.time()
     time.sleep(0.1)
     sampler.stop()
     clocks = sampler.summary(t0, t1)
-
-    step_ms = sum(e[0].elapsed_time(e[3]) for e in evs)
-    write_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
-    part_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
-    merge_ms = sum(e[2].elapsed_time(e[3]) for e in evs)
+    clocks_kernels = sampler.summary(t1, t2)
+    merge_ms = 0.0
 
     # end to end through the public calls: pinned host inputs in, result out, every step
     e2e = None
     if not args.no_e2e:
-        host = {n: t.cpu().pin_memory() for n, t in
-                (("q", q), ("k_new", k_new), ("v_new", v_new), ("slots", slots), ("tables", tables), ("ctx", ctx))}
-        dbuf = {n: torch.empty_like(t, device=dev) for n, t in host.items()}
+        # one pinned host buffer holds every input of a step (q, new K/V rows, slot ids, block
+        # tables, context lengths): one host->device copy in, one device->host copy of out
+        parts = [("q", q), ("k_new", k_new), ("v_new", v_new), ("slots", slots), ("tables", tables), ("ctx", ctx)]
+        offs, total = {}, 0
+        for n, t in parts:
+            offs[n] = total
+            total += (t.numel() * t.element_size() + 255) // 256 * 256
+        host_buf = torch.empty(total, dtype=torch.uint8).pin_memory()
+        dev_buf = torch.empty(total, dtype=torch.uint8, device=dev)
+        view = lambda buf, n, t: buf[offs[n]: offs[n] + t.numel() * t.element_size()].view(t.dtype).view(t.shape)
+        for n, t in parts:
+            view(host_buf, n, t).copy_(t.cpu())
+        dv = {n: view(dev_buf, n, t) for n, t in parts}
         out_host = torch.empty((B, h_q, d), dtype=torch.bfloat16).pin_memory()
-        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        h2d = sum(t.numel() * t.element_size() for _, t in parts)
         d2h = out_host.numel() * out_host.element_size()
+        e_rargs = pa.reshape_call_args(dv["k_new"], dv["v_new"], kc, vc, dv["slots"])
+        e_dargs = pa.decode_call_args(out, dv["q"], kc, vc, dv["tables"], dv["ctx"], mcl, case.scale, P, workspace=ws)
 
         def e2e_step():
-            for n in host:
-                dbuf[n].copy_(host[n], non_blocking=True)
-            pa.pa_reshape_and_cache(dbuf["k_new"], dbuf["v_new"], kc, vc, dbuf["slots"], stream=stream)
-            pa.pa_decode(out, dbuf["q"], kc, vc, dbuf["tables"], dbuf["ctx"], mcl, case.scale, P, workspace=ws,
-                         stream=stream)
+            dev_buf.copy_(host_buf, non_blocking=True)
+            rc = L.pa_reshape_and_cache(*e_rargs, sp)
+            rc |= L.pa_decode(*e_dargs, sp)
             out_host.copy_(out, non_blocking=True)
+            if rc:
+                raise SystemExit("library call failed: %d" % rc)
 
         with torch.cuda.stream(stream):
             for _ in range(args.warmup):
@@ -339,21 +376,23 @@ def run_ours(args):
         "config": {"workload": args.workload, "num_seqs": B, "h_q": h_q, "h_kv": case.h_kv, "head_dim": d,
                    "block_size": case.bs, "ctx": "U{512..4096} incl. appended token", "partition": P,
                    "num_blocks": case.num_blocks, "kv_bytes_per_step_per_gpu": my_bytes,
-                   "step": "reshape_and_cache(64 new tokens) + decode partitions + merge",
+                   "step": "reshape_and_cache(64 new tokens) + split-context decode with in-kernel merge",
                    "l2": "flushed between steps (2x L2 write, outside the events)",
                    "parallelism": "replicas (weak scaling, no collective)" if world > 1 else "single GPU"},
         "tokens_per_s": round(tot_seqs / per_step_s, 1),
         "pct_of_hbm_peak": round(value / world / peak, 4),
         "pct_of_nominal_8tbs": round(value / world / 8000.0, 4),
-        "kernels_ms_per_step": {"reshape_and_cache": round(write_ms / K, 5),
-                                "decode_partitions": round(part_ms / K, 5),
-                                "decode_merge": round(merge_ms / K, 5)},
-        "roofline": {"bound": "hbm", "kernel": "paged_decode_partition_kernel", "achieved": round(achieved, 1),
+        "kernels_ms_alone": {"reshape_and_cache": round(write_ms / K, 5),
+                             "decode (partitions + in-kernel merge)": round(part_ms / K, 5),
+                             "note": "each kernel timed alone over K launches after the timed steps; "
+                                     "an empty CUDA-event pair reads ~2.7 us and is included"},
+        "roofline": {"bound": "hbm", "kernel": "paged_decode_partition_mma_kernel", "achieved": round(achieved, 1),
                      "peak": peak, "peak_kind": peak_kind + " (hbm_gbs copy bandwidth)", "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": ncu_traffic_per_launch(),
                      "algorithmic_bytes_per_launch": part_bytes},
-        "gpu_launches": 3 * K,
+        "gpu_launches": K * (2 + (1 if P > 0 and -(-mcl // P) > 16 else 0)),
         "clocks": clocks,
+        "clocks_kernel_loops": clocks_kernels,
     }
     if e2e:
         line["e2e"] = {"value": round(tot_bytes / (e2e_ms / 1e3 / K) / 1e9, 2), "unit": "GB/s",

@@ -65,6 +65,9 @@ extern "C" {
 
 typedef enum { PA_CACHE_BF16 = 0, PA_CACHE_E4M3 = 1 } pa_cache_dtype;
 
+/* partition_size value of pa_decode: balanced split (see pa_decode) */
+#define PA_PARTITION_AUTO (-1)
+
 /* Human-readable text of a status code (static storage). */
 const char *pa_status_str(int status);
 
@@ -109,7 +112,13 @@ int pa_reshape_and_cache(const void *key, const void *value, int64_t key_stride,
  * Long contexts are split into partitions of partition_size tokens; each
  * partition keeps its own running max, sum and unnormalised output and a
  * second pass merges them (split-context decode).  partition_size = 0 means
- * one partition per sequence; otherwise it must be a multiple of block_size.
+ * one partition per sequence; a positive value must be a multiple of
+ * block_size.  PA_PARTITION_AUTO splits the step's blocks evenly over as many
+ * CTAs as the GPU holds at once (each takes one contiguous range of
+ * (sequence, KV head, block) triples, so all finish together), merging split
+ * sequences in the same launch; it applies to bf16 caches with at most 4096
+ * sequences and otherwise falls back to partitions of max(512, ~max_context_len
+ * / 16) tokens; either way no separate merge pass is needed.
  *   out            device bf16 [num_seqs][h_q][head_dim] (RNE of the fp32 result)
  *   q              device bf16 [num_seqs][h_q][head_dim]
  *   block_tables   device int32 [num_seqs][max_blocks_per_seq]; entries past
@@ -119,7 +128,15 @@ int pa_reshape_and_cache(const void *key, const void *value, int64_t key_stride,
  *                  grid (no device->host read).  A longer context is still
  *                  computed correctly: its last partition grows.
  *   workspace      device, >= pa_decode_workspace_size(...) bytes, 16-byte
- *                  aligned; holds fp32 partials; may be NULL when that size is 0
+ *                  aligned; holds per-group counters and fp32 partials; may be
+ *                  NULL when that size is 0.  It must be zero-filled before its
+ *                  first use (e.g. one cudaMemset); every call leaves it ready
+ *                  for the next one.  Calls sharing a workspace must not overlap
+ *                  on the GPU.  After a call that recorded PA_DEVERR_TIMEOUT,
+ *                  zero it again.
+ * Groups (sequence, KV head) of at most 16 partitions are merged inside the
+ * first pass by the CTA that finishes the group last; pa_decode launches the
+ * merge pass only when a group can have more partitions. 
  * Accuracy: fp32 accumulation; vs an fp64 evaluation of the same formula,
  * max|err| <= 2e-2 and <= 1e-2 * max|ref| for bf16 caches, <= 6e-2 for E4M3. */
 size_t pa_decode_workspace_size(int num_seqs, int h_q, int head_dim, int max_context_len,

@@ -151,22 +151,8 @@ def pa_reshape_and_cache(key: torch.Tensor, value: torch.Tensor, k_cache: torch.
                          slot_mapping: torch.Tensor, k_scale: float = 1.0, v_scale: float = 1.0,
                          stream=None) -> None:
     """key/value bf16 [T, h_kv, d] (rows may be strided in dim 0); caches [NB, h_kv, bs, d]."""
-    for t, n in ((key, "key"), (value, "value")):
-        if t.dtype != torch.bfloat16 or not t.is_cuda or t.dim() != 3 or t.stride(2) != 1 or t.stride(1) != t.shape[2]:
-            raise ValueError("%s must be a CUDA bf16 [T, h_kv, d] tensor with packed heads" % n)
-    _need(k_cache, "k_cache", (torch.bfloat16, torch.uint8, torch.float8_e4m3fn), 4)
-    _need(v_cache, "v_cache", (k_cache.dtype,), 4)
-    _need(slot_mapping, "slot_mapping", (torch.int64,), 1)
-    T, h_kv, d = key.shape
-    NB, h2, bs, d2 = k_cache.shape
-    if h2 != h_kv or d2 != d or tuple(v_cache.shape) != tuple(k_cache.shape) or value.shape != key.shape \
-            or slot_mapping.shape[0] != T:
-        raise ValueError("shape mismatch between key/value, caches and slot_mapping")
-    rc = _lib.pa_reshape_and_cache(key.data_ptr(), value.data_ptr(), key.stride(0), value.stride(0),
-                                   k_cache.data_ptr(), v_cache.data_ptr(), slot_mapping.data_ptr(), T, h_kv, d, bs,
-                                   NB, cache_dtype_code(k_cache), float(k_scale), float(v_scale),
-                                   _stream_ptr(stream))
-    _check(rc, "pa_reshape_and_cache")
+    args = reshape_call_args(key, value, k_cache, v_cache, slot_mapping, k_scale, v_scale)
+    _check(_lib.pa_reshape_and_cache(*args, _stream_ptr(stream)), "pa_reshape_and_cache")
 
 
 def pa_decode_workspace_size(num_seqs: int, h_q: int, head_dim: int, max_context_len: int,
@@ -176,9 +162,10 @@ def pa_decode_workspace_size(num_seqs: int, h_q: int, head_dim: int, max_context
 
 def make_workspace(num_seqs: int, h_q: int, head_dim: int, max_context_len: int, partition_size: int,
                    device="cuda") -> torch.Tensor:
-    """A caller-owned workspace of the size pa_decode needs (uint8, possibly empty)."""
+    """A caller-owned, zero-filled workspace of the size pa_decode needs (uint8, possibly
+    empty).  Reusable by consecutive calls that do not overlap on the GPU."""
     n = pa_decode_workspace_size(num_seqs, h_q, head_dim, max_context_len, partition_size)
-    return torch.empty(max(n, 16), dtype=torch.uint8, device=device)
+    return torch.zeros(max(n, 16), dtype=torch.uint8, device=device)
 
 
 def _decode_args(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len, scale, partition_size,
@@ -204,6 +191,44 @@ def _decode_args(out, q, k_cache, v_cache, block_tables, context_lens, max_conte
             block_tables.shape[1], context_lens.data_ptr(), B, int(max_context_len), h_q, h_kv, d, bs, NB,
             float(scale), cache_dtype_code(k_cache), float(k_scale), float(v_scale), int(partition_size),
             ws_ptr, ws_bytes)
+
+
+def decode_call_args(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len: int,
+                     scale: float = None, partition_size: int = 512, k_scale: float = 1.0, v_scale: float = 1.0,
+                     workspace: Optional[torch.Tensor] = None) -> tuple:
+    """Checked raw arguments of pa_decode / pa_decode_partitions (all but the stream), for
+    callers that issue the same call many times: ``lib().pa_decode(*args, stream)``."""
+    return _decode_args(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len, scale,
+                        partition_size, k_scale, v_scale, workspace)
+
+
+def merge_call_args(out, context_lens, max_context_len: int, partition_size: int,
+                    workspace: Optional[torch.Tensor]) -> tuple:
+    """Checked raw arguments of pa_decode_merge (all but the stream)."""
+    _need(out, "out", (torch.bfloat16,), 3)
+    _need(context_lens, "context_lens", (torch.int32,), 1)
+    B, h_q, d = out.shape
+    ws_ptr, ws_bytes = (workspace.data_ptr(), workspace.numel()) if workspace is not None else (0, 0)
+    return (out.data_ptr(), context_lens.data_ptr(), B, int(max_context_len), h_q, d, int(partition_size), ws_ptr,
+            ws_bytes)
+
+
+def reshape_call_args(key, value, k_cache, v_cache, slot_mapping, k_scale: float = 1.0,
+                      v_scale: float = 1.0) -> tuple:
+    """Checked raw arguments of pa_reshape_and_cache (all but the stream)."""
+    for t, n in ((key, "key"), (value, "value")):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or t.dim() != 3 or t.stride(2) != 1 or t.stride(1) != t.shape[2]:
+            raise ValueError("%s must be a CUDA bf16 [T, h_kv, d] tensor with packed heads" % n)
+    _need(k_cache, "k_cache", (torch.bfloat16, torch.uint8, torch.float8_e4m3fn), 4)
+    _need(v_cache, "v_cache", (k_cache.dtype,), 4)
+    _need(slot_mapping, "slot_mapping", (torch.int64,), 1)
+    T, h_kv, d = key.shape
+    NB, h2, bs, d2 = k_cache.shape
+    if h2 != h_kv or d2 != d or tuple(v_cache.shape) != tuple(k_cache.shape) or value.shape != key.shape \
+            or slot_mapping.shape[0] != T:
+        raise ValueError("shape mismatch between key/value, caches and slot_mapping")
+    return (key.data_ptr(), value.data_ptr(), key.stride(0), value.stride(0), k_cache.data_ptr(), v_cache.data_ptr(),
+            slot_mapping.data_ptr(), T, h_kv, d, bs, NB, cache_dtype_code(k_cache), float(k_scale), float(v_scale))
 
 
 def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len: int, scale: float = None,

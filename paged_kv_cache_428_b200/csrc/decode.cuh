@@ -45,6 +45,7 @@ struct DecodeParams {
     const int32_t *context_lens;   // [B]
     float *ws_ml;                  // [B][h_q][p_max][2]  (m, l), log2 domain
     float *ws_o;                   // [B][h_q][p_max][D]  unnormalised, v_scale applied
+    int *counters;                 // [B][h_kv] partitions finished; zero between launches
     int max_blocks_per_seq;
     int h_q;
     int h_kv;
@@ -54,6 +55,11 @@ struct DecodeParams {
     float qk_scale;                // scale * log2(e) (* k_scale for E4M3)
     float v_scale;                 // 1 for bf16
 };
+
+// Groups (sequence, KV head) with at most this many partitions are merged inside the
+// partition kernel by the CTA that finishes last; larger groups go to the merge kernel,
+// whose many CTAs keep more partial reads in flight than one CTA could.
+constexpr int kFusedMergeMaxPartitions = 16;
 
 __host__ __device__ __forceinline__ int decode_num_partitions(int ctx, int partition_size, int p_max)
 {
@@ -138,7 +144,8 @@ struct DecodeConfig {
     static constexpr int STAGE_BYTES = STAGES * 2 * S::TILE;
     static constexpr int PBUF_FLOATS = ((S::SUBT * G + G) + 3) / 4 * 4;   // per warp
     static constexpr int COMBINE_BYTES = NW * G * (D + 2) * 4;
-    static constexpr int REGION0 = cmax(STAGE_BYTES, COMBINE_BYTES);  // stages, then combine area
+    static constexpr int MERGE_BYTES = (2 * G * kFusedMergeMaxPartitions + 1) * 4;
+    static constexpr int REGION0 = cmax(STAGE_BYTES, COMBINE_BYTES + MERGE_BYTES);  // stages, then combine + merge
     static constexpr int OFF_BARS = (REGION0 + 127) / 128 * 128;
     static constexpr int OFF_FLAGS = OFF_BARS + 2 * STAGES * 8;
     static constexpr int OFF_PBUF = (OFF_FLAGS + (STAGES + 4) * 4 + 15) / 16 * 16;
@@ -149,9 +156,15 @@ struct DecodeConfig {
 // row when the sequence has a single partition, else this partition's (m, l, o) partial.
 // Shared memory holds cm[NW][G] (running max, log2 domain), cl[NW][G] (running sum) and
 // co[NW][G][D] (unnormalised output); a warp that saw no token has m = -inf, l = 0, o = 0.
+// For a group of at most kFusedMergeMaxPartitions partitions, the CTA then publishes its
+// partial (fence, then one atomic increment of the group's counter); the CTA that makes the
+// count complete merges all partials of the group (out = sum_p 2^(m_p - M) o_p /
+// sum_p 2^(m_p - M) l_p) and resets the counter to zero.  No CTA waits on another.
+// `scratch` is shared memory for 2 * G * kFusedMergeMaxPartitions + 1 floats, not
+// overlapping cm/cl/co.
 template <int NW, int G, int D>
 __device__ __forceinline__ void cta_combine_and_write(const DecodeParams &p, const float *cm, int part, int n_part,
-                                                      int kvh, int seq, bool failed)
+                                                      int kvh, int seq, bool failed, float *scratch)
 {
     const float *cl = cm + NW * G;
     const float *co = cl + NW * G;
@@ -182,6 +195,63 @@ __device__ __forceinline__ void cta_combine_and_write(const DecodeParams &p, con
                 p.ws_ml[prow * 2 + 1] = failed ? __int_as_float(0x7fc00000) : L;
             }
         }
+    }
+    if (n_part == 1 || n_part > kFusedMergeMaxPartitions) return;
+
+    // ---- publish this partial; the last CTA of the group merges ----
+    // The CTA barrier orders every thread's partial writes before thread 0's device-scope
+    // fence, which publishes them before the counter update (release); the CTA that sees
+    // the count complete fences again before its threads read the other partials (acquire).
+    int *last = reinterpret_cast<int *>(scratch + 2 * G * kFusedMergeMaxPartitions);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int *cnt = p.counters + (size_t)seq * p.h_kv + kvh;
+        __threadfence();
+        const int prev = atomicAdd(cnt, 1);
+        const int is_last = (prev == n_part - 1);
+        if (is_last) {
+            *cnt = 0;                      // every partition of this launch has counted
+            __threadfence();
+        }
+        *last = is_last;
+    }
+    __syncthreads();
+    if (!*last) return;
+    float *mw = scratch;                                         // [G][16] m_p, then weights
+    float *lw = scratch + G * kFusedMergeMaxPartitions;          // [G][16] l_p
+    const size_t row0 = (size_t)seq * p.h_q + (size_t)kvh * G;
+    for (int idx = threadIdx.x; idx < G * n_part; idx += blockDim.x) {
+        const int h = idx / n_part, q = idx % n_part;
+        const float2 ml = __ldcg(reinterpret_cast<const float2 *>(p.ws_ml + ((row0 + h) * p.p_max + q) * 2));
+        mw[h * kFusedMergeMaxPartitions + q] = ml.x;
+        lw[h * kFusedMergeMaxPartitions + q] = ml.y;
+    }
+    __syncthreads();
+    if (threadIdx.x < G) {
+        const int h = threadIdx.x;
+        float M = -INFINITY;
+        for (int q = 0; q < n_part; ++q) M = fmaxf(M, mw[h * kFusedMergeMaxPartitions + q]);
+        float L = 0.f;
+        for (int q = 0; q < n_part; ++q) {
+            const float w = exp2f(mw[h * kFusedMergeMaxPartitions + q] - M);
+            mw[h * kFusedMergeMaxPartitions + q] = w;
+            L += w * lw[h * kFusedMergeMaxPartitions + q];
+        }
+        const float inv = 1.f / L;
+        for (int q = 0; q < n_part; ++q) mw[h * kFusedMergeMaxPartitions + q] *= inv;
+    }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < G * D / 4; idx += blockDim.x) {
+        const int h = idx / (D / 4), d4 = idx % (D / 4);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        const float *po = p.ws_o + (row0 + h) * p.p_max * D + 4 * d4;
+        for (int q = 0; q < n_part; ++q) {
+            const float w = mw[h * kFusedMergeMaxPartitions + q];
+            const float4 x = __ldcg(reinterpret_cast<const float4 *>(po + (size_t)q * D));
+            acc.x += w * x.x; acc.y += w * x.y; acc.z += w * x.z; acc.w += w * x.w;
+        }
+        __nv_bfloat16 *dst = p.out + (row0 + h) * D + 4 * d4;
+        *reinterpret_cast<uint2 *>(dst) = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
     }
 }
 
@@ -514,7 +584,8 @@ __global__ void __launch_bounds__(DecodeConfig<D, BS, G, FP8>::THREADS)
                 *reinterpret_cast<float2 *>(co + ((size_t)(warp * G + h) * D) + lane * S::DPL + 2 * e) = o[h][e];
     }
     __syncthreads();
-    cta_combine_and_write<NW, G, D>(p, cm, part, n_part, kvh, seq, (*abort_flag != 0) || (*bad_flag != 0));
+    cta_combine_and_write<NW, G, D>(p, cm, part, n_part, kvh, seq, (*abort_flag != 0) || (*bad_flag != 0),
+                                    reinterpret_cast<float *>(smem + C::COMBINE_BYTES));
 }
 
 // ---- pass 2: merge the partitions of each (sequence, query head) ------------------------
@@ -535,7 +606,7 @@ __global__ void __launch_bounds__(128) paged_decode_merge_kernel(const MergePara
     const int qh = blockIdx.x, seq = blockIdx.y;
     const int ctx = p.context_lens[seq];
     const int n_part = decode_num_partitions(ctx, p.partition_size, p.p_max);
-    if (n_part <= 1) return;                                     // finished by pass 1
+    if (n_part <= kFusedMergeMaxPartitions) return;              // finished by pass 1
     const size_t row = (size_t)seq * p.h_q + qh;
     const float *ml = p.ws_ml + row * p.p_max * 2;
     const float *po = p.ws_o + row * p.p_max * D;

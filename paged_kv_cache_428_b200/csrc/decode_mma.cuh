@@ -31,7 +31,7 @@
 namespace pa {
 
 // NW_ consumer warps; RING_ bytes of shared memory for the stage ring (at least NW_ stages).
-template <int D, int BS, int G, int NW_ = 4, int RING_ = 65536>
+template <int D, int BS, int G, int NW_ = 2, int RING_ = 32768>
 struct MmaDecodeConfig {
     static constexpr int NW = NW_;                        // consumer warps
     static constexpr int THREADS = (NW + 1) * 32;         // + producer warp
@@ -49,7 +49,8 @@ struct MmaDecodeConfig {
     static constexpr int NSUB = BS / 16;
     static constexpr int RING = STAGES * STAGE_BYTES;
     static constexpr int COMBINE_BYTES = NW * G * (D + 2) * 4;
-    static constexpr int REGION0 = cmax(RING, COMBINE_BYTES);
+    static constexpr int MERGE_BYTES = (2 * G * kFusedMergeMaxPartitions + 1) * 4;
+    static constexpr int REGION0 = cmax(RING, COMBINE_BYTES + MERGE_BYTES);
     static constexpr int OFF_BARS = (REGION0 + 127) / 128 * 128;
     static constexpr int OFF_FLAGS = OFF_BARS + 2 * STAGES * 8;
     static constexpr int SMEM_USED = OFF_FLAGS + (STAGES + 4) * 4;
@@ -67,7 +68,102 @@ __device__ __forceinline__ uint32_t swz128(int row, int chunk)
     return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
-template <int D, int BS, int G, int NW_ = 4, int RING_ = 65536>
+// B fragments of Q^T for one group: column n = query head T/4 of the group (zero when
+// >= G); k-step ks covers dims [16 ks, 16 ks + 16): lo pair at 2 tq, hi pair at 8 + 2 tq.
+// `qg` points at the group's first query head.
+template <class C, int G, int D>
+__device__ __forceinline__ void mma_load_q(uint32_t (&qb)[C::KS][2], const __nv_bfloat16 *qg, int lane)
+{
+    const int gq = lane >> 2, tq = lane & 3;
+    const uint32_t *qrow = reinterpret_cast<const uint32_t *>(qg + (size_t)(gq < G ? gq : 0) * D);
+#pragma unroll
+    for (int ks = 0; ks < C::KS; ++ks) {
+        qb[ks][0] = gq < G ? qrow[8 * ks + tq] : 0u;
+        qb[ks][1] = gq < G ? qrow[8 * ks + 4 + tq] : 0u;
+    }
+}
+
+// One physical block of one KV head, already in shared memory (K tile at `ktile`, V tile
+// right after it, both as 128B-swizzled boxes), folded into a warp's online-softmax state:
+// `valid` tokens of the block count; rows past them are masked and their V rows zeroed.
+// State: m_run/l_run for heads 2tq, 2tq+1 (log2 domain), o = O^T fragments.
+template <class C, int BS, int G>
+__device__ __forceinline__ void mma_consume_block(uint8_t *ktile, int valid, const uint32_t (&qb)[C::KS][2],
+                                                  float qk_scale, float (&m_run)[2], float (&l_run)[2],
+                                                  float (&o)[C::MT][4], int lane)
+{
+    constexpr unsigned FULL = 0xffffffffu;
+    uint8_t *vtile = ktile + C::TILE;
+    if (valid < BS) {
+        // zero the V rows past the context (both halves, whole 128-byte rows)
+        const int n16 = (BS - valid) * 8 * C::HALVES;
+        for (int e = lane; e < n16; e += 32) {
+            const int hf = e / ((BS - valid) * 8);
+            const int row = valid + (e / 8) % (BS - valid);
+            reinterpret_cast<uint4 *>(vtile + hf * C::HALF_BYTES + row * 128)[e % 8] = make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+    }
+    const uint32_t kbase = smem_addr(ktile);
+    const uint32_t vbase = smem_addr(vtile);
+    const int mrow = lane & 7, mat = lane >> 3;     // ldmatrix: row address this lane supplies
+    const int r = lane >> 2;                        // token row of this lane's scores
+#pragma unroll 1
+    for (int sub = 0; sub < C::NSUB; ++sub) {
+        if (sub * 16 >= valid) break;
+        // ---- S^T = K . Q^T for 16 tokens ----
+        float sT[4] = {0.f, 0.f, 0.f, 0.f};
+        {
+            const int tok = sub * 16 + (mat & 1) * 8 + mrow;
+#pragma unroll
+            for (int ks = 0; ks < C::KS; ++ks) {
+                const int chunk = 2 * (ks & 3) + (mat >> 1);
+                uint32_t a[4];
+                ldmatrix_x4(a, kbase + (ks >> 2) * C::HALF_BYTES + swz128(tok, chunk));
+                mma_bf16_16816(sT, a[0], a[1], a[2], a[3], qb[ks][0], qb[ks][1]);
+            }
+        }
+        // ---- online softmax: tokens r and r + 8, heads 2tq and 2tq + 1 ----
+        const int t0 = sub * 16 + r;
+        const float x0 = t0 < valid ? sT[0] * qk_scale : -INFINITY;
+        const float x1 = t0 < valid ? sT[1] * qk_scale : -INFINITY;
+        const float x2 = t0 + 8 < valid ? sT[2] * qk_scale : -INFINITY;
+        const float x3 = t0 + 8 < valid ? sT[3] * qk_scale : -INFINITY;
+        float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(FULL, mx0, off));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(FULL, mx1, off));
+        }
+        const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);
+        const float al0 = exp2f(m_run[0] - mn0), al1 = exp2f(m_run[1] - mn1);
+        m_run[0] = mn0;
+        m_run[1] = mn1;
+        const float p0 = exp2f(x0 - mn0), p1 = exp2f(x1 - mn1);
+        const float p2 = exp2f(x2 - mn0), p3 = exp2f(x3 - mn1);
+        l_run[0] = l_run[0] * al0 + (p0 + p2);
+        l_run[1] = l_run[1] * al1 + (p1 + p3);
+        // P^T as the B operand: b0 = P[head T/4][tokens 2tq, 2tq+1], b1 = tokens + 8
+        const uint32_t pb0 = movmatrix_trans(pack_bf16x2(p0, p1));
+        const uint32_t pb1 = movmatrix_trans(pack_bf16x2(p2, p3));
+        // ---- O^T += V^T . P^T (m-tiles of 16 head dims) ----
+        const int tok = sub * 16 + (mat >> 1) * 8 + mrow;
+#pragma unroll
+        for (int mt = 0; mt < C::MT; ++mt) {
+            o[mt][0] *= al0;
+            o[mt][1] *= al1;
+            o[mt][2] *= al0;
+            o[mt][3] *= al1;
+            const int chunk = ((2 * mt) & 7) + (mat & 1);
+            uint32_t a[4];
+            ldmatrix_x4_trans(a, vbase + (mt >> 2) * C::HALF_BYTES + swz128(tok, chunk));
+            mma_bf16_16816(o[mt], a[0], a[1], a[2], a[3], pb0, pb1);
+        }
+    }
+}
+
+template <int D, int BS, int G, int NW_ = 2, int RING_ = 32768>
 __global__ void __launch_bounds__(MmaDecodeConfig<D, BS, G, NW_, RING_>::THREADS)
     paged_decode_partition_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
                                       const __grid_constant__ CUtensorMap tmap_v)
@@ -172,23 +268,8 @@ __global__ void __launch_bounds__(MmaDecodeConfig<D, BS, G, NW_, RING_>::THREADS
         }
     } else {
         // ------------------------------ consumers ------------------------------
-        // B fragments of Q^T: column n = query head T/4 of the group (zero when >= G);
-        // k-step ks covers dims [16 ks, 16 ks + 16): lo pair at 2 tq, hi pair at 8 + 2 tq.
         uint32_t qb[C::KS][2];
-        {
-            const int gq = lane >> 2;
-            const uint32_t *qrow = reinterpret_cast<const uint32_t *>(
-                p.q + ((size_t)seq * p.h_q + (size_t)kvh * G + (gq < G ? gq : 0)) * D);
-#pragma unroll
-            for (int ks = 0; ks < C::KS; ++ks) {
-                qb[ks][0] = gq < G ? qrow[8 * ks + tq] : 0u;
-                qb[ks][1] = gq < G ? qrow[8 * ks + 4 + tq] : 0u;
-            }
-        }
-        const float qk_scale = p.qk_scale;
-        const int mrow = lane & 7, mat = lane >> 3;     // ldmatrix: row address this lane supplies
-        const int r = lane >> 2;                        // token row of this lane's scores
-
+        mma_load_q<C, G, D>(qb, p.q + ((size_t)seq * p.h_q + (size_t)kvh * G) * D, lane);
         for (int i = warp; i < nblk; i += NW) {
             if (*abort_flag) break;
             const int st = i % STAGES;
@@ -203,74 +284,8 @@ __global__ void __launch_bounds__(MmaDecodeConfig<D, BS, G, NW_, RING_>::THREADS
             if (stage_bad[st]) {
                 if (lane == 0) *bad_flag = 1;
             } else {
-                uint8_t *ktile = stages + st * C::STAGE_BYTES;
-                uint8_t *vtile = ktile + C::TILE;
-                const int valid = min(BS, tok_end - (tok_begin + i * BS));
-                if (valid < BS) {
-                    // zero the V rows past the context (both halves, whole 128-byte rows)
-                    const int n16 = (BS - valid) * 8 * C::HALVES;
-                    for (int e = lane; e < n16; e += 32) {
-                        const int hf = e / ((BS - valid) * 8);
-                        const int row = valid + (e / 8) % (BS - valid);
-                        reinterpret_cast<uint4 *>(vtile + hf * C::HALF_BYTES + row * 128)[e % 8] = make_uint4(0, 0, 0, 0);
-                    }
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                }
-                const uint32_t kbase = smem_addr(ktile);
-                const uint32_t vbase = smem_addr(vtile);
-#pragma unroll 1
-                for (int sub = 0; sub < C::NSUB; ++sub) {
-                    if (sub * 16 >= valid) break;
-                    // ---- S^T = K . Q^T for 16 tokens ----
-                    float sT[4] = {0.f, 0.f, 0.f, 0.f};
-                    {
-                        const int tok = sub * 16 + (mat & 1) * 8 + mrow;
-#pragma unroll
-                        for (int ks = 0; ks < C::KS; ++ks) {
-                            const int chunk = 2 * (ks & 3) + (mat >> 1);
-                            uint32_t a[4];
-                            ldmatrix_x4(a, kbase + (ks >> 2) * C::HALF_BYTES + swz128(tok, chunk));
-                            mma_bf16_16816(sT, a[0], a[1], a[2], a[3], qb[ks][0], qb[ks][1]);
-                        }
-                    }
-                    // ---- online softmax: tokens r and r + 8, heads 2tq and 2tq + 1 ----
-                    const int t0 = sub * 16 + r;
-                    const float x0 = t0 < valid ? sT[0] * qk_scale : -INFINITY;
-                    const float x1 = t0 < valid ? sT[1] * qk_scale : -INFINITY;
-                    const float x2 = t0 + 8 < valid ? sT[2] * qk_scale : -INFINITY;
-                    const float x3 = t0 + 8 < valid ? sT[3] * qk_scale : -INFINITY;
-                    float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
-#pragma unroll
-                    for (int off = 4; off < 32; off <<= 1) {
-                        mx0 = fmaxf(mx0, __shfl_xor_sync(FULL, mx0, off));
-                        mx1 = fmaxf(mx1, __shfl_xor_sync(FULL, mx1, off));
-                    }
-                    const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);
-                    const float al0 = exp2f(m_run[0] - mn0), al1 = exp2f(m_run[1] - mn1);
-                    m_run[0] = mn0;
-                    m_run[1] = mn1;
-                    const float p0 = exp2f(x0 - mn0), p1 = exp2f(x1 - mn1);
-                    const float p2 = exp2f(x2 - mn0), p3 = exp2f(x3 - mn1);
-                    l_run[0] = l_run[0] * al0 + (p0 + p2);
-                    l_run[1] = l_run[1] * al1 + (p1 + p3);
-                    // P^T as the B operand: b0 = P[head T/4][tokens 2tq, 2tq+1], b1 = tokens + 8
-                    const uint32_t pb0 = movmatrix_trans(pack_bf16x2(p0, p1));
-                    const uint32_t pb1 = movmatrix_trans(pack_bf16x2(p2, p3));
-                    // ---- O^T += V^T . P^T (m-tiles of 16 head dims) ----
-                    const int tok = sub * 16 + (mat >> 1) * 8 + mrow;
-#pragma unroll
-                    for (int mt = 0; mt < C::MT; ++mt) {
-                        o[mt][0] *= al0;
-                        o[mt][1] *= al1;
-                        o[mt][2] *= al0;
-                        o[mt][3] *= al1;
-                        const int chunk = ((2 * mt) & 7) + (mat & 1);
-                        uint32_t a[4];
-                        ldmatrix_x4_trans(a, vbase + (mt >> 2) * C::HALF_BYTES + swz128(tok, chunk));
-                        mma_bf16_16816(o[mt], a[0], a[1], a[2], a[3], pb0, pb1);
-                    }
-                }
+                mma_consume_block<C, BS, G>(stages + st * C::STAGE_BYTES, min(BS, tok_end - (tok_begin + i * BS)),
+                                            qb, p.qk_scale, m_run, l_run, o, lane);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty_bar[st]);
@@ -305,7 +320,8 @@ __global__ void __launch_bounds__(MmaDecodeConfig<D, BS, G, NW_, RING_>::THREADS
         }
     }
     __syncthreads();
-    cta_combine_and_write<NW, G, D>(p, cm, part, n_part, kvh, seq, (*abort_flag != 0) || (*bad_flag != 0));
+    cta_combine_and_write<NW, G, D>(p, cm, part, n_part, kvh, seq, (*abort_flag != 0) || (*bad_flag != 0),
+                                    reinterpret_cast<float *>(smem + C::COMBINE_BYTES));
 }
 
 }  // namespace pa

@@ -10,6 +10,7 @@
 #include "cache_ops.cuh"
 #include "decode.cuh"
 #include "decode_mma.cuh"
+#include "decode_balanced.cuh"
 
 using namespace pa;
 
@@ -35,10 +36,23 @@ int grid_partitions(int max_context_len, int partition_size)
     return n < 1 ? 1 : static_cast<int>(n);
 }
 
-size_t ml_bytes(int num_seqs, int h_q, int p_max)
+size_t round256(size_t b) { return (b + 255) / 256 * 256; }
+
+// Workspace of the split-context decode: [group counters][m, l partials][o partials].
+// The counters (one int per sequence x query head, an upper bound of the KV heads) must be
+// zero before the first launch; every launch leaves them zero again.
+struct WsLayout {
+    size_t ml = 0, o = 0, total = 0, counters_bytes = 0;
+};
+
+WsLayout ws_layout(int num_seqs, int h_q, int head_dim, int p_max)
 {
-    const size_t b = (size_t)num_seqs * h_q * p_max * 2 * sizeof(float);
-    return (b + 255) / 256 * 256;
+    WsLayout L;
+    L.counters_bytes = round256((size_t)num_seqs * h_q * sizeof(int));
+    L.ml = L.counters_bytes;
+    L.o = L.ml + round256((size_t)num_seqs * h_q * p_max * 2 * sizeof(float));
+    L.total = L.o + (size_t)num_seqs * h_q * p_max * head_dim * sizeof(float);
+    return L;
 }
 
 // ---------------------------------------------------------------------------------------
@@ -95,6 +109,42 @@ int make_cache_map(CUtensorMap *map, const void *cache, int num_blocks, int h_kv
     return r == CUDA_SUCCESS ? PA_OK : PA_ERR_CUDA;
 }
 
+// Encoded maps of recently used caches (per host thread): a decode step reuses the same
+// cache tensors call after call, and encoding costs host time on every launch otherwise.
+struct CachedMap {
+    const void *base = nullptr;
+    int num_blocks = 0, h_kv = 0, block_size = 0, head_dim = 0;
+    CUtensorMap map;
+};
+
+int cached_cache_map(CUtensorMap *map, const void *cache, int num_blocks, int h_kv, int block_size, int head_dim)
+{
+    constexpr int kSlots = 8;
+    static thread_local CachedMap slots[kSlots];
+    static thread_local int next = 0;
+    for (const CachedMap &c : slots) {
+        if (c.base == cache && c.num_blocks == num_blocks && c.h_kv == h_kv && c.block_size == block_size &&
+            c.head_dim == head_dim) {
+            *map = c.map;
+            return PA_OK;
+        }
+    }
+    CachedMap &c = slots[next];
+    next = (next + 1) % kSlots;
+    const int rc = make_cache_map(&c.map, cache, num_blocks, h_kv, block_size, head_dim);
+    if (rc != PA_OK) {
+        c.base = nullptr;
+        return rc;
+    }
+    c.base = cache;
+    c.num_blocks = num_blocks;
+    c.h_kv = h_kv;
+    c.block_size = block_size;
+    c.head_dim = head_dim;
+    *map = c.map;
+    return PA_OK;
+}
+
 template <int D, int BS, int G>
 int launch_partition_mma(const DecodeParams &prm, int num_seqs, cudaStream_t st)
 {
@@ -110,8 +160,8 @@ int launch_partition_mma(const DecodeParams &prm, int num_seqs, cudaStream_t st)
         smem_set.fetch_or(bit, std::memory_order_release);
     }
     CUtensorMap mk, mv;
-    int rc = make_cache_map(&mk, prm.k_cache, prm.num_blocks, prm.h_kv, BS, D);
-    if (rc == PA_OK) rc = make_cache_map(&mv, prm.v_cache, prm.num_blocks, prm.h_kv, BS, D);
+    int rc = cached_cache_map(&mk, prm.k_cache, prm.num_blocks, prm.h_kv, BS, D);
+    if (rc == PA_OK) rc = cached_cache_map(&mv, prm.v_cache, prm.num_blocks, prm.h_kv, BS, D);
     if (rc != PA_OK) return rc;
     const dim3 grid(prm.p_max, prm.h_kv, num_seqs);
     paged_decode_partition_mma_kernel<D, BS, G><<<grid, C::THREADS, C::SMEM, st>>>(prm, mk, mv);
@@ -170,6 +220,133 @@ int dispatch_partition(int d, int bs, int g, bool fp8, const DecodeParams &prm, 
     return PA_ERR_UNSUPPORTED;
 }
 
+// ---- balanced schedule (PA_PARTITION_AUTO) ------------------------------------------------
+// Workspace: [group counters][partial (m, l): kBalancedMaxCtas x 2 x Gmax x 2][partial o].
+// Gmax = min(8, h_q) bounds the query heads per KV head (h_kv is not an argument of
+// pa_decode_workspace_size).  The same workspace also serves the 512-token fallback.
+// Partitions of the AUTO fallback: at least 512 tokens, and never more than
+// kFusedMergeMaxPartitions per sequence (a multiple of 64 tokens, so of every block size),
+// so that every group is merged inside the partition kernel.
+int auto_fallback_partition(int max_context_len)
+{
+    const long long need = ((long long)max_context_len + kFusedMergeMaxPartitions - 1) / kFusedMergeMaxPartitions;
+    const long long p = (need + 63) / 64 * 64;
+    return (int)(p > 512 ? p : 512);
+}
+
+struct BalLayout {
+    size_t ml = 0, o = 0, total = 0, counters_bytes = 0;
+};
+
+BalLayout bal_layout(int num_seqs, int h_q, int head_dim)
+{
+    const size_t gmax = (size_t)(h_q < kBalancedMaxGroup ? h_q : kBalancedMaxGroup);
+    BalLayout L;
+    L.counters_bytes = round256((size_t)num_seqs * h_q * sizeof(int));
+    L.ml = L.counters_bytes;
+    L.o = L.ml + round256((size_t)kBalancedMaxCtas * 2 * gmax * 2 * sizeof(float));
+    L.total = L.o + (size_t)kBalancedMaxCtas * 2 * gmax * head_dim * sizeof(float);
+    return L;
+}
+
+bool balanced_applies(int num_seqs, int h_q, int h_kv, int cache_dtype)
+{
+    return cache_dtype == PA_CACHE_BF16 && !bf16_on_cuda_cores() && num_seqs <= kBalancedMaxSeqs &&
+           h_q / h_kv <= kBalancedMaxGroup;
+}
+
+struct SmCount {
+    int dev = -1, count = 0;
+};
+
+int sm_count()
+{
+    static thread_local SmCount cache;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    if (cache.dev != dev) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+        cache.dev = dev;
+        cache.count = n;
+    }
+    return cache.count;
+}
+
+template <int D, int BS, int G>
+int launch_balanced(const DecodeParams &prm, int num_seqs, const BalLayout &lay, void *workspace, cudaStream_t st)
+{
+    using BC = BalancedConfig<D, BS, G>;
+    static std::atomic<unsigned long long> smem_set{0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (!(smem_set.load(std::memory_order_acquire) & bit)) {
+        if (cudaFuncSetAttribute(paged_decode_balanced_kernel<D, BS, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 BC::smem_bytes(kBalancedMaxSeqs)) != cudaSuccess)
+            return PA_ERR_CUDA;
+        smem_set.fetch_or(bit, std::memory_order_release);
+    }
+    const int smem = BC::smem_bytes(num_seqs);
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, paged_decode_balanced_kernel<D, BS, G>, BC::THREADS,
+                                                      smem) != cudaSuccess || per_sm < 1)
+        return PA_ERR_CUDA;
+    const int sms = sm_count();
+    if (sms < 1) return PA_ERR_CUDA;
+    int ctas = per_sm * sms;
+    if (ctas > kBalancedMaxCtas) ctas = kBalancedMaxCtas;
+    CUtensorMap mk, mv;
+    int rc = cached_cache_map(&mk, prm.k_cache, prm.num_blocks, prm.h_kv, BS, D);
+    if (rc == PA_OK) rc = cached_cache_map(&mv, prm.v_cache, prm.num_blocks, prm.h_kv, BS, D);
+    if (rc != PA_OK) return rc;
+    BalancedParams bp{};
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    bp.out = prm.out;
+    bp.q = prm.q;
+    bp.block_tables = prm.block_tables;
+    bp.context_lens = prm.context_lens;
+    bp.counters = reinterpret_cast<int *>(ws);
+    bp.part_ml = reinterpret_cast<float *>(ws + lay.ml);
+    bp.part_o = reinterpret_cast<float *>(ws + lay.o);
+    bp.max_blocks_per_seq = prm.max_blocks_per_seq;
+    bp.num_seqs = num_seqs;
+    bp.h_q = prm.h_q;
+    bp.h_kv = prm.h_kv;
+    bp.num_blocks = prm.num_blocks;
+    bp.num_ctas = ctas;
+    bp.qk_scale = prm.qk_scale;
+    paged_decode_balanced_kernel<D, BS, G><<<ctas, BC::THREADS, smem, st>>>(bp, mk, mv);
+    return launch_status();
+}
+
+template <int D, int BS>
+int dispatch_balanced_group(int g, const DecodeParams &prm, int n, const BalLayout &lay, void *ws, cudaStream_t st)
+{
+    switch (g) {
+    case 1: return launch_balanced<D, BS, 1>(prm, n, lay, ws, st);
+    case 2: return launch_balanced<D, BS, 2>(prm, n, lay, ws, st);
+    case 4: return launch_balanced<D, BS, 4>(prm, n, lay, ws, st);
+    case 8: return launch_balanced<D, BS, 8>(prm, n, lay, ws, st);
+    default: return PA_ERR_UNSUPPORTED;
+    }
+}
+
+int dispatch_balanced(int d, int bs, int g, const DecodeParams &prm, int n, const BalLayout &lay, void *ws,
+                      cudaStream_t st)
+{
+    if (d == 64) {
+        if (bs == 16) return dispatch_balanced_group<64, 16>(g, prm, n, lay, ws, st);
+        if (bs == 32) return dispatch_balanced_group<64, 32>(g, prm, n, lay, ws, st);
+        if (bs == 64) return dispatch_balanced_group<64, 64>(g, prm, n, lay, ws, st);
+    } else if (d == 128) {
+        if (bs == 16) return dispatch_balanced_group<128, 16>(g, prm, n, lay, ws, st);
+        if (bs == 32) return dispatch_balanced_group<128, 32>(g, prm, n, lay, ws, st);
+        if (bs == 64) return dispatch_balanced_group<128, 64>(g, prm, n, lay, ws, st);
+    }
+    return PA_ERR_UNSUPPORTED;
+}
+
 // Shared argument checks of the decode calls.  Returns PA_OK and fills `prm`.
 int prepare_decode(DecodeParams &prm, void *out, const void *q, const void *k_cache, const void *v_cache,
                    const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
@@ -178,7 +355,7 @@ int prepare_decode(DecodeParams &prm, void *out, const void *q, const void *k_ca
                    int partition_size, void *workspace, size_t workspace_bytes)
 {
     if (num_seqs < 0 || max_context_len < 0 || h_q <= 0 || h_kv <= 0 || num_blocks <= 0 ||
-        max_blocks_per_seq <= 0 || partition_size < 0)
+        max_blocks_per_seq <= 0 || partition_size < PA_PARTITION_AUTO)
         return PA_ERR_INVALID_ARG;
     if (h_q % h_kv != 0) return PA_ERR_INVALID_ARG;
     if (cache_dtype != PA_CACHE_BF16 && cache_dtype != PA_CACHE_E4M3) return PA_ERR_INVALID_ARG;
@@ -189,6 +366,15 @@ int prepare_decode(DecodeParams &prm, void *out, const void *q, const void *k_ca
     if (!supported_head_dim(head_dim) || !supported_block_size(block_size) || !supported_group(h_q / h_kv))
         return PA_ERR_UNSUPPORTED;
     if (partition_size > 0 && partition_size % block_size != 0) return PA_ERR_INVALID_ARG;
+    if (partition_size == PA_PARTITION_AUTO) {
+        // the balanced kernel (set up by the caller) or, where it does not apply, 512-token partitions
+        if (pa_decode_workspace_size(num_seqs, h_q, head_dim, max_context_len, PA_PARTITION_AUTO) > 0 &&
+            (workspace == nullptr || workspace_bytes < pa_decode_workspace_size(num_seqs, h_q, head_dim,
+                                                                                max_context_len, PA_PARTITION_AUTO) ||
+             !aligned16(workspace)))
+            return PA_ERR_WORKSPACE;
+        partition_size = auto_fallback_partition(max_context_len);
+    }
     if (h_kv > 65535 || num_seqs > 65535) return PA_ERR_UNSUPPORTED;
     if (num_seqs > 0) {
         if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PA_ERR_INVALID_ARG;
@@ -206,10 +392,11 @@ int prepare_decode(DecodeParams &prm, void *out, const void *q, const void *k_ca
     prm.v_cache = static_cast<const uint8_t *>(v_cache);
     prm.block_tables = block_tables;
     prm.context_lens = context_lens;
-    prm.ws_ml = need > 0 ? static_cast<float *>(workspace) : nullptr;
-    prm.ws_o = need > 0 ? reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
-                                                    ml_bytes(num_seqs, h_q, p_max))
-                        : nullptr;
+    const WsLayout lay = ws_layout(num_seqs, h_q, head_dim, p_max);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    prm.counters = need > 0 ? reinterpret_cast<int *>(ws) : nullptr;
+    prm.ws_ml = need > 0 ? reinterpret_cast<float *>(ws + lay.ml) : nullptr;
+    prm.ws_o = need > 0 ? reinterpret_cast<float *>(ws + lay.o) : nullptr;
     prm.max_blocks_per_seq = max_blocks_per_seq;
     prm.h_q = h_q;
     prm.h_kv = h_kv;
@@ -267,6 +454,11 @@ int pa_decode_static_ws(void *out, const void *q, const void *k_cache, const voi
     if (need > 0) {
         const int rc = static_ws_address(&ws);
         if (rc != PA_OK) return rc;
+        // the group counters at the front of the scratch must start at zero (a launch that
+        // stopped early could have left counts behind); the rest needs no clearing
+        const size_t counters = ws_layout(num_seqs, h_q, head_dim,
+                                          grid_partitions(max_context_len, partition_size)).counters_bytes;
+        if (cudaMemsetAsync(ws, 0, counters, static_cast<cudaStream_t>(stream)) != cudaSuccess) return PA_ERR_CUDA;
     }
     return pa_decode(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
                      max_context_len, h_q, h_kv, head_dim, block_size, num_blocks, scale, cache_dtype, k_scale,
@@ -275,10 +467,17 @@ int pa_decode_static_ws(void *out, const void *q, const void *k_cache, const voi
 
 size_t pa_decode_workspace_size(int num_seqs, int h_q, int head_dim, int max_context_len, int partition_size)
 {
-    if (num_seqs <= 0 || h_q <= 0 || head_dim <= 0 || partition_size <= 0) return 0;
+    if (num_seqs <= 0 || h_q <= 0 || head_dim <= 0) return 0;
+    if (partition_size == PA_PARTITION_AUTO) {
+        const size_t bal = bal_layout(num_seqs, h_q, head_dim).total;
+        const size_t grid = pa_decode_workspace_size(num_seqs, h_q, head_dim, max_context_len,
+                                                     auto_fallback_partition(max_context_len));
+        return bal > grid ? bal : grid;
+    }
+    if (partition_size <= 0) return 0;
     const int p_max = grid_partitions(max_context_len, partition_size);
     if (p_max <= 1) return 0;
-    return ml_bytes(num_seqs, h_q, p_max) + (size_t)num_seqs * h_q * p_max * head_dim * sizeof(float);
+    return ws_layout(num_seqs, h_q, head_dim, p_max).total;
 }
 
 int pa_decode_partitions(void *out, const void *q, const void *k_cache, const void *v_cache,
@@ -292,6 +491,9 @@ int pa_decode_partitions(void *out, const void *q, const void *k_cache, const vo
                             num_seqs, max_context_len, h_q, h_kv, head_dim, block_size, num_blocks, scale,
                             cache_dtype, k_scale, v_scale, partition_size, workspace, workspace_bytes);
     if (rc != PA_OK || num_seqs == 0) return rc;
+    if (partition_size == PA_PARTITION_AUTO && balanced_applies(num_seqs, h_q, h_kv, cache_dtype))
+        return dispatch_balanced(head_dim, block_size, h_q / h_kv, prm, num_seqs, bal_layout(num_seqs, h_q, head_dim),
+                                 workspace, static_cast<cudaStream_t>(stream));
     return dispatch_partition(head_dim, block_size, h_q / h_kv, cache_dtype == PA_CACHE_E4M3, prm, num_seqs,
                               static_cast<cudaStream_t>(stream));
 }
@@ -300,19 +502,23 @@ int pa_decode_merge(void *out, const int32_t *context_lens, int num_seqs, int ma
                     int head_dim, int partition_size, const void *workspace, size_t workspace_bytes,
                     void *stream)
 {
-    if (num_seqs < 0 || h_q <= 0 || max_context_len < 0 || partition_size < 0) return PA_ERR_INVALID_ARG;
+    if (num_seqs < 0 || h_q <= 0 || max_context_len < 0 || partition_size < PA_PARTITION_AUTO)
+        return PA_ERR_INVALID_ARG;
     if (!supported_head_dim(head_dim)) return PA_ERR_UNSUPPORTED;
+    if (partition_size == PA_PARTITION_AUTO) return PA_OK;       // merged inside the first pass
     if (num_seqs > 65535 || h_q > 65535) return PA_ERR_UNSUPPORTED;
     const size_t need = pa_decode_workspace_size(num_seqs, h_q, head_dim, max_context_len, partition_size);
     if (need == 0 || num_seqs == 0) return PA_OK;                 // single partition: nothing to merge
     if (!out || !context_lens) return PA_ERR_INVALID_ARG;
     if (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)) return PA_ERR_WORKSPACE;
     const int p_max = grid_partitions(max_context_len, partition_size);
+    if (p_max <= kFusedMergeMaxPartitions) return PA_OK;         // every group merged by pass 1
+    const WsLayout lay = ws_layout(num_seqs, h_q, head_dim, p_max);
     MergeParams mp{};
     mp.out = static_cast<__nv_bfloat16 *>(out);
     mp.context_lens = context_lens;
-    mp.ws_ml = static_cast<const float *>(workspace);
-    mp.ws_o = reinterpret_cast<const float *>(static_cast<const uint8_t *>(workspace) + ml_bytes(num_seqs, h_q, p_max));
+    mp.ws_ml = reinterpret_cast<const float *>(static_cast<const uint8_t *>(workspace) + lay.ml);
+    mp.ws_o = reinterpret_cast<const float *>(static_cast<const uint8_t *>(workspace) + lay.o);
     mp.h_q = h_q;
     mp.partition_size = partition_size;
     mp.p_max = p_max;

@@ -52,8 +52,9 @@ def test_workspace_size():
     assert pa.pa_decode_workspace_size(64, 32, 128, 4096, 0) == 0
     assert pa.pa_decode_workspace_size(64, 32, 128, 512, 512) == 0        # one partition: no partials
     n = pa.pa_decode_workspace_size(64, 32, 128, 4096, 512)
+    counters = (64 * 32 * 4 + 255) // 256 * 256              # one int per (sequence, query head)
     ml = (64 * 32 * 8 * 2 * 4 + 255) // 256 * 256
-    assert n == ml + 64 * 32 * 8 * 128 * 4
+    assert n == counters + ml + 64 * 32 * 8 * 128 * 4
 
 
 L = pa.lib()

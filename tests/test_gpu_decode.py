@@ -290,3 +290,105 @@ def test_sentinel_slots_never_reach_the_result():
     case = _with_appended(workloads.make_case("llama3_8b_b64", 12, device=DEV, B=8))
     for P in (0, 16, 512):
         assert torch.isfinite(_decode(case, case.k_cache, case.v_cache, P=P).float()).all()
+
+
+def test_workspace_reused_across_calls(orc):
+    """One workspace for many calls: the per-group counters of the in-kernel merge are left at
+    zero by every call, so consecutive calls with different inputs stay exact."""
+    ws = None
+    for seed in (31, 32, 33):
+        case = workloads.make_case("llama3_8b_b64", seed, B=12, ctx_range=(600, 4000))
+        out, kc, vc = gpu_step(case)            # warm the kernels; fresh workspace inside
+        if ws is None:
+            ws = pa.make_workspace(case.B, case.h_q, case.d, 4096, case.partition, DEV)
+        out2 = torch.empty_like(out)
+        pa.pa_decode(out2, case.q.to(DEV), kc, vc, case.block_tables.to(DEV), case.context_lens.to(DEV), 4096,
+                     case.scale, case.partition, workspace=ws)
+        torch.cuda.synchronize()
+        okc, ovc = oracle_caches(case, orc)
+        check_close(out2, oracle_out(case, orc, okc, ovc), False, "reuse %d" % seed)
+        assert torch.equal(out.view(torch.int16), out2.view(torch.int16))
+    counters = ws[: case.B * case.h_q * 4].view(torch.int32)
+    assert int(counters.abs().sum()) == 0
+
+
+# ---------------------------------------------------------------- balanced schedule (AUTO)
+AUTO = -1
+
+
+@pytest.mark.parametrize("name,kw", [
+    ("tiny_gqa2_d64", {}),
+    ("llama3_8b_b64", {}),
+    ("llama3_8b_b64", dict(B=3, ctx_range=(1, 90))),          # tiny groups, many per CTA
+    ("llama3_8b_b64", dict(B=1, ctx_range=(60000, 60000))),    # one group over every CTA
+    ("shared_prefix_4x8", {}),
+])
+def test_auto_schedule_parity(orc, name, kw):
+    case = workloads.make_case(name, 5, device=DEV, **kw)
+    _full_parity(orc, case, partition_size=AUTO)
+
+
+def test_auto_schedule_long_context_sampled(orc):
+    case = workloads.make_case("long_context_b8", 1, device=DEV)
+    rows = [(s, h) for s in (1, 6) for h in (0, 9, 31)] + [(3, 5)]
+    _full_parity(orc, case, rows=rows, partition_size=AUTO)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("bs", [16, 32, 64])
+@pytest.mark.parametrize("g", [1, 2, 4, 8])
+def test_auto_schedule_every_variant(orc, d, bs, g):
+    case = workloads.make_case("llama3_8b_b64", 11 * d + bs + g, B=7, h_q=2 * g, h_kv=2, d=d, bs=bs,
+                               ctx_range=(1, 3000), pool_factor=1.2)
+    _full_parity(orc, case, partition_size=AUTO)
+
+
+def test_auto_schedule_e4m3_falls_back(orc):
+    case = workloads.make_case("fp8_mha_b32_bs16", 2, B=3, ctx_fixed=1500)
+    _full_parity(orc, case, partition_size=AUTO)
+
+
+def test_auto_schedule_edge_cases(orc):
+    case = _with_appended(workloads.make_case("llama3_8b_b64", 14, device=DEV, B=10))
+    ctx = case.context_lens.clone()
+    ctx[0] = 0
+    ctx[4] = 0
+    ctx[9] = 1
+    out = _decode(case, case.k_cache, case.v_cache, ctx=ctx, P=AUTO)
+    assert torch.count_nonzero(out[0].float()) == 0 and torch.count_nonzero(out[4].float()) == 0
+    assert torch.isfinite(out.float()).all()
+    ref = _decode(case, case.k_cache, case.v_cache, ctx=ctx, P=512)
+    tol = 2.0 ** -7 * torch.maximum(ref.float().abs(), out.float().abs()) + 2.0 ** -8
+    assert ((out.float() - ref.float()).abs() <= tol).all()
+    # a bad block id poisons its own sequence only and is flagged
+    tab = case.block_tables.clone()
+    tab[6, 3] = case.num_blocks + 1
+    pa.pa_device_errors(clear=True)
+    bad = _decode(case, case.k_cache, case.v_cache, tables=tab, P=AUTO)
+    assert pa.pa_device_errors(clear=True) & pa.PA_DEVERR_BAD_BLOCK
+    assert torch.isnan(bad[6].float()).all()
+    good = _decode(case, case.k_cache, case.v_cache, P=AUTO)
+    for s in (0, 5, 7, 9):
+        assert torch.equal(bad[s].view(torch.int16), good[s].view(torch.int16))
+    assert pa.pa_device_errors(clear=True) == 0
+
+
+def test_auto_schedule_permutation_invariance_and_reuse():
+    case = _with_appended(workloads.make_case("llama3_8b_b64", 15, device=DEV, B=20))
+    ws = pa.make_workspace(case.B, case.h_q, case.d, case.max_context_len, AUTO, DEV)
+    out1 = torch.empty((case.B, case.h_q, case.d), dtype=torch.bfloat16, device=DEV)
+    for _ in range(3):                                         # the same workspace, three calls
+        pa.pa_decode(out1, case.q, case.k_cache, case.v_cache, case.block_tables, case.context_lens,
+                     case.max_context_len, case.scale, AUTO, workspace=ws)
+    perm = torch.randperm(case.num_blocks, generator=torch.Generator().manual_seed(3)).to(DEV)
+    kc2, vc2 = torch.empty_like(case.k_cache), torch.empty_like(case.v_cache)
+    kc2[perm], vc2[perm] = case.k_cache, case.v_cache
+    tab = case.block_tables
+    tab2 = torch.where(tab >= 0, perm[tab.clamp(min=0).long()].to(torch.int32), tab)
+    out2 = torch.empty_like(out1)
+    pa.pa_decode(out2, case.q, kc2, vc2, tab2, case.context_lens, case.max_context_len, case.scale, AUTO, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out1.float()).all()
+    assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
+    counters = ws[: case.B * case.h_q * 4].view(torch.int32)
+    assert int(counters.abs().sum()) == 0
