@@ -53,6 +53,7 @@ def parse_args(argv=None):
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--warm-l2", action="store_true", help="do not flush L2 between steps")
     return ap.parse_args(argv)
 
 
@@ -107,6 +108,22 @@ def partition_kernel_bytes(case) -> int:
     ctx = case.context_lens.to("cpu").tolist()
     blocks = sum(-(-c // case.bs) for c in ctx)
     return kv_bytes(case) + case.B * case.h_q * case.d * 2 + 4 * blocks + 4 * case.B
+
+
+def ctx_desc(case) -> str:
+    c = workloads_configs()[case.name]
+    if "ctx_range" in c:
+        return "U{%d..%d} incl. appended token" % tuple(c["ctx_range"])
+    if "ctx_fixed" in c:
+        return "%d incl. appended token" % c["ctx_fixed"]
+    if "tail_range" in c:
+        return "%d-token shared prompt + U{%d..%d} private tail + 1" % ((c["prompt_len"],) + tuple(c["tail_range"]))
+    return str(case.context_lens.tolist())
+
+
+def workloads_configs():
+    import workloads
+    return workloads.CONFIGS
 
 
 def measured_peaks():
@@ -206,12 +223,24 @@ def run_ours(args):
     dist = init_dist(world, "nccl")
     seed = shard_seeds(args.seed, world)[rank]
     case = workloads.make_case(args.workload, seed, device=dev)
-    if case.cache == "e4m3":
-        raise SystemExit("bench.py times the bf16 workloads; E4M3 runs go through tests")
     P = case.partition if args.partition is None else args.partition
     B, h_q, d = case.B, case.h_q, case.d
     mcl = case.max_context_len
-    kc, vc = case.k_cache, case.v_cache
+    per_head = case.per_head_scales
+    if per_head:
+        ks_dev, vs_dev = case.k_scale.to(dev), case.v_scale.to(dev)
+        ks_arg, vs_arg = 1.0, 1.0                      # placeholders of the per-tensor arguments
+    else:
+        ks_arg, vs_arg = case.k_scale, case.v_scale
+    if case.quantised:
+        # quantise the cached tokens into code pools with the library's own cache write
+        # (outside the timed region); the step then writes and quantises the appended tokens
+        kc, vc = workloads.empty_quant_pool(case, dev)
+        pa.pa_reshape_and_cache(case.fill_k_rows, case.fill_v_rows, kc, vc, case.fill_slots,
+                                *((ks_dev, vs_dev) if per_head else (ks_arg, vs_arg)))
+        case.fill_k_rows = case.fill_v_rows = None
+    else:
+        kc, vc = case.k_cache, case.v_cache
     q, k_new, v_new = case.q, case.key_new, case.value_new
     slots, tables, ctx = case.slot_mapping, case.block_tables, case.context_lens
     out = torch.empty((B, h_q, d), dtype=torch.bfloat16, device=dev)
@@ -224,15 +253,26 @@ def run_ours(args):
     # so that the host stays ahead of the GPU
     L = pa.lib()
     sp = stream.cuda_stream
-    rargs = pa.reshape_call_args(k_new, v_new, kc, vc, slots)
-    dargs = pa.decode_call_args(out, q, kc, vc, tables, ctx, mcl, case.scale, P, workspace=ws)
+    rargs = pa.reshape_call_args(k_new, v_new, kc, vc, slots, ks_arg, vs_arg)
+    dargs = pa.decode_call_args(out, q, kc, vc, tables, ctx, mcl, case.scale, P, ks_arg, vs_arg, workspace=ws)
     margs = pa.merge_call_args(out, ctx, mcl, P, ws)
+    if per_head:
+        # per-KV-head scales: the *_head_scales calls (their decode call includes the merge
+        # pass, which launches nothing while every group has at most 16 partitions)
+        hp = (ks_dev.data_ptr(), vs_dev.data_ptr())
+        write_call = lambda ra, s_: L.pa_reshape_and_cache_head_scales(*ra[:-2], *hp, s_)
+        part_call = lambda da, s_: L.pa_decode_head_scales(*da[:16], *hp, *da[18:], s_)
+        decode_call = part_call
+    else:
+        write_call = lambda ra, s_: L.pa_reshape_and_cache(*ra, s_)
+        part_call = lambda da, s_: L.pa_decode_partitions(*da, s_)
+        decode_call = lambda da, s_: L.pa_decode(*da, s_)
 
     def step(evs=None):
         if evs:
             evs[0].record(stream)
-        rc = L.pa_reshape_and_cache(*rargs, sp)
-        rc |= L.pa_decode_partitions(*dargs, sp)
+        rc = write_call(rargs, sp)
+        rc |= part_call(dargs, sp)
         rc |= L.pa_decode_merge(*margs, sp)
         if evs:
             evs[1].record(stream)
@@ -249,7 +289,8 @@ def run_ours(args):
         torch.cuda.nvtx.range_push(nvtx)
         with torch.cuda.stream(stream):
             for i in range(args.steps):
-                flush.zero_()
+                if not args.warm_l2:
+                    flush.zero_()
                 body(evs[i])
         torch.cuda.synchronize(dev)
         torch.cuda.nvtx.range_pop()
@@ -281,14 +322,15 @@ def run_ours(args):
             if rc:
                 raise SystemExit("library call failed: %d" % rc)
         return body
-    write_ms = timed(only(L.pa_reshape_and_cache, rargs), 2, "kernel_write")[0]
-    part_ms = timed(only(L.pa_decode_partitions, dargs), 2, "kernel_decode")[0]
+    write_ms = timed(only(lambda *a: write_call(a[:-1], a[-1]), rargs), 2, "kernel_write")[0]
+    part_ms = timed(only(lambda *a: part_call(a[:-1], a[-1]), dargs), 2, "kernel_decode")[0]
+    merge_launches = P > 0 and -(-mcl // P) > 16
+    merge_ms = timed(only(L.pa_decode_merge, margs), 2, "kernel_merge")[0] if merge_launches else 0.0
     t2 = time.time()
     time.sleep(0.1)
     sampler.stop()
     clocks = sampler.summary(t0, t1)
     clocks_kernels = sampler.summary(t1, t2)
-    merge_ms = 0.0
 
     # end to end through the public calls: pinned host inputs in, result out, every step
     e2e = None
@@ -309,13 +351,14 @@ def run_ours(args):
         out_host = torch.empty((B, h_q, d), dtype=torch.bfloat16).pin_memory()
         h2d = sum(t.numel() * t.element_size() for _, t in parts)
         d2h = out_host.numel() * out_host.element_size()
-        e_rargs = pa.reshape_call_args(dv["k_new"], dv["v_new"], kc, vc, dv["slots"])
-        e_dargs = pa.decode_call_args(out, dv["q"], kc, vc, dv["tables"], dv["ctx"], mcl, case.scale, P, workspace=ws)
+        e_rargs = pa.reshape_call_args(dv["k_new"], dv["v_new"], kc, vc, dv["slots"], ks_arg, vs_arg)
+        e_dargs = pa.decode_call_args(out, dv["q"], kc, vc, dv["tables"], dv["ctx"], mcl, case.scale, P,
+                                      ks_arg, vs_arg, workspace=ws)
 
         def e2e_step():
             dev_buf.copy_(host_buf, non_blocking=True)
-            rc = L.pa_reshape_and_cache(*e_rargs, sp)
-            rc |= L.pa_decode(*e_dargs, sp)
+            rc = write_call(e_rargs, sp)
+            rc |= decode_call(e_dargs, sp)
             out_host.copy_(out, non_blocking=True)
             if rc:
                 raise SystemExit("library call failed: %d" % rc)
@@ -332,7 +375,8 @@ def run_ours(args):
         torch.cuda.nvtx.range_push("timed_e2e")
         with torch.cuda.stream(stream):
             for i in range(args.steps):
-                flush.zero_()
+                if not args.warm_l2:
+                    flush.zero_()
                 eev[i][0].record(stream)
                 e2e_step()
                 eev[i][1].record(stream)
@@ -356,6 +400,14 @@ def run_ours(args):
 
     K = args.steps
     per_step_s = step_ms / 1e3 / K
+    if case.cache == "e4m3" and os.environ.get("PA_DECODE_E4M3_CUDA_CORES") == "1":
+        kernel = "paged_decode_partition_kernel (E4M3, CUDA cores)"
+    elif case.quantised:
+        kernel = "paged_decode_partition_mma_quant_kernel (%s codes -> fp16, tensor cores)" % case.cache.upper()
+    elif P == -1:
+        kernel = "paged_decode_balanced_kernel"
+    else:
+        kernel = "paged_decode_partition_mma_kernel"
     value = tot_bytes / per_step_s / 1e9
     peak, peak_kind = measured_peaks()
     part_bytes = partition_kernel_bytes(case)
@@ -371,13 +423,15 @@ def run_ours(args):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": "bf16 q/out, %s KV, fp32 accumulate" % case.cache,
         "data": "synthetic",
         "config": {"workload": args.workload, "num_seqs": B, "h_q": h_q, "h_kv": case.h_kv, "head_dim": d,
-                   "block_size": case.bs, "ctx": "U{512..4096} incl. appended token", "partition": P,
+                   "block_size": case.bs, "ctx": ctx_desc(case), "partition": P,
                    "num_blocks": case.num_blocks, "kv_bytes_per_step_per_gpu": my_bytes,
-                   "step": "reshape_and_cache(64 new tokens) + split-context decode with in-kernel merge",
-                   "l2": "flushed between steps (2x L2 write, outside the events)",
+                   "step": "reshape_and_cache(%d new tokens) + split-context decode with in-kernel merge" % B,
+                   "scales": ("per KV head" if case.per_head_scales else "per tensor") if case.quantised else None,
+                   "l2": ("warm: no flush between steps" if args.warm_l2 else
+                          "flushed between steps (2x L2 write, outside the events)"),
                    "parallelism": "replicas (weak scaling, no collective)" if world > 1 else "single GPU"},
         "tokens_per_s": round(tot_seqs / per_step_s, 1),
         "pct_of_hbm_peak": round(value / world / peak, 4),
@@ -386,14 +440,20 @@ def run_ours(args):
                              "decode (partitions + in-kernel merge)": round(part_ms / K, 5),
                              "note": "each kernel timed alone over K launches after the timed steps; "
                                      "an empty CUDA-event pair reads ~2.7 us and is included"},
-        "roofline": {"bound": "hbm", "kernel": "paged_decode_partition_mma_kernel", "achieved": round(achieved, 1),
+        "roofline": {"bound": "hbm", "kernel": kernel, "achieved": round(achieved, 1),
                      "peak": peak, "peak_kind": peak_kind + " (hbm_gbs copy bandwidth)", "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": ncu_traffic_per_launch(),
+                     "frac": round(achieved / peak, 4),
+                     "traffic": ncu_traffic_per_launch() if (args.workload, P) == ("llama3_8b_b64", 512) else None,
                      "algorithmic_bytes_per_launch": part_bytes},
         "gpu_launches": K * (2 + (1 if P > 0 and -(-mcl // P) > 16 else 0)),
         "clocks": clocks,
         "clocks_kernel_loops": clocks_kernels,
     }
+    if merge_launches:
+        line["kernels_ms_alone"]["merge"] = round(merge_ms / K, 5)
+    if "unique_tokens" in case.meta:      # shared prompts: bytes that are distinct in memory
+        ub = case.meta["unique_tokens"] * case.h_kv * d * case.elem_bytes * 2
+        line["unique_kv_GBs"] = round(ub * world / per_step_s / 1e9, 2)
     if e2e:
         line["e2e"] = {"value": round(tot_bytes / (e2e_ms / 1e3 / K) / 1e9, 2), "unit": "GB/s",
                        "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
@@ -405,20 +465,48 @@ def run_ours(args):
     return line
 
 
+def oracle_step_state(case, orc):
+    """The oracle's caches before the step (quantised by the oracle itself for E4M3 / INT8 caches,
+    untimed) and the keyword arguments of its calls."""
+    import numpy as np
+    import torch
+    import workloads
+    u16 = lambda t: t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+    ks, vs = case.k_scale, case.v_scale
+    if case.per_head_scales:
+        ks, vs = ks.numpy(), vs.numpy()
+    kw = dict(h_kv=case.h_kv, bs=case.bs, cache=case.cache, k_scale=ks, v_scale=vs)
+    if case.quantised:
+        shape = (case.num_blocks, case.h_kv, case.bs, case.d)
+        if case.cache == "int8":
+            kc = np.full(shape, workloads.INT8_UNUSED, np.int8)
+        else:
+            kc = np.full(shape, workloads.E4M3_NAN, np.uint8)
+        vc = kc.copy()
+        orc.reshape_and_cache(u16(case.fill_k_rows), u16(case.fill_v_rows), kc, vc, case.fill_slots.cpu().numpy(),
+                              d=case.d, num_blocks=case.num_blocks, **kw)
+    else:
+        kc, vc = u16(case.k_cache).copy(), u16(case.v_cache).copy()
+    return kc, vc, kw
+
+
 def cpu_baseline(case):
     """The oracle as it stands, single-threaded, on the host: the whole step (cache write of the
     appended tokens and every (sequence, query head) row of the decode), once."""
     import numpy as np
     import torch
     import oracle
+    import workloads
     orc = oracle.load()
     u16 = lambda t: t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
-    kc, vc = u16(case.k_cache).copy(), u16(case.v_cache).copy()
+    if case.quantised:            # the bench's own copy dropped the fill rows: draw them again
+        case = workloads.make_case(case.name, case.meta["seed"])
+    kc, vc, kw = oracle_step_state(case, orc)
     q, kn, vn = u16(case.q), u16(case.key_new), u16(case.value_new)
     tab, ctx, sl = case.block_tables.cpu().numpy(), case.context_lens.cpu().numpy(), case.slot_mapping.cpu().numpy()
     t0 = time.perf_counter()
-    orc.reshape_and_cache(kn, vn, kc, vc, sl, h_kv=case.h_kv, d=case.d, bs=case.bs, num_blocks=case.num_blocks)
-    orc.paged_decode(q, kc, vc, tab, ctx, h_kv=case.h_kv, bs=case.bs, scale=case.scale)
+    orc.reshape_and_cache(kn, vn, kc, vc, sl, d=case.d, num_blocks=case.num_blocks, **kw)
+    orc.paged_decode(q, kc, vc, tab, ctx, scale=case.scale, **kw)
     dt = time.perf_counter() - t0
     return {"value": round(kv_bytes(case) / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
             "seconds": round(dt, 2), "host_cpus": os.cpu_count(),
@@ -439,20 +527,20 @@ def run_reference(args):
     orc = oracle.load()
     case = workloads.make_case(args.workload, args.seed)
     u16 = lambda t: t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
-    kc, vc = u16(case.k_cache).copy(), u16(case.v_cache).copy()
+    kc, vc, kw = oracle_step_state(case, orc)
     q, kn, vn = u16(case.q), u16(case.key_new), u16(case.value_new)
     tab, ctx, sl = case.block_tables.numpy(), case.context_lens.numpy(), case.slot_mapping.numpy()
-    orc.reshape_and_cache(kn, vn, kc, vc, sl, h_kv=case.h_kv, d=case.d, bs=case.bs, num_blocks=case.num_blocks)
+    orc.reshape_and_cache(kn, vn, kc, vc, sl, d=case.d, num_blocks=case.num_blocks, **kw)
     g = case.h_q // case.h_kv
     all_rows = [(s, h) for s in range(case.B) for h in range(case.h_q)]
-    kw = dict(h_kv=case.h_kv, bs=case.bs, scale=case.scale)
+    kw["scale"] = case.scale
     t = time.perf_counter()
     orc.paged_decode_rows(all_rows[:4], q, kc, vc, tab, ctx, **kw)
     per_row = (time.perf_counter() - t) / 4
     budget = 90.0 / max(1, args.steps + args.warmup)              # whole run within a few minutes
     n_rows = int(max(1, min(len(all_rows), budget / max(per_row, 1e-6))))
     pos = 0
-    row_bytes = lambda r: int(ctx[r[0]]) * case.d * 2 * 2 / g      # 1/g of the KV head's bytes
+    row_bytes = lambda r: int(ctx[r[0]]) * case.d * case.elem_bytes * 2 / g   # 1/g of the KV head's bytes
 
     def take():
         nonlocal pos
@@ -475,7 +563,7 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(tot_s / args.steps * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": args.workload, "num_seqs": case.B, "h_q": case.h_q, "h_kv": case.h_kv,
-                       "head_dim": case.d, "block_size": case.bs, "ctx": "U{512..4096} incl. appended token"},
+                       "head_dim": case.d, "block_size": case.bs, "ctx": ctx_desc(case), "kv_cache": case.cache},
             "cpu_baseline": {"value": round(value, 5), "unit": "GB/s", "cores": 1, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": round(value, 5), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}

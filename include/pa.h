@@ -27,9 +27,11 @@
  *     launched when an argument check fails.  No exception crosses the ABI.
  *   - Cache layout: k_cache and v_cache are [num_blocks][h_kv][block_size]
  *     [head_dim], row-major; each (block, head) tile is one contiguous span
- *     of block_size*head_dim elements.  Elements are bf16 (PA_CACHE_BF16) or
- *     OCP FP8 E4M3 bytes (PA_CACHE_E4M3) dequantised as code * scale with one
- *     fp32 scale per tensor.
+ *     of block_size*head_dim elements.  Elements are bf16 (PA_CACHE_BF16),
+ *     OCP FP8 E4M3 bytes (PA_CACHE_E4M3) or symmetric INT8 codes
+ *     (PA_CACHE_INT8, -127..127), a quantised element being worth code * scale
+ *     with one fp32 scale per tensor (the calls below) or per KV head (the
+ *     *_head_scales calls).
  *   - Supported shapes: head_dim in {64, 128}; block_size in {16, 32, 64};
  *     h_q / h_kv in {1, 2, 4, 8}.  Query head h reads KV head
  *     h / (h_q / h_kv) (contiguous groups).
@@ -63,7 +65,7 @@ extern "C" {
 #define PA_DEVERR_BAD_PAIR  0x4u  /* a copy pair outside the pool was skipped */
 #define PA_DEVERR_TIMEOUT   0x8u  /* a bounded in-kernel wait ran out */
 
-typedef enum { PA_CACHE_BF16 = 0, PA_CACHE_E4M3 = 1 } pa_cache_dtype;
+typedef enum { PA_CACHE_BF16 = 0, PA_CACHE_E4M3 = 1, PA_CACHE_INT8 = 2 } pa_cache_dtype;
 
 /* partition_size value of pa_decode: balanced split (see pa_decode) */
 #define PA_PARTITION_AUTO (-1)
@@ -93,12 +95,32 @@ size_t pa_kv_bytes_per_token(int layers, int h_kv, int head_dim, int elem_bytes)
  *   cache_dtype    PA_CACHE_BF16: bits are copied unchanged.
  *                  PA_CACHE_E4M3: code = RNE-satfinite(x / scale) with an IEEE
  *                  fp32 division ("深度解构…" section 3.2, FP8 KV cache)
- *   k_scale/v_scale per-tensor fp32 scales (E4M3 only; must be > 0 and finite)
+ *                  PA_CACHE_INT8: code = the integer nearest to x / scale (ties
+ *                  to even, IEEE fp32 division) limited to [-127, 127]; NaN
+ *                  gives 0 ("深度解构…" section 4 item 1 and "现代 AI…" section
+ *                  3.C: INT8 KV quantisation)
+ *   k_scale/v_scale per-tensor fp32 scales (quantised caches only; must be > 0
+ *                  and finite)
  * Bit-exact by construction: no arithmetic other than the quantisation. */
 int pa_reshape_and_cache(const void *key, const void *value, int64_t key_stride, int64_t value_stride,
                          void *k_cache, void *v_cache, const int64_t *slot_mapping, int num_tokens,
                          int h_kv, int head_dim, int block_size, int num_blocks,
                          int cache_dtype, float k_scale, float v_scale, void *stream);
+
+/* pa_reshape_and_cache with one scale per KV head: KV head h is quantised with
+ * k_scales[h] (resp. v_scales[h]).  The pages name KV quantisation but fix no
+ * scale granularity; this is the finer of the two readings (per tensor, per
+ * head) and reduces to the per-tensor call when all scales are equal.
+ *   cache_dtype    PA_CACHE_E4M3 or PA_CACHE_INT8 (bf16 -> PA_ERR_INVALID_ARG)
+ *   k_scales/v_scales device fp32 [h_kv], each > 0 and finite (not checked on
+ *                  the host: the values are never read there); owned by the
+ *                  caller and read by the kernel, so they must stay valid until
+ *                  the call has run on the stream. */
+int pa_reshape_and_cache_head_scales(const void *key, const void *value, int64_t key_stride,
+                                     int64_t value_stride, void *k_cache, void *v_cache,
+                                     const int64_t *slot_mapping, int num_tokens, int h_kv, int head_dim,
+                                     int block_size, int num_blocks, int cache_dtype, const float *k_scales,
+                                     const float *v_scales, void *stream);
 
 /* ---- decode attention ----------------------------------------------------
  * One decode step: for sequence s and query head h,
@@ -137,8 +159,12 @@ int pa_reshape_and_cache(const void *key, const void *value, int64_t key_stride,
  * Groups (sequence, KV head) of at most 16 partitions are merged inside the
  * first pass by the CTA that finishes the group last; pa_decode launches the
  * merge pass only when a group can have more partitions. 
- * Accuracy: fp32 accumulation; vs an fp64 evaluation of the same formula,
- * max|err| <= 2e-2 and <= 1e-2 * max|ref| for bf16 caches, <= 6e-2 for E4M3. */
+ * Quantised caches (E4M3, INT8) are converted to fp16 in shared memory (both
+ * code sets are exact there) and attended on the tensor cores; the K scale is
+ * folded into the logit scale and the V scale into the output.
+ * Accuracy: fp32 accumulation; vs an fp64 evaluation of the same formula over
+ * the cache contents, max|err| <= 2e-2 and <= 1e-2 * max|ref| for bf16 and INT8
+ * caches, <= 6e-2 for E4M3. */
 size_t pa_decode_workspace_size(int num_seqs, int h_q, int head_dim, int max_context_len,
                                 int partition_size);
 
@@ -162,6 +188,18 @@ int pa_decode_partitions(void *out, const void *q, const void *k_cache, const vo
 int pa_decode_merge(void *out, const int32_t *context_lens, int num_seqs, int max_context_len, int h_q,
                     int head_dim, int partition_size, const void *workspace, size_t workspace_bytes,
                     void *stream);
+
+/* pa_decode over a quantised cache with one scale per KV head (the scales the
+ * cache was written with by pa_reshape_and_cache_head_scales): KV head k's
+ * elements are worth code * k_scales[k] (resp. v_scales[k]).  Same arguments
+ * and result as pa_decode otherwise; cache_dtype must be PA_CACHE_E4M3 or
+ * PA_CACHE_INT8.  k_scales/v_scales: device fp32 [h_kv], owned by the caller. */
+int pa_decode_head_scales(void *out, const void *q, const void *k_cache, const void *v_cache,
+                          const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
+                          int num_seqs, int max_context_len, int h_q, int h_kv, int head_dim, int block_size,
+                          int num_blocks, float scale, int cache_dtype, const float *k_scales,
+                          const float *v_scales, int partition_size, void *workspace, size_t workspace_bytes,
+                          void *stream);
 
 /* ---- decode without any allocation (static scratch) ---------------------------
  * The pages have no counterpart for this call; it exists for callers that cannot

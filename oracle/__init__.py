@@ -46,6 +46,26 @@ def _stale(src: Path, out: Path) -> bool:
 
 _cache: dict[str, "Oracle"] = {}
 
+CACHE_CODES = {"bf16": 0, "e4m3": 1, "int8": 2}
+
+
+def _cache_code(cache: str | None, fp8: bool) -> int:
+    if cache is None:
+        cache = "e4m3" if fp8 else "bf16"
+    if cache not in CACHE_CODES:
+        raise ValueError("unknown cache type %r" % (cache,))
+    return CACHE_CODES[cache]
+
+
+def _head_scales(scale, h_kv: int) -> np.ndarray:
+    """fp32 [h_kv]: a scalar is the per-tensor case (the same scale for every KV head)."""
+    a = np.asarray(scale, dtype=np.float32).reshape(-1)
+    if a.size == 1:
+        a = np.full(h_kv, a[0], dtype=np.float32)
+    if a.size != h_kv:
+        raise ValueError("expected one scale or %d per-head scales, got %d" % (h_kv, a.size))
+    return np.ascontiguousarray(a)
+
 
 class Oracle:
     """ctypes façade over one compiled copy of oracle.c (the tests may load a
@@ -62,8 +82,10 @@ class Oracle:
         L.or_e4m3_decode.restype = f64; L.or_e4m3_decode.argtypes = [ctypes.c_uint8]
         L.or_e4m3_encode_satfinite.restype = ctypes.c_uint8; L.or_e4m3_encode_satfinite.argtypes = [f32]
         L.or_div_f32.restype = f32; L.or_div_f32.argtypes = [f32, f32]
+        L.or_int8_encode_sat.restype = ctypes.c_int8; L.or_int8_encode_sat.argtypes = [f32]
+        L.or_int8_decode.restype = f64; L.or_int8_decode.argtypes = [ctypes.c_int8]
         for name in ("or_bf16_decode_n", "or_bf16_encode_rne_n", "or_e4m3_decode_n",
-                     "or_e4m3_encode_satfinite_n"):
+                     "or_e4m3_encode_satfinite_n", "or_int8_encode_sat_n", "or_int8_decode_n"):
             getattr(L, name).restype = None
             getattr(L, name).argtypes = [vp, vp, i64]
         L.or_div_f32_n.restype = None; L.or_div_f32_n.argtypes = [vp, f32, vp, i64]
@@ -71,15 +93,15 @@ class Oracle:
         L.or_kv_bytes_sequence.restype = u64
         L.or_kv_bytes_sequence.argtypes = [i32, u64, i32, i32, i32]
         L.or_reshape_and_cache.restype = i32
-        L.or_reshape_and_cache.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, f32]
+        L.or_reshape_and_cache.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp]
         L.or_copy_blocks.restype = i32
         L.or_copy_blocks.argtypes = [vp, vp, i32, vp, i32, u64, i32]
         L.or_paged_decode.restype = i32
         L.or_paged_decode.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32, i32,
-                                      f64, i32, f64, f64]
+                                      f64, i32, vp, vp]
         L.or_paged_decode_rows.restype = i32
         L.or_paged_decode_rows.argtypes = [vp, vp, i32, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32,
-                                           i32, f64, i32, f64, f64]
+                                           i32, f64, i32, vp, vp]
 
     # -- number formats ---------------------------------------------------
     def bf16_decode(self, bits) -> np.ndarray:
@@ -106,6 +128,18 @@ class Oracle:
         self._L.or_e4m3_encode_satfinite_n(a.ctypes.data, out.ctypes.data, a.size)
         return out
 
+    def int8_encode_sat(self, x) -> np.ndarray:
+        a = np.ascontiguousarray(x, dtype=np.float32)
+        out = np.empty(a.shape, dtype=np.int8)
+        self._L.or_int8_encode_sat_n(a.ctypes.data, out.ctypes.data, a.size)
+        return out
+
+    def int8_decode(self, codes) -> np.ndarray:
+        c = np.ascontiguousarray(codes, dtype=np.int8)
+        out = np.empty(c.shape, dtype=np.float64)
+        self._L.or_int8_decode_n(c.ctypes.data, out.ctypes.data, c.size)
+        return out
+
     def div_f32(self, x, s: float) -> np.ndarray:
         a = np.ascontiguousarray(x, dtype=np.float32)
         out = np.empty(a.shape, dtype=np.float32)
@@ -122,20 +156,24 @@ class Oracle:
 
     # -- cache operations (in place on numpy arrays) -----------------------
     def reshape_and_cache(self, key_bits, value_bits, k_cache, v_cache, slot_mapping, *,
-                          h_kv: int, d: int, bs: int, num_blocks: int, fp8: bool = False,
-                          k_scale: float = 1.0, v_scale: float = 1.0) -> None:
+                          h_kv: int, d: int, bs: int, num_blocks: int, cache: str | None = None,
+                          fp8: bool = False, k_scale=1.0, v_scale=1.0) -> None:
+        """``cache`` is "bf16", "e4m3" or "int8" (``fp8=True`` means "e4m3"); ``k_scale`` /
+        ``v_scale`` are one float (per tensor) or ``h_kv`` floats (per KV head)."""
+        dt = _cache_code(cache, fp8)
         key = np.ascontiguousarray(key_bits, dtype=np.uint16)
         val = np.ascontiguousarray(value_bits, dtype=np.uint16)
         slots = np.ascontiguousarray(slot_mapping, dtype=np.int64)
-        want = np.uint8 if fp8 else np.uint16
+        want = (np.uint16, np.uint8, np.int8)[dt]
         for c in (k_cache, v_cache):
             if c.dtype != want or not c.flags["C_CONTIGUOUS"]:
                 raise TypeError("cache must be a C-contiguous %s array" % np.dtype(want).name)
+        ks, vs = _head_scales(k_scale, h_kv), _head_scales(v_scale, h_kv)
         rc = self._L.or_reshape_and_cache(key.ctypes.data, val.ctypes.data, k_cache.ctypes.data,
                                           v_cache.ctypes.data, slots.ctypes.data, slots.size,
-                                          h_kv, d, bs, num_blocks, int(fp8), k_scale, v_scale)
+                                          h_kv, d, bs, num_blocks, dt, ks.ctypes.data, vs.ctypes.data)
         if rc:
-            raise ValueError("oracle reshape_and_cache: slot outside the pool")
+            raise ValueError("oracle reshape_and_cache failed with code %d" % rc)
 
     def copy_blocks(self, k_caches, v_caches, pairs, *, block_bytes: int, num_blocks: int) -> None:
         n_layers = len(k_caches)
@@ -149,35 +187,39 @@ class Oracle:
 
     # -- decode attention --------------------------------------------------
     def paged_decode(self, q_bits, k_cache, v_cache, block_tables, context_lens, *, h_kv: int,
-                     bs: int, scale: float, fp8: bool = False, k_scale: float = 1.0,
-                     v_scale: float = 1.0) -> np.ndarray:
+                     bs: int, scale: float, cache: str | None = None, fp8: bool = False, k_scale=1.0,
+                     v_scale=1.0) -> np.ndarray:
+        dt = _cache_code(cache, fp8)
         q = np.ascontiguousarray(q_bits, dtype=np.uint16)
         B, h_q, d = q.shape
         tab = np.ascontiguousarray(block_tables, dtype=np.int32)
         ctx = np.ascontiguousarray(context_lens, dtype=np.int32)
         num_blocks = k_cache.shape[0]
+        ks, vs = _head_scales(k_scale, h_kv), _head_scales(v_scale, h_kv)
         out = np.empty((B, h_q, d), dtype=np.float64)
         rc = self._L.or_paged_decode(out.ctypes.data, q.ctypes.data, k_cache.ctypes.data,
                                      v_cache.ctypes.data, tab.ctypes.data, tab.shape[1], ctx.ctypes.data,
-                                     B, h_q, h_kv, d, bs, num_blocks, scale, int(fp8), k_scale, v_scale)
+                                     B, h_q, h_kv, d, bs, num_blocks, scale, dt, ks.ctypes.data, vs.ctypes.data)
         if rc:
             raise ValueError("oracle paged_decode failed with code %d" % rc)
         return out
 
     def paged_decode_rows(self, rows, q_bits, k_cache, v_cache, block_tables, context_lens, *,
-                          h_kv: int, bs: int, scale: float, fp8: bool = False, k_scale: float = 1.0,
-                          v_scale: float = 1.0) -> np.ndarray:
+                          h_kv: int, bs: int, scale: float, cache: str | None = None, fp8: bool = False,
+                          k_scale=1.0, v_scale=1.0) -> np.ndarray:
         """Outputs for the listed (sequence, query head) rows only: [len(rows), d]."""
+        dt = _cache_code(cache, fp8)
         q = np.ascontiguousarray(q_bits, dtype=np.uint16)
         _, h_q, d = q.shape
         pr = np.ascontiguousarray(rows, dtype=np.int32).reshape(-1, 2)
         tab = np.ascontiguousarray(block_tables, dtype=np.int32)
         ctx = np.ascontiguousarray(context_lens, dtype=np.int32)
+        ks, vs = _head_scales(k_scale, h_kv), _head_scales(v_scale, h_kv)
         out = np.empty((pr.shape[0], d), dtype=np.float64)
         rc = self._L.or_paged_decode_rows(out.ctypes.data, pr.ctypes.data, pr.shape[0], q.ctypes.data,
                                           k_cache.ctypes.data, v_cache.ctypes.data, tab.ctypes.data,
                                           tab.shape[1], ctx.ctypes.data, h_q, h_kv, d, bs,
-                                          k_cache.shape[0], scale, int(fp8), k_scale, v_scale)
+                                          k_cache.shape[0], scale, dt, ks.ctypes.data, vs.ctypes.data)
         if rc:
             raise ValueError("oracle paged_decode_rows failed with code %d" % rc)
         return out

@@ -15,8 +15,12 @@
  *  [Evolve]   "现代 AI 的“推理加速之谜”：从 KV Cache 到 PagedAttention 的演进"
  *  [MemMgmt]  "KVCache技术背景与核心挑战 / PageAttention内存管理机制" (intelliparadigm)
  *  [vLLMNote] "vLLM 推理原理 从 KV Cache 到分页与连续批处理"
- * Number formats: bfloat16 (1-8-7, bias 127) and OCP 8-bit float E4M3
- * (1-4-3, bias 7, no infinities, S.1111.111 = NaN, max finite 448).
+ * Number formats: bfloat16 (1-8-7, bias 127), OCP 8-bit float E4M3
+ * (1-4-3, bias 7, no infinities, S.1111.111 = NaN, max finite 448) and
+ * symmetric INT8 (two's complement codes -127..127, value = code x scale).
+ * Cache element types are numbered 0 = bf16, 1 = E4M3, 2 = INT8; a quantised
+ * cache has one fp32 scale per KV head (a per-tensor scale is the case of
+ * equal per-head scales).
  *
  * Pins (what ties each function to something other than itself) live in
  * tests/test_oracle_pins.py; every function below is pinned there.
@@ -104,6 +108,28 @@ float or_div_f32(float x, float s)
     return r;
 }
 
+/* Symmetric INT8 code of a binary32 value: the nearest integer, ties to the
+ * even one, limited to [-127, 127] (-128 is never produced, so the range is
+ * symmetric about zero); NaN gives 0.  The value of a code is code x scale.
+ * [Dissect] section 4 item 1 and [Evolve] section 3.C name INT8 KV
+ * quantisation; the rounding, the symmetric range and the NaN rule are the
+ * readings adopted where the pages give no scheme. */
+int8_t or_int8_encode_sat(float x)
+{
+    if (x != x) return 0;
+    if (x >= 127.0f) return 127;
+    if (x <= -127.0f) return -127;
+    double f = floor((double)x);        /* exact: |x| < 127 */
+    double frac = (double)x - f;        /* exact, in [0, 1) */
+    double r;
+    if (frac > 0.5) r = f + 1.0;
+    else if (frac < 0.5) r = f;
+    else r = (fmod(f, 2.0) == 0.0) ? f : f + 1.0;   /* tie: the even neighbour */
+    return (int8_t)r;
+}
+
+double or_int8_decode(int8_t c) { return (double)c; }
+
 /* ------------------------------------------------------------------------ */
 /* Closed forms                                                              */
 /* ------------------------------------------------------------------------ */
@@ -136,17 +162,21 @@ static size_t cache_index(int64_t blk, int h, int off, int i, int h_kv, int bs, 
 /* Store the new step's K and V rows into their physical slots.
  * A token's slot is phys_block * bs + offset; slot < 0 means "no write"
  * (padding).  bf16 caches receive the input bits unchanged.  E4M3 caches
- * receive enc(x / scale) with an fp32 division and a saturating RNE encode.
+ * receive enc(x / scale) with an fp32 division and a saturating RNE encode;
+ * INT8 caches the same with the INT8 encode.  scale = k_scales[h] (resp.
+ * v_scales[h]) for KV head h; the scale arrays are not read for bf16.
  * [Evolve] section 1 (every step computes only the new token's Q, K, V and
  * keeps K, V in the cache); [vLLMNote] section "KV Cache 缓存的究竟是什么";
- * [Dissect] section 3.2 (FP8 KV cache quantisation).
- * Returns 0, or -1 if a slot lies outside the pool. */
+ * [Dissect] section 3.2 (FP8 KV cache quantisation) and section 4 item 1
+ * (INT8/FP8 KV quantisation).
+ * Returns 0, -1 if a slot lies outside the pool, -5 on an unknown type. */
 int or_reshape_and_cache(const uint16_t *key, const uint16_t *value,
                          void *k_cache, void *v_cache,
                          const int64_t *slot_mapping, int T,
                          int h_kv, int d, int bs, int num_blocks,
-                         int cache_is_e4m3, float k_scale, float v_scale)
+                         int cache_dtype, const float *k_scales, const float *v_scales)
 {
+    if (cache_dtype < 0 || cache_dtype > 2) return -5;
     for (int t = 0; t < T; ++t) {
         int64_t slot = slot_mapping[t];
         if (slot < 0) continue;
@@ -157,11 +187,16 @@ int or_reshape_and_cache(const uint16_t *key, const uint16_t *value,
             for (int i = 0; i < d; ++i) {
                 size_t src = ((size_t)t * h_kv + h) * d + i;
                 size_t dst = cache_index(blk, h, off, i, h_kv, bs, d);
-                if (cache_is_e4m3) {
+                if (cache_dtype == 1) {
                     float kx = (float)or_bf16_decode(key[src]);
                     float vx = (float)or_bf16_decode(value[src]);
-                    ((uint8_t *)k_cache)[dst] = or_e4m3_encode_satfinite(or_div_f32(kx, k_scale));
-                    ((uint8_t *)v_cache)[dst] = or_e4m3_encode_satfinite(or_div_f32(vx, v_scale));
+                    ((uint8_t *)k_cache)[dst] = or_e4m3_encode_satfinite(or_div_f32(kx, k_scales[h]));
+                    ((uint8_t *)v_cache)[dst] = or_e4m3_encode_satfinite(or_div_f32(vx, v_scales[h]));
+                } else if (cache_dtype == 2) {
+                    float kx = (float)or_bf16_decode(key[src]);
+                    float vx = (float)or_bf16_decode(value[src]);
+                    ((int8_t *)k_cache)[dst] = or_int8_encode_sat(or_div_f32(kx, k_scales[h]));
+                    ((int8_t *)v_cache)[dst] = or_int8_encode_sat(or_div_f32(vx, v_scales[h]));
                 } else {
                     ((uint16_t *)k_cache)[dst] = key[src];
                     ((uint16_t *)v_cache)[dst] = value[src];
@@ -197,9 +232,11 @@ int or_copy_blocks(uint8_t *const *k_caches, uint8_t *const *v_caches, int num_l
 /* Decode attention                                                           */
 /* ------------------------------------------------------------------------ */
 
-static double cache_elem(const void *cache, size_t idx, int cache_is_e4m3, double scale)
+/* Value of a cache element: bf16 exactly; a quantised code times its scale. */
+static double cache_elem(const void *cache, size_t idx, int cache_dtype, double scale)
 {
-    if (cache_is_e4m3) return or_e4m3_decode(((const uint8_t *)cache)[idx]) * scale;
+    if (cache_dtype == 1) return or_e4m3_decode(((const uint8_t *)cache)[idx]) * scale;
+    if (cache_dtype == 2) return or_int8_decode(((const int8_t *)cache)[idx]) * scale;
     return or_bf16_decode(((const uint16_t *)cache)[idx]);
 }
 
@@ -208,7 +245,8 @@ static double cache_elem(const void *cache, size_t idx, int cache_is_e4m3, doubl
  * tokens in logical order, each found through the block table:
  * token t lives in physical block table[s][t / bs] at offset t % bs.
  * Query head h reads KV head h / (H_q / H_kv) (contiguous grouping).
- * ctx = 0 gives a zero row.
+ * ctx = 0 gives a zero row.  Quantised caches are read as code x the KV
+ * head's scale (k_scales[kvh], v_scales[kvh]), in fp64.
  * [Evolve] section 1 (Attention(Q,K,V) = softmax(QK^T / sqrt(d_k)) V);
  * [Dissect] section 2.1 (block table: logical -> physical block);
  * [vLLMNote] section "PagedAttention 怎样整理这些缓存" (A's logical blocks map
@@ -222,10 +260,12 @@ static int decode_one(double *out_row, int s, int h,
                       const int32_t *block_tables, int max_blocks_per_seq,
                       const int32_t *context_lens,
                       int h_q, int h_kv, int d, int bs, int num_blocks,
-                      double scale, int cache_is_e4m3, double k_scale, double v_scale)
+                      double scale, int cache_dtype, const float *k_scales, const float *v_scales)
 {
     int g = h_q / h_kv;
     int kvh = h / g;
+    double k_scale = cache_dtype ? (double)k_scales[kvh] : 1.0;
+    double v_scale = cache_dtype ? (double)v_scales[kvh] : 1.0;
     int n = context_lens[s];
     for (int i = 0; i < d; ++i) out_row[i] = 0.0;
     if (n <= 0) return 0;
@@ -243,7 +283,7 @@ static int decode_one(double *out_row, int s, int h,
         double dot = 0.0;
         for (int i = 0; i < d; ++i)
             dot += or_bf16_decode(qrow[i]) *
-                   cache_elem(k_cache, cache_index(phys, kvh, off, i, h_kv, bs, d), cache_is_e4m3, k_scale);
+                   cache_elem(k_cache, cache_index(phys, kvh, off, i, h_kv, bs, d), cache_dtype, k_scale);
         logit[t] = scale * dot;
         if (logit[t] > m) m = logit[t];
     }
@@ -254,7 +294,7 @@ static int decode_one(double *out_row, int s, int h,
         int off = t % bs;
         denom += w;
         for (int i = 0; i < d; ++i)
-            out_row[i] += w * cache_elem(v_cache, cache_index(phys, kvh, off, i, h_kv, bs, d), cache_is_e4m3, v_scale);
+            out_row[i] += w * cache_elem(v_cache, cache_index(phys, kvh, off, i, h_kv, bs, d), cache_dtype, v_scale);
     }
     for (int i = 0; i < d; ++i) out_row[i] /= denom;
     free(logit);
@@ -265,14 +305,15 @@ static int decode_one(double *out_row, int s, int h,
 int or_paged_decode(double *out, const uint16_t *q, const void *k_cache, const void *v_cache,
                     const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
                     int B, int h_q, int h_kv, int d, int bs, int num_blocks,
-                    double scale, int cache_is_e4m3, double k_scale, double v_scale)
+                    double scale, int cache_dtype, const float *k_scales, const float *v_scales)
 {
     if (h_kv <= 0 || h_q % h_kv != 0) return -4;
+    if (cache_dtype < 0 || cache_dtype > 2) return -5;
     for (int s = 0; s < B; ++s)
         for (int h = 0; h < h_q; ++h) {
             int rc = decode_one(out + ((size_t)s * h_q + h) * d, s, h, q, k_cache, v_cache,
                                 block_tables, max_blocks_per_seq, context_lens, h_q, h_kv, d, bs,
-                                num_blocks, scale, cache_is_e4m3, k_scale, v_scale);
+                                num_blocks, scale, cache_dtype, k_scales, v_scales);
             if (rc) return rc;
         }
     return 0;
@@ -284,13 +325,14 @@ int or_paged_decode_rows(double *out, const int32_t *pairs, int npairs,
                          const uint16_t *q, const void *k_cache, const void *v_cache,
                          const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
                          int h_q, int h_kv, int d, int bs, int num_blocks,
-                         double scale, int cache_is_e4m3, double k_scale, double v_scale)
+                         double scale, int cache_dtype, const float *k_scales, const float *v_scales)
 {
     if (h_kv <= 0 || h_q % h_kv != 0) return -4;
+    if (cache_dtype < 0 || cache_dtype > 2) return -5;
     for (int i = 0; i < npairs; ++i) {
         int rc = decode_one(out + (size_t)i * d, pairs[2 * i], pairs[2 * i + 1], q, k_cache, v_cache,
                             block_tables, max_blocks_per_seq, context_lens, h_q, h_kv, d, bs,
-                            num_blocks, scale, cache_is_e4m3, k_scale, v_scale);
+                            num_blocks, scale, cache_dtype, k_scales, v_scales);
         if (rc) return rc;
     }
     return 0;
@@ -311,6 +353,12 @@ void or_e4m3_decode_n(const uint8_t *in, double *out, int64_t n)
 
 void or_e4m3_encode_satfinite_n(const float *in, uint8_t *out, int64_t n)
 { for (int64_t i = 0; i < n; ++i) out[i] = or_e4m3_encode_satfinite(in[i]); }
+
+void or_int8_encode_sat_n(const float *in, int8_t *out, int64_t n)
+{ for (int64_t i = 0; i < n; ++i) out[i] = or_int8_encode_sat(in[i]); }
+
+void or_int8_decode_n(const int8_t *in, double *out, int64_t n)
+{ for (int64_t i = 0; i < n; ++i) out[i] = or_int8_decode(in[i]); }
 
 void or_div_f32_n(const float *x, float s, float *out, int64_t n)
 { for (int64_t i = 0; i < n; ++i) out[i] = or_div_f32(x[i], s); }

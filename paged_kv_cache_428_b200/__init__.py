@@ -30,6 +30,7 @@ LIB_PATH = _PKG / "libpa.so"
 
 PA_CACHE_BF16 = 0
 PA_CACHE_E4M3 = 1
+PA_CACHE_INT8 = 2
 PA_DEVERR_BAD_SLOT = 0x1
 PA_DEVERR_BAD_BLOCK = 0x2
 PA_DEVERR_BAD_PAIR = 0x4
@@ -60,12 +61,16 @@ def _load() -> ctypes.CDLL:
         "pa_version": (i32, []),
         "pa_kv_bytes_per_token": (sz, [i32, i32, i32, i32]),
         "pa_reshape_and_cache": (i32, [vp, vp, i64, i64, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, f32, vp]),
+        "pa_reshape_and_cache_head_scales": (i32, [vp, vp, i64, i64, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp,
+                                                   vp, vp]),
         "pa_decode_workspace_size": (sz, [i32, i32, i32, i32, i32]),
         "pa_decode": (i32, [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32, i32, i32, f32, i32, f32, f32,
                             i32, vp, sz, vp]),
         "pa_decode_partitions": (i32, [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32, i32, i32, f32, i32,
                                        f32, f32, i32, vp, sz, vp]),
         "pa_decode_merge": (i32, [vp, vp, i32, i32, i32, i32, i32, vp, sz, vp]),
+        "pa_decode_head_scales": (i32, [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32, i32, i32, f32, i32,
+                                        vp, vp, i32, vp, sz, vp]),
         "pa_decode_static_ws": (i32, [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32, i32, i32, f32, i32,
                                       f32, f32, i32, vp]),
         "pa_copy_blocks": (i32, [vp, vp, i32, vp, i32, sz, i32, vp]),
@@ -126,12 +131,34 @@ def _need(t: torch.Tensor, name: str, dtypes, ndim: Optional[int] = None, cuda: 
         raise ValueError("%s must be contiguous" % name)
 
 
+CACHE_DTYPES = (torch.bfloat16, torch.uint8, torch.float8_e4m3fn, torch.int8)
+
+
 def cache_dtype_code(cache: torch.Tensor) -> int:
+    """bf16 -> PA_CACHE_BF16; uint8 / float8_e4m3fn (E4M3 codes) -> PA_CACHE_E4M3;
+    int8 (symmetric INT8 codes) -> PA_CACHE_INT8."""
     if cache.dtype == torch.bfloat16:
         return PA_CACHE_BF16
     if cache.dtype in (torch.uint8, torch.float8_e4m3fn):
         return PA_CACHE_E4M3
-    raise TypeError("cache dtype must be bfloat16, uint8 or float8_e4m3fn (E4M3 codes), got %s" % cache.dtype)
+    if cache.dtype == torch.int8:
+        return PA_CACHE_INT8
+    raise TypeError("cache dtype must be bfloat16, uint8 / float8_e4m3fn (E4M3 codes) or int8, got %s"
+                    % cache.dtype)
+
+
+def _head_scales(k_scale, v_scale, h_kv: int):
+    """(k_ptr, v_ptr) of per-KV-head scale tensors, or None for per-tensor float scales."""
+    per_head = [isinstance(x, torch.Tensor) for x in (k_scale, v_scale)]
+    if not any(per_head):
+        return None
+    if not all(per_head):
+        raise TypeError("k_scale and v_scale must both be floats (per tensor) or both tensors (per KV head)")
+    for t, n in ((k_scale, "k_scale"), (v_scale, "v_scale")):
+        _need(t, n, (torch.float32,), 1)
+        if t.shape[0] != h_kv:
+            raise ValueError("%s: expected %d per-head scales, got %d" % (n, h_kv, t.shape[0]))
+    return k_scale.data_ptr(), v_scale.data_ptr()
 
 
 # ----------------------------------------------------------------------------------------------
@@ -148,11 +175,18 @@ def pa_status_str(status: int) -> str:
 
 
 def pa_reshape_and_cache(key: torch.Tensor, value: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
-                         slot_mapping: torch.Tensor, k_scale: float = 1.0, v_scale: float = 1.0,
-                         stream=None) -> None:
-    """key/value bf16 [T, h_kv, d] (rows may be strided in dim 0); caches [NB, h_kv, bs, d]."""
-    args = reshape_call_args(key, value, k_cache, v_cache, slot_mapping, k_scale, v_scale)
-    _check(_lib.pa_reshape_and_cache(*args, _stream_ptr(stream)), "pa_reshape_and_cache")
+                         slot_mapping: torch.Tensor, k_scale=1.0, v_scale=1.0, stream=None) -> None:
+    """key/value bf16 [T, h_kv, d] (rows may be strided in dim 0); caches [NB, h_kv, bs, d].
+    Quantised caches take float scales (per tensor) or CUDA fp32 [h_kv] tensors (per KV head,
+    pa_reshape_and_cache_head_scales)."""
+    heads = _head_scales(k_scale, v_scale, key.shape[1])
+    if heads is None:
+        args = reshape_call_args(key, value, k_cache, v_cache, slot_mapping, k_scale, v_scale)
+        _check(_lib.pa_reshape_and_cache(*args, _stream_ptr(stream)), "pa_reshape_and_cache")
+    else:
+        args = reshape_call_args(key, value, k_cache, v_cache, slot_mapping)[:-2]
+        _check(_lib.pa_reshape_and_cache_head_scales(*args, *heads, _stream_ptr(stream)),
+               "pa_reshape_and_cache_head_scales")
 
 
 def pa_decode_workspace_size(num_seqs: int, h_q: int, head_dim: int, max_context_len: int,
@@ -172,7 +206,7 @@ def _decode_args(out, q, k_cache, v_cache, block_tables, context_lens, max_conte
                  k_scale, v_scale, workspace):
     _need(out, "out", (torch.bfloat16,), 3)
     _need(q, "q", (torch.bfloat16,), 3)
-    _need(k_cache, "k_cache", (torch.bfloat16, torch.uint8, torch.float8_e4m3fn), 4)
+    _need(k_cache, "k_cache", CACHE_DTYPES, 4)
     _need(v_cache, "v_cache", (k_cache.dtype,), 4)
     _need(block_tables, "block_tables", (torch.int32,), 2)
     _need(context_lens, "context_lens", (torch.int32,), 1)
@@ -189,8 +223,12 @@ def _decode_args(out, q, k_cache, v_cache, block_tables, context_lens, max_conte
         ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel()
     return (out.data_ptr(), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_tables.data_ptr(),
             block_tables.shape[1], context_lens.data_ptr(), B, int(max_context_len), h_q, h_kv, d, bs, NB,
-            float(scale), cache_dtype_code(k_cache), float(k_scale), float(v_scale), int(partition_size),
+            float(scale), cache_dtype_code(k_cache), _f(k_scale), _f(v_scale), int(partition_size),
             ws_ptr, ws_bytes)
+
+
+def _f(x) -> float:
+    return 1.0 if isinstance(x, torch.Tensor) else float(x)
 
 
 def decode_call_args(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len: int,
@@ -219,7 +257,7 @@ def reshape_call_args(key, value, k_cache, v_cache, slot_mapping, k_scale: float
     for t, n in ((key, "key"), (value, "value")):
         if t.dtype != torch.bfloat16 or not t.is_cuda or t.dim() != 3 or t.stride(2) != 1 or t.stride(1) != t.shape[2]:
             raise ValueError("%s must be a CUDA bf16 [T, h_kv, d] tensor with packed heads" % n)
-    _need(k_cache, "k_cache", (torch.bfloat16, torch.uint8, torch.float8_e4m3fn), 4)
+    _need(k_cache, "k_cache", CACHE_DTYPES, 4)
     _need(v_cache, "v_cache", (k_cache.dtype,), 4)
     _need(slot_mapping, "slot_mapping", (torch.int64,), 1)
     T, h_kv, d = key.shape
@@ -232,20 +270,29 @@ def reshape_call_args(key, value, k_cache, v_cache, slot_mapping, k_scale: float
 
 
 def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len: int, scale: float = None,
-              partition_size: int = 512, k_scale: float = 1.0, v_scale: float = 1.0,
+              partition_size: int = 512, k_scale=1.0, v_scale=1.0,
               workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """out[s, h] = softmax(scale * q[s, h] . K^T) . V over the paged cache; returns out."""
+    """out[s, h] = softmax(scale * q[s, h] . K^T) . V over the paged cache; returns out.
+    Quantised caches take float scales (per tensor) or CUDA fp32 [h_kv] tensors (per KV head,
+    pa_decode_head_scales)."""
     if workspace is None:
         workspace = make_workspace(q.shape[0], q.shape[1], q.shape[2], max_context_len, partition_size, q.device)
     args = _decode_args(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len, scale,
                         partition_size, k_scale, v_scale, workspace)
-    _check(_lib.pa_decode(*args, _stream_ptr(stream)), "pa_decode")
+    heads = _head_scales(k_scale, v_scale, k_cache.shape[1])
+    if heads is None:
+        _check(_lib.pa_decode(*args, _stream_ptr(stream)), "pa_decode")
+    else:
+        _check(_lib.pa_decode_head_scales(*args[:16], *heads, *args[18:], _stream_ptr(stream)),
+               "pa_decode_head_scales")
     return out
 
 
 def pa_decode_partitions(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len: int,
                          scale: float = None, partition_size: int = 512, k_scale: float = 1.0,
                          v_scale: float = 1.0, workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+    if _head_scales(k_scale, v_scale, k_cache.shape[1]) is not None:
+        raise TypeError("pa_decode_partitions takes per-tensor scales; use pa_decode for per-head scales")
     args = _decode_args(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len, scale,
                         partition_size, k_scale, v_scale, workspace)
     _check(_lib.pa_decode_partitions(*args, _stream_ptr(stream)), "pa_decode_partitions")
@@ -271,6 +318,8 @@ def pa_decode_static_ws(out, q, k_cache, v_cache, block_tables, context_lens, ma
     the library's static per-device array (PA_STATIC_WS_BYTES).  For callers that may not
     allocate device memory where they run.  Calls that can overlap on the GPU race on that
     array; a request needing more scratch than the array raises PagedKVError (workspace)."""
+    if _head_scales(k_scale, v_scale, k_cache.shape[1]) is not None:
+        raise TypeError("pa_decode_static_ws takes per-tensor scales")
     args = _decode_args(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len, scale,
                         partition_size, k_scale, v_scale, None)
     _check(_lib.pa_decode_static_ws(*args[:-2], _stream_ptr(stream)), "pa_decode_static_ws")

@@ -1,6 +1,6 @@
 // cache_ops.cuh -- cache write (reshape_and_cache) and copy-on-write block copy.
 //
-// Both are pure data movement (plus the E4M3 quantisation of the write), bound by
+// Both are pure data movement (plus the E4M3 / INT8 quantisation of the write), bound by
 // latency at decode-step sizes.  Every thread moves one 16-byte chunk, so a warp
 // touches 512 contiguous bytes of a row or block: fully coalesced on both sides.
 #pragma once
@@ -27,7 +27,14 @@ struct CacheWriteParams {
     long long num_slots;     // num_blocks * block_size
     float k_scale;
     float v_scale;
+    const float *k_scales;   // per-KV-head scales [h_kv] (device), or null: k_scale for all
+    const float *v_scales;
 };
+
+__device__ __forceinline__ float head_scale(const float *per_head, float per_tensor, int h)
+{
+    return per_head ? __ldg(per_head + h) : per_tensor;
+}
 
 // bf16 cache: bits copied unchanged.  Thread -> (token, head, K|V, 16-byte chunk).
 template <int D>
@@ -59,10 +66,13 @@ __global__ void __launch_bounds__(256) reshape_and_cache_bf16_kernel(CacheWriteP
     reinterpret_cast<uint4 *>(cache + dst)[chunk] = v;
 }
 
-// E4M3 cache: code = RNE-satfinite(x / scale), x / scale an IEEE fp32 division.
-// Thread -> (token, head, K|V, 8-element chunk): reads 16 bytes, writes 8.
-template <int D>
-__global__ void __launch_bounds__(256) reshape_and_cache_e4m3_kernel(CacheWriteParams p)
+// Quantised caches, 8 elements per thread (reads 16 bytes, writes 8), x / scale an IEEE fp32
+// division with the KV head's scale:
+//   QT = 1 (E4M3): code = RNE-satfinite(x / scale)
+//   QT = 2 (INT8): code = nearest integer of x / scale (ties to even) limited to [-127, 127]
+// Thread -> (token, head, K|V, 8-element chunk).
+template <int D, int QT>
+__global__ void __launch_bounds__(256) reshape_and_cache_quant_kernel(CacheWriteParams p)
 {
     constexpr int CHUNKS = D / 8;
     const long long tid = blockIdx.x * (long long)blockDim.x + threadIdx.x;
@@ -84,7 +94,7 @@ __global__ void __launch_bounds__(256) reshape_and_cache_e4m3_kernel(CacheWriteP
     const long long blk = slot / p.block_size;
     const int off = static_cast<int>(slot % p.block_size);
     const __nv_bfloat16 *src = (is_v ? p.value + t * p.value_stride : p.key + t * p.key_stride) + (size_t)h * D;
-    const float scale = is_v ? p.v_scale : p.k_scale;
+    const float scale = is_v ? head_scale(p.v_scales, p.v_scale, h) : head_scale(p.k_scales, p.k_scale, h);
     const uint4 raw = reinterpret_cast<const uint4 *>(src)[chunk];
     const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
     uint32_t out[2];
@@ -92,9 +102,18 @@ __global__ void __launch_bounds__(256) reshape_and_cache_e4m3_kernel(CacheWriteP
     for (int i = 0; i < 2; ++i) {
         const float2 a = bf16x2_to_float2(w[2 * i]);
         const float2 b = bf16x2_to_float2(w[2 * i + 1]);
-        const uint16_t lo = float2_to_e4m3x2(__fdiv_rn(a.x, scale), __fdiv_rn(a.y, scale));
-        const uint16_t hi = float2_to_e4m3x2(__fdiv_rn(b.x, scale), __fdiv_rn(b.y, scale));
-        out[i] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+        const float x0 = __fdiv_rn(a.x, scale), x1 = __fdiv_rn(a.y, scale);
+        const float x2 = __fdiv_rn(b.x, scale), x3 = __fdiv_rn(b.y, scale);
+        if constexpr (QT == 1) {
+            const uint16_t lo = float2_to_e4m3x2(x0, x1);
+            const uint16_t hi = float2_to_e4m3x2(x2, x3);
+            out[i] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+        } else {
+            out[i] = (static_cast<uint32_t>(float_to_s8_sym(x0)) & 0xffu) |
+                     ((static_cast<uint32_t>(float_to_s8_sym(x1)) & 0xffu) << 8) |
+                     ((static_cast<uint32_t>(float_to_s8_sym(x2)) & 0xffu) << 16) |
+                     (static_cast<uint32_t>(float_to_s8_sym(x3)) << 24);
+        }
     }
     uint8_t *cache = is_v ? p.v_cache : p.k_cache;
     const size_t dst = (((size_t)blk * p.h_kv + h) * p.block_size + off) * (size_t)D;

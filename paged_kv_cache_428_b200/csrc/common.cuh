@@ -157,6 +157,68 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t a)
     return d;
 }
 
+// d = a * b + d with fp16 inputs (same fragment layouts as the bf16 form).
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                              uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Two fp32 -> fp16x2 (round to nearest even); `lo` lands in the low half.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi)
+{
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Two E4M3 codes (low byte first) -> fp16x2, exact.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t v16)
+{
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(static_cast<uint16_t>(v16)));
+    return h2;
+}
+
+// Four INT8 codes (byte 0 first) -> two fp16x2 words, exact.  Each code c is biased to
+// c + 128 (flip of the top bit) and placed as the low mantissa byte of the fp16 1024 + (c + 128)
+// (exponent byte 0x64); subtracting 1152 = 1024 + 128 leaves c.  Every step is exact since
+// all values are integers below 2048.
+__device__ __forceinline__ void s8x4_to_f16x2x2(uint32_t w, uint32_t &lo, uint32_t &hi)
+{
+    const uint32_t u = w ^ 0x80808080u;
+    uint32_t a, b;
+    asm("prmt.b32 %0, %1, %2, 0x4140;" : "=r"(a) : "r"(u), "r"(0x64646464u));
+    asm("prmt.b32 %0, %1, %2, 0x4342;" : "=r"(b) : "r"(u), "r"(0x64646464u));
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(lo) : "r"(a), "r"(0x64806480u));
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(hi) : "r"(b), "r"(0x64806480u));
+}
+
+// Four INT8 codes (byte 0 first) -> fp16 pairs (codes 0, 2) and (codes 1, 3), exact (the
+// same biasing as s8x4_to_f16x2x2, with the other byte pairing).
+__device__ __forceinline__ void s8x4_to_f16x2x2_cross(uint32_t w, uint32_t &even, uint32_t &odd)
+{
+    const uint32_t u = w ^ 0x80808080u;
+    uint32_t a, b;
+    asm("prmt.b32 %0, %1, %2, 0x4240;" : "=r"(a) : "r"(u), "r"(0x64646464u));
+    asm("prmt.b32 %0, %1, %2, 0x4341;" : "=r"(b) : "r"(u), "r"(0x64646464u));
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(even) : "r"(a), "r"(0x64806480u));
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(odd) : "r"(b), "r"(0x64806480u));
+}
+
+// INT8 code of a binary32 value: the nearest integer (ties to even), limited to
+// [-127, 127]; NaN gives 0.
+__device__ __forceinline__ int float_to_s8_sym(float x)
+{
+    if (x != x) return 0;
+    const int r = __float2int_rn(x);
+    return r < -127 ? -127 : (r > 127 ? 127 : r);
+}
+
 // Two fp32 -> bf16x2 (round to nearest even); `lo` lands in the low half.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 {

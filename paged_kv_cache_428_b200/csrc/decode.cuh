@@ -52,9 +52,21 @@ struct DecodeParams {
     int num_blocks;
     int partition_size;            // tokens per partition, 0 = whole context
     int p_max;                     // partitions per sequence in the grid
-    float qk_scale;                // scale * log2(e) (* k_scale for E4M3)
-    float v_scale;                 // 1 for bf16
+    float qk_scale;                // scale * log2(e) (* the per-tensor k_scale of a quantised cache)
+    float v_scale;                 // per-tensor V scale (1 for bf16)
+    const float *k_scales;         // per-KV-head scales [h_kv] of a quantised cache, or null
+    const float *v_scales;         //   (then qk_scale holds no K scale and v_scale is unused)
 };
+
+// Factors of KV head kvh: the K scale folded into the logit scale and the V scale.
+__device__ __forceinline__ float head_k_factor(const DecodeParams &p, int kvh)
+{
+    return p.k_scales ? __ldg(p.k_scales + kvh) : 1.f;
+}
+__device__ __forceinline__ float head_v_scale(const DecodeParams &p, int kvh)
+{
+    return p.v_scales ? __ldg(p.v_scales + kvh) : p.v_scale;
+}
 
 // Groups (sequence, KV head) with at most this many partitions are merged inside the
 // partition kernel by the CTA that finishes last; larger groups go to the merge kernel,
@@ -168,6 +180,7 @@ __device__ __forceinline__ void cta_combine_and_write(const DecodeParams &p, con
 {
     const float *cl = cm + NW * G;
     const float *co = cl + NW * G;
+    const float v_scale = head_v_scale(p, kvh);
     for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
         const int h = idx / D, dd = idx % D;
         float M = -INFINITY;
@@ -184,12 +197,12 @@ __device__ __forceinline__ void cta_combine_and_write(const DecodeParams &p, con
         }
         const size_t qrow = (size_t)seq * p.h_q + (size_t)kvh * G + h;
         if (n_part == 1) {
-            float r = L > 0.f ? (O / L) * p.v_scale : 0.f;
+            float r = L > 0.f ? (O / L) * v_scale : 0.f;
             if (failed) r = __int_as_float(0x7fc00000);
             p.out[qrow * D + dd] = __float2bfloat16_rn(r);
         } else {
             const size_t prow = qrow * p.p_max + part;
-            p.ws_o[prow * D + dd] = failed ? __int_as_float(0x7fc00000) : O * p.v_scale;
+            p.ws_o[prow * D + dd] = failed ? __int_as_float(0x7fc00000) : O * v_scale;
             if (dd == 0) {
                 p.ws_ml[prow * 2] = M;
                 p.ws_ml[prow * 2 + 1] = failed ? __int_as_float(0x7fc00000) : L;
@@ -411,6 +424,7 @@ __global__ void __launch_bounds__(DecodeConfig<D, BS, G, FP8>::THREADS)
         float2 qf[G][S::QD / 2];
         {
             const __nv_bfloat16 *qrow = p.q + ((size_t)seq * p.h_q + (size_t)kvh * G) * D;
+            const float qs = p.qk_scale * head_k_factor(p, kvh);
 #pragma unroll
             for (int h = 0; h < G; ++h) {
 #pragma unroll
@@ -423,7 +437,7 @@ __global__ void __launch_bounds__(DecodeConfig<D, BS, G, FP8>::THREADS)
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             const float2 f = bf16x2_to_float2(w[e]);
-                            qf[h][k * (S::CHUNK / 2) + w8 * 4 + e] = make_float2(f.x * p.qk_scale, f.y * p.qk_scale);
+                            qf[h][k * (S::CHUNK / 2) + w8 * 4 + e] = make_float2(f.x * qs, f.y * qs);
                         }
                     }
                 }
@@ -599,10 +613,13 @@ struct MergeParams {
     int p_max;
 };
 
+// One CTA of 16 warps per (sequence, query head): warp w takes partitions w, w+16, ... with
+// two independent accumulators, so that many partial rows are in flight at once (a group
+// can have hundreds of partitions: 256 for a 131072-token context at 512 tokens each).
 template <int D>
-__global__ void __launch_bounds__(128) paged_decode_merge_kernel(const MergeParams p)
+__global__ void __launch_bounds__(512) paged_decode_merge_kernel(const MergeParams p)
 {
-    constexpr int NWM = 4, DPL = D / 32;
+    constexpr int NWM = 16, DPL = D / 32;
     const int qh = blockIdx.x, seq = blockIdx.y;
     const int ctx = p.context_lens[seq];
     const int n_part = decode_num_partitions(ctx, p.partition_size, p.p_max);
@@ -625,27 +642,42 @@ __global__ void __launch_bounds__(128) paged_decode_merge_kernel(const MergePara
 #pragma unroll
     for (int w = 1; w < NWM; ++w) M = fmaxf(M, red[w]);
 
-    float L = 0.f;
-    float acc[DPL];
+    float L0 = 0.f, L1 = 0.f;
+    float a0[DPL], a1[DPL];
 #pragma unroll
-    for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
-#pragma unroll 4
-    for (int i = warp; i < n_part; i += NWM) {
+    for (int e = 0; e < DPL; ++e) a0[e] = a1[e] = 0.f;
+    int i = warp;
+    for (; i + NWM < n_part; i += 2 * NWM) {
         const float2 mi = *reinterpret_cast<const float2 *>(ml + 2 * i);
-        const float w = exp2f(mi.x - M);
-        L += w * mi.y;
+        const float2 mj = *reinterpret_cast<const float2 *>(ml + 2 * (i + NWM));
         const float *oi = po + (size_t)i * D + lane * DPL;
-        if constexpr (DPL == 4) {
-            const float4 x = *reinterpret_cast<const float4 *>(oi);
-            acc[0] += w * x.x; acc[1] += w * x.y; acc[2] += w * x.z; acc[3] += w * x.w;
-        } else {
-            const float2 x = *reinterpret_cast<const float2 *>(oi);
-            acc[0] += w * x.x; acc[1] += w * x.y;
+        const float *oj = po + (size_t)(i + NWM) * D + lane * DPL;
+        float xi[DPL], xj[DPL];
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) {
+            xi[e] = oi[e];
+            xj[e] = oj[e];
+        }
+        const float wi = exp2f(mi.x - M), wj = exp2f(mj.x - M);
+        L0 += wi * mi.y;
+        L1 += wj * mj.y;
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) {
+            a0[e] += wi * xi[e];
+            a1[e] += wj * xj[e];
         }
     }
-    if (lane == 0) lsum[warp] = L;
+    if (i < n_part) {
+        const float2 mi = *reinterpret_cast<const float2 *>(ml + 2 * i);
+        const float wi = exp2f(mi.x - M);
+        L0 += wi * mi.y;
+        const float *oi = po + (size_t)i * D + lane * DPL;
 #pragma unroll
-    for (int e = 0; e < DPL; ++e) acc_s[warp][lane * DPL + e] = acc[e];
+        for (int e = 0; e < DPL; ++e) a0[e] += wi * oi[e];
+    }
+    if (lane == 0) lsum[warp] = L0 + L1;
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) acc_s[warp][lane * DPL + e] = a0[e] + a1[e];
     __syncthreads();
     if (threadIdx.x < D) {
         float Lt = 0.f, Ot = 0.f;

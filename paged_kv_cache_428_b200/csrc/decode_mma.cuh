@@ -325,3 +325,4 @@ __global__ void __launch_bounds__(MmaDecodeConfig<D, BS, G, NW_, RING_>::THREADS
 }
 
 }  // namespace pa
+

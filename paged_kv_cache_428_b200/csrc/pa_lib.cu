@@ -5,11 +5,13 @@
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
+#include <type_traits>
 
 #include "common.cuh"
 #include "cache_ops.cuh"
 #include "decode.cuh"
 #include "decode_mma.cuh"
+#include "decode_q8.cuh"
 #include "decode_balanced.cuh"
 
 using namespace pa;
@@ -28,6 +30,18 @@ int launch_status()
 bool supported_head_dim(int d) { return d == 64 || d == 128; }
 bool supported_block_size(int bs) { return bs == 16 || bs == 32 || bs == 64; }
 bool supported_group(int g) { return g == 1 || g == 2 || g == 4 || g == 8; }
+
+bool valid_cache_dtype(int t) { return t == PA_CACHE_BF16 || t == PA_CACHE_E4M3 || t == PA_CACHE_INT8; }
+
+// Scales of a quantised cache: per tensor (k_scales == v_scales == null; both floats finite
+// and > 0) or per KV head (both device arrays given; their values are the caller's to check).
+bool valid_scales(int cache_dtype, float k_scale, float v_scale, const float *k_scales, const float *v_scales)
+{
+    if (!valid_cache_dtype(cache_dtype)) return false;
+    if (cache_dtype == PA_CACHE_BF16) return k_scales == nullptr && v_scales == nullptr;
+    if (k_scales != nullptr || v_scales != nullptr) return k_scales != nullptr && v_scales != nullptr;
+    return std::isfinite(k_scale) && std::isfinite(v_scale) && k_scale > 0.f && v_scale > 0.f;
+}
 
 int grid_partitions(int max_context_len, int partition_size)
 {
@@ -93,19 +107,25 @@ EncodeTiledFn encode_tiled()
     return fn;
 }
 
-// The cache viewed as [num_blocks * h_kv * block_size rows][head_dim] bf16; a box is 64
-// elements (128 bytes) by block_size rows, swizzled in 128-byte atoms.
-int make_cache_map(CUtensorMap *map, const void *cache, int num_blocks, int h_kv, int block_size, int head_dim)
+// The cache viewed as [num_blocks * h_kv * block_size rows][head_dim] elements.  bf16: a box is
+// 64 elements (128 bytes) by block_size rows, swizzled in 128-byte atoms (two boxes per row at
+// head_dim 128).  One-byte codes: a box is a whole row (head_dim bytes) by block_size rows,
+// 128-byte swizzle for 128-byte rows, 64-byte swizzle for 64-byte rows.
+int make_cache_map(CUtensorMap *map, const void *cache, int num_blocks, int h_kv, int block_size, int head_dim,
+                   int elem_bytes)
 {
     EncodeTiledFn enc = encode_tiled();
     if (!enc) return PA_ERR_CUDA;
     const cuuint64_t dims[2] = {(cuuint64_t)head_dim, (cuuint64_t)num_blocks * h_kv * block_size};
-    const cuuint64_t strides[1] = {(cuuint64_t)head_dim * 2};
-    const cuuint32_t box[2] = {64, (cuuint32_t)block_size};
+    const cuuint64_t strides[1] = {(cuuint64_t)head_dim * elem_bytes};
+    const cuuint32_t box[2] = {elem_bytes == 2 ? 64u : (cuuint32_t)head_dim, (cuuint32_t)block_size};
     const cuuint32_t estr[2] = {1, 1};
-    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(cache), dims, strides, box, estr,
-                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    const CUtensorMapDataType dt = elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    const CUtensorMapSwizzle sw = (elem_bytes == 1 && head_dim == 64) ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                                       : CU_TENSOR_MAP_SWIZZLE_128B;
+    const CUresult r = enc(map, dt, 2, const_cast<void *>(cache), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? PA_OK : PA_ERR_CUDA;
 }
 
@@ -113,25 +133,26 @@ int make_cache_map(CUtensorMap *map, const void *cache, int num_blocks, int h_kv
 // cache tensors call after call, and encoding costs host time on every launch otherwise.
 struct CachedMap {
     const void *base = nullptr;
-    int num_blocks = 0, h_kv = 0, block_size = 0, head_dim = 0;
+    int num_blocks = 0, h_kv = 0, block_size = 0, head_dim = 0, elem_bytes = 0;
     CUtensorMap map;
 };
 
-int cached_cache_map(CUtensorMap *map, const void *cache, int num_blocks, int h_kv, int block_size, int head_dim)
+int cached_cache_map(CUtensorMap *map, const void *cache, int num_blocks, int h_kv, int block_size, int head_dim,
+                     int elem_bytes = 2)
 {
     constexpr int kSlots = 8;
     static thread_local CachedMap slots[kSlots];
     static thread_local int next = 0;
     for (const CachedMap &c : slots) {
         if (c.base == cache && c.num_blocks == num_blocks && c.h_kv == h_kv && c.block_size == block_size &&
-            c.head_dim == head_dim) {
+            c.head_dim == head_dim && c.elem_bytes == elem_bytes) {
             *map = c.map;
             return PA_OK;
         }
     }
     CachedMap &c = slots[next];
     next = (next + 1) % kSlots;
-    const int rc = make_cache_map(&c.map, cache, num_blocks, h_kv, block_size, head_dim);
+    const int rc = make_cache_map(&c.map, cache, num_blocks, h_kv, block_size, head_dim, elem_bytes);
     if (rc != PA_OK) {
         c.base = nullptr;
         return rc;
@@ -141,6 +162,7 @@ int cached_cache_map(CUtensorMap *map, const void *cache, int num_blocks, int h_
     c.h_kv = h_kv;
     c.block_size = block_size;
     c.head_dim = head_dim;
+    c.elem_bytes = elem_bytes;
     *map = c.map;
     return PA_OK;
 }
@@ -168,55 +190,106 @@ int launch_partition_mma(const DecodeParams &prm, int num_seqs, cudaStream_t st)
     return launch_status();
 }
 
-// bf16 caches run on the tensor cores; PA_DECODE_BF16_CUDA_CORES=1 selects the CUDA-core
-// kernel instead (kept for A/B measurements; read once per process).
+template <int D, int BS, int G, int QT>
+int launch_partition_q8(const DecodeParams &prm, int num_seqs, cudaStream_t st)
+{
+    using C = MmaQ8Config<D, BS, G>;
+    static std::atomic<unsigned long long> smem_set{0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (!(smem_set.load(std::memory_order_acquire) & bit)) {
+        if (cudaFuncSetAttribute(paged_decode_partition_q8_kernel<D, BS, G, QT>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
+            return PA_ERR_CUDA;
+        smem_set.fetch_or(bit, std::memory_order_release);
+    }
+    CUtensorMap mk, mv;
+    int rc = cached_cache_map(&mk, prm.k_cache, prm.num_blocks, prm.h_kv, BS, D, 1);
+    if (rc == PA_OK) rc = cached_cache_map(&mv, prm.v_cache, prm.num_blocks, prm.h_kv, BS, D, 1);
+    if (rc != PA_OK) return rc;
+    const dim3 grid(prm.p_max, prm.h_kv, num_seqs);
+    paged_decode_partition_q8_kernel<D, BS, G, QT><<<grid, C::THREADS, C::SMEM, st>>>(prm, mk, mv);
+    return launch_status();
+}
+
+bool env_flag(const char *name)
+{
+    const char *e = std::getenv(name);
+    return e != nullptr && std::strcmp(e, "1") == 0;
+}
+
+// Both cache types run on the tensor cores; PA_DECODE_BF16_CUDA_CORES=1 and
+// PA_DECODE_E4M3_CUDA_CORES=1 select the CUDA-core kernel instead (kept for A/B
+// measurements; each read once per process).
 bool bf16_on_cuda_cores()
 {
-    static const bool v = [] {
-        const char *e = std::getenv("PA_DECODE_BF16_CUDA_CORES");
-        return e != nullptr && std::strcmp(e, "1") == 0;
-    }();
+    static const bool v = env_flag("PA_DECODE_BF16_CUDA_CORES");
     return v;
 }
 
-template <int D, int BS, bool FP8>
-int dispatch_group(int g, const DecodeParams &prm, int n, cudaStream_t st)
+bool e4m3_on_cuda_cores()
 {
-    if constexpr (!FP8) {
-        if (!bf16_on_cuda_cores()) {
-            switch (g) {
-            case 1: return launch_partition_mma<D, BS, 1>(prm, n, st);
-            case 2: return launch_partition_mma<D, BS, 2>(prm, n, st);
-            case 4: return launch_partition_mma<D, BS, 4>(prm, n, st);
-            case 8: return launch_partition_mma<D, BS, 8>(prm, n, st);
-            default: return PA_ERR_UNSUPPORTED;
-            }
-        }
-    }
+    static const bool v = env_flag("PA_DECODE_E4M3_CUDA_CORES");
+    return v;
+}
+
+// Cache element types of the kernels: 0 = bf16, 1 = E4M3, 2 = INT8 (the pa_cache_dtype values).
+template <class F>
+int switch_group(int g, F &&f)
+{
     switch (g) {
-    case 1: return launch_partition<D, BS, 1, FP8>(prm, n, st);
-    case 2: return launch_partition<D, BS, 2, FP8>(prm, n, st);
-    case 4: return launch_partition<D, BS, 4, FP8>(prm, n, st);
-    case 8: return launch_partition<D, BS, 8, FP8>(prm, n, st);
+    case 1: return f(std::integral_constant<int, 1>{});
+    case 2: return f(std::integral_constant<int, 2>{});
+    case 4: return f(std::integral_constant<int, 4>{});
+    case 8: return f(std::integral_constant<int, 8>{});
     default: return PA_ERR_UNSUPPORTED;
     }
 }
 
-template <int D, bool FP8>
+template <int D, int BS, int QT>
+int dispatch_group(int g, const DecodeParams &prm, int n, cudaStream_t st)
+{
+    return switch_group(g, [&](auto gc) {
+        constexpr int G = decltype(gc)::value;
+        if constexpr (QT == PA_CACHE_BF16) {
+            if (!bf16_on_cuda_cores()) return launch_partition_mma<D, BS, G>(prm, n, st);
+            return launch_partition<D, BS, G, false>(prm, n, st);
+        } else if constexpr (QT == PA_CACHE_E4M3) {
+            if (!e4m3_on_cuda_cores()) return launch_partition_q8<D, BS, G, QT>(prm, n, st);
+            return launch_partition<D, BS, G, true>(prm, n, st);
+        } else {
+            return launch_partition_q8<D, BS, G, QT>(prm, n, st);
+        }
+    });
+}
+
+template <int D, int QT>
 int dispatch_block(int bs, int g, const DecodeParams &prm, int n, cudaStream_t st)
 {
     switch (bs) {
-    case 16: return dispatch_group<D, 16, FP8>(g, prm, n, st);
-    case 32: return dispatch_group<D, 32, FP8>(g, prm, n, st);
-    case 64: return dispatch_group<D, 64, FP8>(g, prm, n, st);
+    case 16: return dispatch_group<D, 16, QT>(g, prm, n, st);
+    case 32: return dispatch_group<D, 32, QT>(g, prm, n, st);
+    case 64: return dispatch_group<D, 64, QT>(g, prm, n, st);
     default: return PA_ERR_UNSUPPORTED;
     }
 }
 
-int dispatch_partition(int d, int bs, int g, bool fp8, const DecodeParams &prm, int n, cudaStream_t st)
+template <int D>
+int dispatch_type(int qt, int bs, int g, const DecodeParams &prm, int n, cudaStream_t st)
 {
-    if (d == 64) return fp8 ? dispatch_block<64, true>(bs, g, prm, n, st) : dispatch_block<64, false>(bs, g, prm, n, st);
-    if (d == 128) return fp8 ? dispatch_block<128, true>(bs, g, prm, n, st) : dispatch_block<128, false>(bs, g, prm, n, st);
+    switch (qt) {
+    case PA_CACHE_BF16: return dispatch_block<D, PA_CACHE_BF16>(bs, g, prm, n, st);
+    case PA_CACHE_E4M3: return dispatch_block<D, PA_CACHE_E4M3>(bs, g, prm, n, st);
+    case PA_CACHE_INT8: return dispatch_block<D, PA_CACHE_INT8>(bs, g, prm, n, st);
+    default: return PA_ERR_INVALID_ARG;
+    }
+}
+
+int dispatch_partition(int d, int bs, int g, int qt, const DecodeParams &prm, int n, cudaStream_t st)
+{
+    if (d == 64) return dispatch_type<64>(qt, bs, g, prm, n, st);
+    if (d == 128) return dispatch_type<128>(qt, bs, g, prm, n, st);
     return PA_ERR_UNSUPPORTED;
 }
 
@@ -352,17 +425,15 @@ int prepare_decode(DecodeParams &prm, void *out, const void *q, const void *k_ca
                    const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
                    int num_seqs, int max_context_len, int h_q, int h_kv, int head_dim, int block_size,
                    int num_blocks, float scale, int cache_dtype, float k_scale, float v_scale,
-                   int partition_size, void *workspace, size_t workspace_bytes)
+                   const float *k_scales, const float *v_scales, int partition_size, void *workspace,
+                   size_t workspace_bytes)
 {
     if (num_seqs < 0 || max_context_len < 0 || h_q <= 0 || h_kv <= 0 || num_blocks <= 0 ||
         max_blocks_per_seq <= 0 || partition_size < PA_PARTITION_AUTO)
         return PA_ERR_INVALID_ARG;
     if (h_q % h_kv != 0) return PA_ERR_INVALID_ARG;
-    if (cache_dtype != PA_CACHE_BF16 && cache_dtype != PA_CACHE_E4M3) return PA_ERR_INVALID_ARG;
     if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
-    if (cache_dtype == PA_CACHE_E4M3 &&
-        !(std::isfinite(k_scale) && std::isfinite(v_scale) && k_scale > 0.f && v_scale > 0.f))
-        return PA_ERR_INVALID_ARG;
+    if (!valid_scales(cache_dtype, k_scale, v_scale, k_scales, v_scales)) return PA_ERR_INVALID_ARG;
     if (!supported_head_dim(head_dim) || !supported_block_size(block_size) || !supported_group(h_q / h_kv))
         return PA_ERR_UNSUPPORTED;
     if (partition_size > 0 && partition_size % block_size != 0) return PA_ERR_INVALID_ARG;
@@ -403,10 +474,84 @@ int prepare_decode(DecodeParams &prm, void *out, const void *q, const void *k_ca
     prm.num_blocks = num_blocks;
     prm.partition_size = need > 0 ? partition_size : 0;
     prm.p_max = need > 0 ? p_max : 1;
-    const float ks = cache_dtype == PA_CACHE_E4M3 ? k_scale : 1.f;
-    prm.qk_scale = scale * kLog2e * ks;
-    prm.v_scale = cache_dtype == PA_CACHE_E4M3 ? v_scale : 1.f;
+    const bool per_tensor = cache_dtype != PA_CACHE_BF16 && k_scales == nullptr;
+    prm.qk_scale = scale * kLog2e * (per_tensor ? k_scale : 1.f);
+    prm.v_scale = per_tensor ? v_scale : 1.f;
+    prm.k_scales = cache_dtype != PA_CACHE_BF16 ? k_scales : nullptr;
+    prm.v_scales = cache_dtype != PA_CACHE_BF16 ? v_scales : nullptr;
     return PA_OK;
+}
+
+// Decode first pass for both scale forms (per tensor: k_scales == v_scales == null).
+int decode_partitions_impl(void *out, const void *q, const void *k_cache, const void *v_cache,
+                           const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
+                           int num_seqs, int max_context_len, int h_q, int h_kv, int head_dim, int block_size,
+                           int num_blocks, float scale, int cache_dtype, float k_scale, float v_scale,
+                           const float *k_scales, const float *v_scales, int partition_size, void *workspace,
+                           size_t workspace_bytes, void *stream)
+{
+    DecodeParams prm{};
+    int rc = prepare_decode(prm, out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                            num_seqs, max_context_len, h_q, h_kv, head_dim, block_size, num_blocks, scale,
+                            cache_dtype, k_scale, v_scale, k_scales, v_scales, partition_size, workspace,
+                            workspace_bytes);
+    if (rc != PA_OK || num_seqs == 0) return rc;
+    if (partition_size == PA_PARTITION_AUTO && balanced_applies(num_seqs, h_q, h_kv, cache_dtype))
+        return dispatch_balanced(head_dim, block_size, h_q / h_kv, prm, num_seqs, bal_layout(num_seqs, h_q, head_dim),
+                                 workspace, static_cast<cudaStream_t>(stream));
+    return dispatch_partition(head_dim, block_size, h_q / h_kv, cache_dtype, prm, num_seqs,
+                              static_cast<cudaStream_t>(stream));
+}
+
+template <int D>
+void launch_reshape(int cache_dtype, unsigned blocks, const CacheWriteParams &p, cudaStream_t st)
+{
+    if (cache_dtype == PA_CACHE_E4M3) reshape_and_cache_quant_kernel<D, 1><<<blocks, 256, 0, st>>>(p);
+    else if (cache_dtype == PA_CACHE_INT8) reshape_and_cache_quant_kernel<D, 2><<<blocks, 256, 0, st>>>(p);
+    else reshape_and_cache_bf16_kernel<D><<<blocks, 256, 0, st>>>(p);
+}
+
+int reshape_impl(const void *key, const void *value, int64_t key_stride, int64_t value_stride, void *k_cache,
+                 void *v_cache, const int64_t *slot_mapping, int num_tokens, int h_kv, int head_dim, int block_size,
+                 int num_blocks, int cache_dtype, float k_scale, float v_scale, const float *k_scales,
+                 const float *v_scales, void *stream)
+{
+    if (num_tokens < 0 || h_kv <= 0 || num_blocks <= 0) return PA_ERR_INVALID_ARG;
+    if (!valid_scales(cache_dtype, k_scale, v_scale, k_scales, v_scales)) return PA_ERR_INVALID_ARG;
+    if (!supported_head_dim(head_dim) || !supported_block_size(block_size)) return PA_ERR_UNSUPPORTED;
+    const int64_t row = (int64_t)h_kv * head_dim;
+    if (key_stride == 0) key_stride = row;
+    if (value_stride == 0) value_stride = row;
+    if (key_stride < row || value_stride < row || key_stride % 8 != 0 || value_stride % 8 != 0)
+        return PA_ERR_INVALID_ARG;
+    if (num_tokens == 0) return PA_OK;
+    if (!key || !value || !k_cache || !v_cache || !slot_mapping) return PA_ERR_INVALID_ARG;
+    if (!aligned16(key) || !aligned16(value) || !aligned16(k_cache) || !aligned16(v_cache))
+        return PA_ERR_INVALID_ARG;
+
+    CacheWriteParams p{};
+    p.key = static_cast<const __nv_bfloat16 *>(key);
+    p.value = static_cast<const __nv_bfloat16 *>(value);
+    p.key_stride = key_stride;
+    p.value_stride = value_stride;
+    p.k_cache = static_cast<uint8_t *>(k_cache);
+    p.v_cache = static_cast<uint8_t *>(v_cache);
+    p.slot_mapping = slot_mapping;
+    p.num_tokens = num_tokens;
+    p.h_kv = h_kv;
+    p.block_size = block_size;
+    p.num_slots = (long long)num_blocks * block_size;
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
+    p.k_scales = k_scales;
+    p.v_scales = v_scales;
+    const long long threads = (long long)num_tokens * h_kv * 2 * (head_dim / 8);
+    const long long blocks = (threads + 255) / 256;
+    if (blocks > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (head_dim == 64) launch_reshape<64>(cache_dtype, (unsigned)blocks, p, st);
+    else launch_reshape<128>(cache_dtype, (unsigned)blocks, p, st);
+    return launch_status();
 }
 
 }  // namespace
@@ -486,16 +631,10 @@ int pa_decode_partitions(void *out, const void *q, const void *k_cache, const vo
                          int num_blocks, float scale, int cache_dtype, float k_scale, float v_scale,
                          int partition_size, void *workspace, size_t workspace_bytes, void *stream)
 {
-    DecodeParams prm{};
-    int rc = prepare_decode(prm, out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
-                            num_seqs, max_context_len, h_q, h_kv, head_dim, block_size, num_blocks, scale,
-                            cache_dtype, k_scale, v_scale, partition_size, workspace, workspace_bytes);
-    if (rc != PA_OK || num_seqs == 0) return rc;
-    if (partition_size == PA_PARTITION_AUTO && balanced_applies(num_seqs, h_q, h_kv, cache_dtype))
-        return dispatch_balanced(head_dim, block_size, h_q / h_kv, prm, num_seqs, bal_layout(num_seqs, h_q, head_dim),
-                                 workspace, static_cast<cudaStream_t>(stream));
-    return dispatch_partition(head_dim, block_size, h_q / h_kv, cache_dtype == PA_CACHE_E4M3, prm, num_seqs,
-                              static_cast<cudaStream_t>(stream));
+    return decode_partitions_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                                  num_seqs, max_context_len, h_q, h_kv, head_dim, block_size, num_blocks, scale,
+                                  cache_dtype, k_scale, v_scale, nullptr, nullptr, partition_size, workspace,
+                                  workspace_bytes, stream);
 }
 
 int pa_decode_merge(void *out, const int32_t *context_lens, int num_seqs, int max_context_len, int h_q,
@@ -525,9 +664,9 @@ int pa_decode_merge(void *out, const int32_t *context_lens, int num_seqs, int ma
     const dim3 grid(h_q, num_seqs);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (head_dim == 64)
-        paged_decode_merge_kernel<64><<<grid, 128, 0, st>>>(mp);
+        paged_decode_merge_kernel<64><<<grid, 512, 0, st>>>(mp);
     else
-        paged_decode_merge_kernel<128><<<grid, 128, 0, st>>>(mp);
+        paged_decode_merge_kernel<128><<<grid, 512, 0, st>>>(mp);
     return launch_status();
 }
 
@@ -546,54 +685,40 @@ int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache
                            workspace, workspace_bytes, stream);
 }
 
+int pa_decode_head_scales(void *out, const void *q, const void *k_cache, const void *v_cache,
+                          const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
+                          int num_seqs, int max_context_len, int h_q, int h_kv, int head_dim, int block_size,
+                          int num_blocks, float scale, int cache_dtype, const float *k_scales,
+                          const float *v_scales, int partition_size, void *workspace, size_t workspace_bytes,
+                          void *stream)
+{
+    if (cache_dtype == PA_CACHE_BF16 || k_scales == nullptr || v_scales == nullptr) return PA_ERR_INVALID_ARG;
+    int rc = decode_partitions_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                                    num_seqs, max_context_len, h_q, h_kv, head_dim, block_size, num_blocks, scale,
+                                    cache_dtype, 1.f, 1.f, k_scales, v_scales, partition_size, workspace,
+                                    workspace_bytes, stream);
+    if (rc != PA_OK) return rc;
+    return pa_decode_merge(out, context_lens, num_seqs, max_context_len, h_q, head_dim, partition_size,
+                           workspace, workspace_bytes, stream);
+}
+
 int pa_reshape_and_cache(const void *key, const void *value, int64_t key_stride, int64_t value_stride,
                          void *k_cache, void *v_cache, const int64_t *slot_mapping, int num_tokens, int h_kv,
                          int head_dim, int block_size, int num_blocks, int cache_dtype, float k_scale,
                          float v_scale, void *stream)
 {
-    if (num_tokens < 0 || h_kv <= 0 || num_blocks <= 0) return PA_ERR_INVALID_ARG;
-    if (cache_dtype != PA_CACHE_BF16 && cache_dtype != PA_CACHE_E4M3) return PA_ERR_INVALID_ARG;
-    if (!supported_head_dim(head_dim) || !supported_block_size(block_size)) return PA_ERR_UNSUPPORTED;
-    const int64_t row = (int64_t)h_kv * head_dim;
-    if (key_stride == 0) key_stride = row;
-    if (value_stride == 0) value_stride = row;
-    if (key_stride < row || value_stride < row || key_stride % 8 != 0 || value_stride % 8 != 0)
-        return PA_ERR_INVALID_ARG;
-    if (cache_dtype == PA_CACHE_E4M3 &&
-        !(std::isfinite(k_scale) && std::isfinite(v_scale) && k_scale > 0.f && v_scale > 0.f))
-        return PA_ERR_INVALID_ARG;
-    if (num_tokens == 0) return PA_OK;
-    if (!key || !value || !k_cache || !v_cache || !slot_mapping) return PA_ERR_INVALID_ARG;
-    if (!aligned16(key) || !aligned16(value) || !aligned16(k_cache) || !aligned16(v_cache))
-        return PA_ERR_INVALID_ARG;
+    return reshape_impl(key, value, key_stride, value_stride, k_cache, v_cache, slot_mapping, num_tokens, h_kv,
+                        head_dim, block_size, num_blocks, cache_dtype, k_scale, v_scale, nullptr, nullptr, stream);
+}
 
-    CacheWriteParams p{};
-    p.key = static_cast<const __nv_bfloat16 *>(key);
-    p.value = static_cast<const __nv_bfloat16 *>(value);
-    p.key_stride = key_stride;
-    p.value_stride = value_stride;
-    p.k_cache = static_cast<uint8_t *>(k_cache);
-    p.v_cache = static_cast<uint8_t *>(v_cache);
-    p.slot_mapping = slot_mapping;
-    p.num_tokens = num_tokens;
-    p.h_kv = h_kv;
-    p.block_size = block_size;
-    p.num_slots = (long long)num_blocks * block_size;
-    p.k_scale = k_scale;
-    p.v_scale = v_scale;
-    const long long threads = (long long)num_tokens * h_kv * 2 * (head_dim / 8);
-    const long long blocks = (threads + 255) / 256;
-    if (blocks > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const bool fp8 = cache_dtype == PA_CACHE_E4M3;
-    if (head_dim == 64) {
-        if (fp8) reshape_and_cache_e4m3_kernel<64><<<(unsigned)blocks, 256, 0, st>>>(p);
-        else     reshape_and_cache_bf16_kernel<64><<<(unsigned)blocks, 256, 0, st>>>(p);
-    } else {
-        if (fp8) reshape_and_cache_e4m3_kernel<128><<<(unsigned)blocks, 256, 0, st>>>(p);
-        else     reshape_and_cache_bf16_kernel<128><<<(unsigned)blocks, 256, 0, st>>>(p);
-    }
-    return launch_status();
+int pa_reshape_and_cache_head_scales(const void *key, const void *value, int64_t key_stride, int64_t value_stride,
+                                     void *k_cache, void *v_cache, const int64_t *slot_mapping, int num_tokens,
+                                     int h_kv, int head_dim, int block_size, int num_blocks, int cache_dtype,
+                                     const float *k_scales, const float *v_scales, void *stream)
+{
+    if (cache_dtype == PA_CACHE_BF16 || k_scales == nullptr || v_scales == nullptr) return PA_ERR_INVALID_ARG;
+    return reshape_impl(key, value, key_stride, value_stride, k_cache, v_cache, slot_mapping, num_tokens, h_kv,
+                        head_dim, block_size, num_blocks, cache_dtype, 1.f, 1.f, k_scales, v_scales, stream);
 }
 
 int pa_copy_blocks(void *const *k_caches, void *const *v_caches, int num_layers, const int64_t *block_pairs,

@@ -9,7 +9,8 @@ import oracle
 import workloads
 import paged_kv_cache_428_b200 as pa
 
-# Tolerances of the decode output against the fp64 oracle (bf16 output, fp32 accumulation)
+# Tolerances of the decode output against the fp64 oracle (bf16 output, fp32 accumulation).
+# bf16 and INT8 caches: 2e-2 absolute and 1e-2 of max|ref|; E4M3: 6e-2 absolute.
 BF16_ABS, BF16_REL = 2e-2, 1e-2
 E4M3_ABS = 6e-2
 
@@ -22,13 +23,35 @@ def u8(t: torch.Tensor) -> np.ndarray:
     return t.detach().contiguous().cpu().view(torch.uint8).numpy()
 
 
-def gpu_fill_e4m3(case, dev="cuda"):
-    """Quantise the case's pre-existing rows into fresh E4M3 pools with pa_reshape_and_cache."""
-    kc, vc = workloads.empty_e4m3_pool(case, dev)
+def codes(t: torch.Tensor, cache: str) -> np.ndarray:
+    """Cache contents as numpy in the oracle's element type (uint16 bits, uint8 or int8 codes)."""
+    if cache == "int8":
+        return t.detach().contiguous().cpu().numpy()
+    return u8(t) if cache == "e4m3" else u16(t)
+
+
+def dev_scales(case, dev="cuda"):
+    """The case's scales as pa_* arguments: floats, or CUDA fp32 [h_kv] tensors per KV head."""
+    if case.per_head_scales:
+        return case.k_scale.to(dev), case.v_scale.to(dev)
+    return case.k_scale, case.v_scale
+
+
+def np_scales(case):
+    """The case's scales as oracle arguments: floats, or fp32 [h_kv] arrays."""
+    if case.per_head_scales:
+        return case.k_scale.numpy(), case.v_scale.numpy()
+    return case.k_scale, case.v_scale
+
+
+def gpu_fill_quant(case, dev="cuda"):
+    """Quantise the case's pre-existing rows into fresh code pools with pa_reshape_and_cache."""
+    kc, vc = workloads.empty_quant_pool(case, dev)
     if case.fill_slots is not None and case.fill_slots.numel():
         pa.pa_reshape_and_cache(case.fill_k_rows.to(dev), case.fill_v_rows.to(dev), kc, vc,
-                                case.fill_slots.to(dev), case.k_scale, case.v_scale)
+                                case.fill_slots.to(dev), *dev_scales(case, dev))
     return kc, vc
+
 
 
 def gpu_step(case, partition_size=None, dev="cuda", max_context_len=None, caches=None):
@@ -36,26 +59,29 @@ def gpu_step(case, partition_size=None, dev="cuda", max_context_len=None, caches
     P = case.partition if partition_size is None else partition_size
     if caches is not None:
         kc, vc = caches
-    elif case.cache == "e4m3":
-        kc, vc = gpu_fill_e4m3(case, dev)
+    elif case.quantised:
+        kc, vc = gpu_fill_quant(case, dev)
     else:
         kc, vc = case.k_cache.to(dev).clone(), case.v_cache.to(dev).clone()
-    pa.pa_reshape_and_cache(case.key_new.to(dev), case.value_new.to(dev), kc, vc, case.slot_mapping.to(dev),
-                            case.k_scale, case.v_scale)
+    ks, vs = dev_scales(case, dev)
+    pa.pa_reshape_and_cache(case.key_new.to(dev), case.value_new.to(dev), kc, vc, case.slot_mapping.to(dev), ks, vs)
     out = torch.empty((case.B, case.h_q, case.d), dtype=torch.bfloat16, device=dev)
     mcl = case.max_context_len if max_context_len is None else max_context_len
     pa.pa_decode(out, case.q.to(dev), kc, vc, case.block_tables.to(dev), case.context_lens.to(dev), mcl,
-                 case.scale, P, case.k_scale, case.v_scale)
+                 case.scale, P, ks, vs)
     return out, kc, vc
 
 
 def oracle_caches(case, orc, seqs=None):
     """The oracle's own caches after the step's writes (numpy, pool layout).  With `seqs`,
     only the rows of those sequences are quantised (the rest keeps the sentinel)."""
-    fp8 = case.cache == "e4m3"
-    if fp8:
+    ks, vs = np_scales(case)
+    if case.quantised:
         shape = (case.num_blocks, case.h_kv, case.bs, case.d)
-        kc = np.full(shape, workloads.E4M3_NAN, np.uint8)
+        if case.cache == "int8":
+            kc = np.full(shape, workloads.INT8_UNUSED, np.int8)
+        else:
+            kc = np.full(shape, workloads.E4M3_NAN, np.uint8)
         vc = kc.copy()
         slots = case.fill_slots.cpu()
         krows, vrows = case.fill_k_rows.cpu(), case.fill_v_rows.cpu()
@@ -64,13 +90,12 @@ def oracle_caches(case, orc, seqs=None):
             keep = torch.tensor([owner.get(int(s) // case.bs, -1) in seqs for s in slots.tolist()], dtype=torch.bool)
             slots, krows, vrows = slots[keep], krows[keep], vrows[keep]
         orc.reshape_and_cache(u16(krows), u16(vrows), kc, vc, slots.numpy(), h_kv=case.h_kv, d=case.d,
-                              bs=case.bs, num_blocks=case.num_blocks, fp8=True, k_scale=case.k_scale,
-                              v_scale=case.v_scale)
+                              bs=case.bs, num_blocks=case.num_blocks, cache=case.cache, k_scale=ks, v_scale=vs)
     else:
         kc, vc = u16(case.k_cache).copy(), u16(case.v_cache).copy()
     orc.reshape_and_cache(u16(case.key_new), u16(case.value_new), kc, vc, case.slot_mapping.cpu().numpy(),
-                          h_kv=case.h_kv, d=case.d, bs=case.bs, num_blocks=case.num_blocks, fp8=fp8,
-                          k_scale=case.k_scale, v_scale=case.v_scale)
+                          h_kv=case.h_kv, d=case.d, bs=case.bs, num_blocks=case.num_blocks, cache=case.cache,
+                          k_scale=ks, v_scale=vs)
     return kc, vc
 
 
@@ -86,8 +111,8 @@ def block_owner(case) -> dict:
 
 
 def oracle_out(case, orc, kc, vc, rows=None):
-    fp8 = case.cache == "e4m3"
-    kw = dict(h_kv=case.h_kv, bs=case.bs, scale=case.scale, fp8=fp8, k_scale=case.k_scale, v_scale=case.v_scale)
+    ks, vs = np_scales(case)
+    kw = dict(h_kv=case.h_kv, bs=case.bs, scale=case.scale, cache=case.cache, k_scale=ks, v_scale=vs)
     q = u16(case.q)
     tab = case.block_tables.cpu().numpy()
     ctx = case.context_lens.cpu().numpy()

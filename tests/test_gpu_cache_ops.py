@@ -5,43 +5,79 @@ import torch
 
 import workloads
 import paged_kv_cache_428_b200 as pa
-from paritylib import u16, u8
+from paritylib import codes, u16, u8
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-def _pool(nb, h_kv, bs, d, fp8):
+def _pool(nb, h_kv, bs, d, cache):
+    """Device pools of the cache type filled with its never-written sentinel."""
     shape = (nb, h_kv, bs, d)
-    if fp8:
+    if cache in (True, "e4m3"):
         return (torch.full(shape, workloads.E4M3_NAN, dtype=torch.uint8, device=DEV),
                 torch.full(shape, workloads.E4M3_NAN, dtype=torch.uint8, device=DEV))
+    if cache == "int8":
+        return (torch.full(shape, workloads.INT8_UNUSED, dtype=torch.int8, device=DEV),
+                torch.full(shape, workloads.INT8_UNUSED, dtype=torch.int8, device=DEV))
     k = torch.full(shape, workloads.BF16_NAN, dtype=torch.int16, device=DEV).view(torch.bfloat16)
     return k, k.clone()
 
 
-@pytest.mark.parametrize("fp8", [False, True])
+@pytest.mark.parametrize("cache,per_head", [("bf16", False), ("e4m3", False), ("int8", False), ("e4m3", True),
+                                            ("int8", True)])
 @pytest.mark.parametrize("d,bs", [(64, 16), (128, 16), (128, 32), (128, 64), (64, 64)])
 @pytest.mark.parametrize("seed", [0, 1, 2])
-def test_reshape_and_cache_bit_exact(orc, fp8, d, bs, seed):
+def test_reshape_and_cache_bit_exact(orc, cache, per_head, d, bs, seed):
     h_kv, nb = 4, 40
     T = 300 if seed else 37                                   # ragged token counts
+    quant = cache != "bf16"
     g = torch.Generator().manual_seed(seed)
-    k_rows = (torch.randn(T, h_kv, d, generator=g) * (30 if fp8 else 1)).to(torch.bfloat16)
-    v_rows = (torch.randn(T, h_kv, d, generator=g) * (30 if fp8 else 1)).to(torch.bfloat16)
+    k_rows = (torch.randn(T, h_kv, d, generator=g) * (30 if quant else 1)).to(torch.bfloat16)
+    v_rows = (torch.randn(T, h_kv, d, generator=g) * (30 if quant else 1)).to(torch.bfloat16)
     slots = torch.randperm(nb * bs, generator=g)[:T].to(torch.int64)
     slots[::7] = -1                                           # padding tokens are skipped
-    ks, vs = (0.05, 0.031) if fp8 else (1.0, 1.0)
-    kc, vc = _pool(nb, h_kv, bs, d, fp8)
+    if per_head:
+        ks_np = np.array([0.05, 0.31, 0.011, 0.9], np.float32)
+        vs_np = np.array([0.2, 0.031, 0.47, 0.07], np.float32)
+        ks, vs = torch.from_numpy(ks_np).to(DEV), torch.from_numpy(vs_np).to(DEV)
+    else:
+        ks_np, vs_np = ks, vs = (0.05, 0.031) if quant else (1.0, 1.0)
+    kc, vc = _pool(nb, h_kv, bs, d, cache)
     pa.pa_reshape_and_cache(k_rows.to(DEV), v_rows.to(DEV), kc, vc, slots.to(DEV), ks, vs)
     torch.cuda.synchronize()
-    conv = u8 if fp8 else u16
-    ok_, ov_ = conv(_pool(nb, h_kv, bs, d, fp8)[0]).copy(), conv(_pool(nb, h_kv, bs, d, fp8)[1]).copy()
+    ok_, ov_ = (codes(t, cache).copy() for t in _pool(nb, h_kv, bs, d, cache))
     orc.reshape_and_cache(u16(k_rows), u16(v_rows), ok_, ov_, slots.numpy(), h_kv=h_kv, d=d, bs=bs, num_blocks=nb,
-                          fp8=fp8, k_scale=ks, v_scale=vs)
-    assert np.array_equal(conv(kc), ok_) and np.array_equal(conv(vc), ov_)
-    if fp8:                                                   # saturation was exercised
-        assert (np.abs(k_rows.float().numpy()) / ks > 448).any()
+                          cache=cache, k_scale=ks_np, v_scale=vs_np)
+    assert np.array_equal(codes(kc, cache), ok_) and np.array_equal(codes(vc, cache), ov_)
+    if quant:                                                 # saturation was exercised
+        qmax = workloads.QUANT_MAX[cache]
+        assert (np.abs(k_rows.float().numpy()) / np.asarray(ks_np).reshape(-1)[:, None] > qmax).any()
+
+
+def test_int8_write_ties_saturation(orc):
+    """scale 1: every bf16 value in [-300, 300] is quantised directly -- exact halves (ties to
+    even), values past +-127 (saturation), -0 and tiny values."""
+    h_kv, d, bs, nb = 2, 64, 16, 64
+    allbits = torch.arange(0, 1 << 16, dtype=torch.int32).to(torch.int16).view(torch.bfloat16)
+    f = allbits.float()
+    vals = allbits[torch.isfinite(f) & (f.abs() <= 300)]
+    per_row = h_kv * d
+    T = -(-vals.numel() // per_row)
+    pad = torch.zeros(T * per_row - vals.numel(), dtype=torch.bfloat16)
+    k_rows = torch.cat([vals, pad]).reshape(T, h_kv, d).contiguous()
+    v_rows = (-k_rows.float()).to(torch.bfloat16).contiguous()
+    assert T <= nb * bs
+    slots = torch.randperm(nb * bs, generator=torch.Generator().manual_seed(2))[:T].to(torch.int64)
+    kc, vc = _pool(nb, h_kv, bs, d, "int8")
+    pa.pa_reshape_and_cache(k_rows.to(DEV), v_rows.to(DEV), kc, vc, slots.to(DEV), 1.0, 1.0)
+    ok_ = np.full((nb, h_kv, bs, d), workloads.INT8_UNUSED, np.int8)
+    ov_ = ok_.copy()
+    orc.reshape_and_cache(u16(k_rows), u16(v_rows), ok_, ov_, slots.numpy(), h_kv=h_kv, d=d, bs=bs, num_blocks=nb,
+                          cache="int8", k_scale=1.0, v_scale=1.0)
+    assert np.array_equal(codes(kc, "int8"), ok_) and np.array_equal(codes(vc, "int8"), ov_)
+    written = ok_[slots.numpy() // bs, :, slots.numpy() % bs, :]
+    assert written.min() == -127 and written.max() == 127          # saturation, never -128
 
 
 def test_e4m3_write_ties_subnormals_saturation(orc):

@@ -1,0 +1,21 @@
+"""The CUDA-core decode kernels (selected by PA_DECODE_BF16_CUDA_CORES=1 and
+PA_DECODE_E4M3_CUDA_CORES=1, read once per process) against the oracle: the shape-grid
+parity tests run again in a child process with both switches set."""
+import os
+import subprocess
+import sys
+from pathlib import Path
+
+import pytest
+
+pytestmark = pytest.mark.gpu
+HERE = Path(__file__).resolve().parent
+
+
+def test_cuda_core_kernels_every_variant():
+    env = dict(os.environ, PA_DECODE_BF16_CUDA_CORES="1", PA_DECODE_E4M3_CUDA_CORES="1")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-m", "gpu", "-p", "no:cacheprovider",
+                        str(HERE / "test_gpu_decode.py"), "-k", "every_kernel_variant or fp8_mha_reduced"],
+                       env=env, cwd=HERE.parent, capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stdout[-4000:] + r.stderr[-2000:]
+    assert " passed" in r.stdout

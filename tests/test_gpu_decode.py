@@ -8,7 +8,7 @@ import torch
 
 import workloads
 import paged_kv_cache_428_b200 as pa
-from paritylib import (check_close, gpu_fill_e4m3, gpu_step, oracle_caches, oracle_out, u16, u8)
+from paritylib import (check_close, codes, gpu_step, oracle_caches, oracle_out, u16, u8)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -19,8 +19,7 @@ def _full_parity(orc, case, rows=None, seqs=None, **kw):
     torch.cuda.synchronize()
     okc, ovc = oracle_caches(case, orc, seqs=seqs)
     if seqs is None:                                       # the step's cache writes are bit-exact
-        conv = u8 if case.cache == "e4m3" else u16
-        assert np.array_equal(conv(kc), okc) and np.array_equal(conv(vc), ovc)
+        assert np.array_equal(codes(kc, case.cache), okc) and np.array_equal(codes(vc, case.cache), ovc)
     ref = oracle_out(case, orc, okc, ovc, rows)
     got = out if rows is None else torch.stack([out[s, h] for s, h in rows])
     return check_close(got, ref, case.cache == "e4m3", case.name)
@@ -81,21 +80,41 @@ def test_fp8_mha_reduced_all_rows(orc, bs, seed):
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("bs", [16, 32, 64])
 @pytest.mark.parametrize("g", [1, 2, 4, 8])
-@pytest.mark.parametrize("cache", ["bf16", "e4m3"])
+@pytest.mark.parametrize("cache", ["bf16", "e4m3", "int8"])
 def test_every_kernel_variant(orc, d, bs, g, cache):
     """Small ragged cases over the whole supported shape grid (each template instance)."""
     h_kv = 2
     case = workloads.make_case("llama3_8b_b64", 7 * d + bs + g, B=5, h_q=h_kv * g, h_kv=h_kv, d=d, bs=bs,
                                ctx_range=(1, 700), pool_factor=1.3, partition=128 if bs <= 64 else 0)
-    if cache == "e4m3":
-        case = _as_e4m3(case)
+    if cache != "bf16":
+        case = _as_quant(case, cache)
     _full_parity(orc, case)
     _full_parity(orc, case, partition_size=0)
 
 
-def _as_e4m3(case):
-    """Turn a bf16 case into an E4M3 one: the same rows become fill rows."""
-    nb, bs = case.num_blocks, case.bs
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("bs", [16, 64])
+@pytest.mark.parametrize("cache", ["e4m3", "int8"])
+def test_per_head_scales(orc, d, bs, cache):
+    """Quantised caches with one scale per KV head (pa_*_head_scales) against the oracle; the
+    heads' ranges are made to differ by 20x so that a wrong head's scale shows."""
+    h_kv, g = 4, 2
+    case = workloads.make_case("llama3_8b_b64", 11 * d + bs, B=4, h_q=h_kv * g, h_kv=h_kv, d=d, bs=bs,
+                               ctx_range=(1, 600), pool_factor=1.2, partition=128)
+    spread = torch.tensor([1.0, 20.0, 0.3, 5.0]).to(case.k_cache.device)[None, :, None, None]
+    case.k_cache = (case.k_cache.float() * spread).to(torch.bfloat16)
+    case.v_cache = (case.v_cache.float() * spread.flip(1)).to(torch.bfloat16)
+    case.key_new = (case.key_new.float() * spread[:, :, :, 0]).to(torch.bfloat16)
+    case.value_new = (case.value_new.float() * spread.flip(1)[:, :, :, 0]).to(torch.bfloat16)
+    case = _as_quant(case, cache, "head")
+    assert case.per_head_scales and float(case.k_scale.max() / case.k_scale.min()) > 10
+    _full_parity(orc, case)
+    _full_parity(orc, case, partition_size=0)
+
+
+def _as_quant(case, cache, granularity="tensor"):
+    """Turn a bf16 case into a quantised one: the same rows become fill rows."""
+    bs = case.bs
     kc, vc = case.k_cache, case.v_cache
     owned = ~torch.isnan(kc.float()).all(dim=3).all(dim=1)            # [nb, bs]
     ids = owned.reshape(-1).nonzero().flatten()
@@ -103,13 +122,37 @@ def _as_e4m3(case):
     case.fill_k_rows = kc.permute(0, 2, 1, 3)[blk, off].contiguous()
     case.fill_v_rows = vc.permute(0, 2, 1, 3)[blk, off].contiguous()
     case.fill_slots = ids.to(torch.int64)
-    kmax = max(float(case.fill_k_rows.float().abs().max()), float(case.key_new.float().abs().max()))
-    vmax = max(float(case.fill_v_rows.float().abs().max()), float(case.value_new.float().abs().max()))
-    case.k_scale = float(torch.tensor(kmax / 448.0, dtype=torch.float32))
-    case.v_scale = float(torch.tensor(vmax / 448.0, dtype=torch.float32))
-    case.cache = "e4m3"
+    case.cache = cache
+    workloads.set_scales(case, granularity)
     case.k_cache = case.v_cache = None
     return case
+
+
+
+@pytest.mark.parametrize("bs", [16, 32, 64])
+def test_int8_mha_b32_sampled_full_size(orc, bs):
+    case = workloads.make_case("int8_mha_b32_bs%d" % bs, 0, device=DEV)
+    g = torch.Generator().manual_seed(bs)
+    rows = [(int(s), int(h)) for s, h in zip(torch.randint(0, case.B, (48,), generator=g),
+                                             torch.randint(0, case.h_q, (48,), generator=g))]
+    seqs = sorted({s for s, _ in rows})
+    _full_parity(orc, case, rows=rows, seqs=seqs)
+
+
+@pytest.mark.parametrize("bs", [16, 32, 64])
+@pytest.mark.parametrize("seed", [0, 1])
+def test_int8_mha_reduced_all_rows(orc, bs, seed):
+    case = workloads.make_case("int8_mha_b32_bs%d" % bs, seed, B=3, ctx_fixed=777, h_q=8, h_kv=8)
+    _full_parity(orc, case)
+
+
+def test_int8_per_head_workload_sampled(orc):
+    case = workloads.make_case("int8_mha_b32_bs16_head", 0, device=DEV)
+    assert case.per_head_scales
+    g = torch.Generator().manual_seed(5)
+    rows = [(int(s), int(h)) for s, h in zip(torch.randint(0, case.B, (32,), generator=g),
+                                             torch.randint(0, case.h_q, (32,), generator=g))]
+    _full_parity(orc, case, rows=rows, seqs=sorted({s for s, _ in rows}))
 
 
 # ---------------------------------------------------------------- invariants and special cases

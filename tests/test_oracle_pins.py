@@ -133,8 +133,47 @@ def pin_div_f32(orc):
     assert np.array_equal(orc.div_f32(x.numpy(), s), want)
 
 
+def _int8_expected(c: int, off: float) -> int:
+    """Integer reasoning for x = c + off, |off| <= 1/2: the nearest integer, the even one on a
+    tie, then limited to [-127, 127]."""
+    if abs(off) < 0.5:
+        r = c
+    else:
+        r = c if c % 2 == 0 else c + (1 if off > 0 else -1)
+    return max(-127, min(127, r))
+
+
+def pin_int8_codec(orc):
+    codes = np.arange(-128, 128, dtype=np.int16).astype(np.int8)
+    assert np.array_equal(orc.int8_decode(codes), np.arange(-128, 128, dtype=np.float64))
+    # brute force around every integer of the range and past both ends (all exact in fp32)
+    offs = [-0.5, -0.49999997, -0.25, 0.0, 0.25, 0.49999997, 0.5]
+    xs, want = [], []
+    for c in range(-140, 141):
+        for o in offs:
+            x = np.float32(c) + np.float32(o)
+            if float(x) - c != o:              # not exactly representable at this magnitude
+                continue
+            xs.append(x)
+            want.append(_int8_expected(c, o))
+    got = orc.int8_encode_sat(np.array(xs, np.float32))
+    assert np.array_equal(got.astype(np.int64), np.array(want, np.int64))
+    special = np.array([np.nan, np.inf, -np.inf, 1e30, -1e30, -127.6, -127.5, -127.4, 127.5, -0.0, 1e-30],
+                       np.float32)
+    assert orc.int8_encode_sat(special).tolist() == [0, 127, -127, 127, -127, -127, -127, -127, 127, 0, 0]
+    # random values against torch's round-half-to-even, clamped
+    g = torch.Generator().manual_seed(12)
+    v = torch.randn(1 << 18, generator=g) * 60
+    exp = torch.round(v).clamp(-127, 127).to(torch.int8).numpy()
+    assert np.array_equal(orc.int8_encode_sat(v.numpy()), exp)
+
+
 def test_bf16_codec(orc):
     pin_bf16_codec(orc)
+
+
+def test_int8_codec(orc):
+    pin_int8_codec(orc)
 
 
 def test_e4m3_codec(orc):
@@ -325,7 +364,7 @@ def pin_fp8_decode(orc):
     for c in codes_k + codes_v:                       # no NaN codes in live slots
         c[(c & 0x7F) == 0x7F] = 0x7E
     q = torch.randn(B, h_q, d, generator=g).to(torch.bfloat16)
-    ksc, vsc = 0.0123, 0.0071
+    ksc, vsc = float(np.float32(0.0123)), float(np.float32(0.0071))    # scales are fp32
     nb = sum(-(-n // bs) for n in ctxs) + 2
     order = torch.randperm(nb, generator=g).tolist()
     kp = torch.full((nb, h_kv, bs, d), E4M3_NAN, dtype=torch.uint8)
@@ -344,6 +383,76 @@ def pin_fp8_decode(orc):
     deq_k = [c.view(torch.float8_e4m3fn).to(torch.float64) * ksc for c in codes_k]
     deq_v = [c.view(torch.float8_e4m3fn).to(torch.float64) * vsc for c in codes_v]
     want = sdpa_reference(q, deq_k, deq_v, 1 / math.sqrt(d)).numpy()
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-13)
+
+
+def _quantised_pool(codes_k, codes_v, ctxs, bs, h_kv, d, g, fill, dtype):
+    nb = sum(-(-n // bs) for n in ctxs) + 2
+    order = torch.randperm(nb, generator=g).tolist()
+    kp = torch.full((nb, h_kv, bs, d), fill, dtype=dtype)
+    vp = kp.clone()
+    table = torch.full((len(ctxs), max(-(-n // bs) for n in ctxs)), -1, dtype=torch.int32)
+    pos = 0
+    for s, n in enumerate(ctxs):
+        for i in range(-(-n // bs)):
+            phys = order[pos]; pos += 1
+            table[s, i] = phys
+            r = slice(i * bs, min((i + 1) * bs, n))
+            kp[phys, :, :r.stop - r.start] = codes_k[s][r].transpose(0, 1)
+            vp[phys, :, :r.stop - r.start] = codes_v[s][r].transpose(0, 1)
+    return kp, vp, table
+
+
+def pin_int8_decode_per_head(orc):
+    """INT8 cache with a different scale per KV head: the oracle equals fp64 SDPA over the
+    rows dequantised by torch (code x the head's scale), and a per-tensor call equals the
+    per-head call with equal scales."""
+    B, h_q, h_kv, d, bs = 3, 8, 4, 64, 16
+    g = torch.Generator().manual_seed(19)
+    ctxs = [33, 16, 70]
+    codes_k = [torch.randint(-127, 128, (n, h_kv, d), generator=g, dtype=torch.int8) for n in ctxs]
+    codes_v = [torch.randint(-127, 128, (n, h_kv, d), generator=g, dtype=torch.int8) for n in ctxs]
+    q = torch.randn(B, h_q, d, generator=g).to(torch.bfloat16)
+    ksc = np.array([0.011, 0.023, 0.0047, 0.031], np.float32)
+    vsc = np.array([0.019, 0.006, 0.027, 0.013], np.float32)
+    kp, vp, table = _quantised_pool(codes_k, codes_v, ctxs, bs, h_kv, d, g, -128, torch.int8)
+    scale = 1 / math.sqrt(d)
+    got = orc.paged_decode(_bits(q), kp.numpy(), vp.numpy(), table.numpy(), np.array(ctxs, np.int32),
+                           h_kv=h_kv, bs=bs, scale=scale, cache="int8", k_scale=ksc, v_scale=vsc)
+    kt = torch.from_numpy(ksc.astype(np.float64))[None, :, None]
+    vt = torch.from_numpy(vsc.astype(np.float64))[None, :, None]
+    deq_k = [c.to(torch.float64) * kt for c in codes_k]
+    deq_v = [c.to(torch.float64) * vt for c in codes_v]
+    want = sdpa_reference(q, deq_k, deq_v, scale).numpy()
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-13)
+    one = orc.paged_decode(_bits(q), kp.numpy(), vp.numpy(), table.numpy(), np.array(ctxs, np.int32),
+                           h_kv=h_kv, bs=bs, scale=scale, cache="int8", k_scale=0.02, v_scale=0.01)
+    same = orc.paged_decode(_bits(q), kp.numpy(), vp.numpy(), table.numpy(), np.array(ctxs, np.int32),
+                            h_kv=h_kv, bs=bs, scale=scale, cache="int8", k_scale=[0.02] * h_kv,
+                            v_scale=[0.01] * h_kv)
+    assert np.array_equal(one, same)
+
+
+def pin_fp8_decode_per_head(orc):
+    """E4M3 cache with per-KV-head scales against fp64 SDPA on torch-dequantised rows."""
+    B, h_q, h_kv, d, bs = 2, 4, 2, 64, 16
+    g = torch.Generator().manual_seed(23)
+    ctxs = [40, 17]
+    codes_k = [torch.randint(0, 256, (n, h_kv, d), generator=g, dtype=torch.uint8) for n in ctxs]
+    codes_v = [torch.randint(0, 256, (n, h_kv, d), generator=g, dtype=torch.uint8) for n in ctxs]
+    for c in codes_k + codes_v:
+        c[(c & 0x7F) == 0x7F] = 0x7E
+    q = torch.randn(B, h_q, d, generator=g).to(torch.bfloat16)
+    ksc = np.array([0.0093, 0.0210], np.float32)
+    vsc = np.array([0.0150, 0.0041], np.float32)
+    kp, vp, table = _quantised_pool(codes_k, codes_v, ctxs, bs, h_kv, d, g, E4M3_NAN, torch.uint8)
+    got = orc.paged_decode(_bits(q), kp.numpy(), vp.numpy(), table.numpy(), np.array(ctxs, np.int32),
+                           h_kv=h_kv, bs=bs, scale=0.125, cache="e4m3", k_scale=ksc, v_scale=vsc)
+    kt = torch.from_numpy(ksc.astype(np.float64))[None, :, None]
+    vt = torch.from_numpy(vsc.astype(np.float64))[None, :, None]
+    deq_k = [c.view(torch.float8_e4m3fn).to(torch.float64) * kt for c in codes_k]
+    deq_v = [c.view(torch.float8_e4m3fn).to(torch.float64) * vt for c in codes_v]
+    want = sdpa_reference(q, deq_k, deq_v, 0.125).numpy()
     np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-13)
 
 
@@ -388,6 +497,14 @@ def test_decode_rows_subset(orc):
     pin_decode_rows_subset(orc)
 
 
+def test_int8_decode_per_head(orc):
+    pin_int8_decode_per_head(orc)
+
+
+def test_fp8_decode_per_head(orc):
+    pin_fp8_decode_per_head(orc)
+
+
 # ----------------------------------------------------------------------------
 # cache write and block copy
 # ----------------------------------------------------------------------------
@@ -425,6 +542,23 @@ def pin_reshape_and_cache(orc):
     assert np.array_equal(kc8, e8k.numpy()) and np.array_equal(vc8, e8v.numpy())
     # saturation is exercised: |x| up to ~4 sigma * 3 / 0.0137 >> 448
     assert (np.abs(key.float().numpy()) / ksc > 448).any()
+    # INT8 with a scale per KV head: torch's round-half-to-even of the fp32 quotient, clamped
+    kh = np.array([0.031, 0.052, 0.017, 0.09], np.float32)
+    vh = np.array([0.044, 0.021, 0.075, 0.012], np.float32)
+    kc_i = np.full((nb, h_kv, bs, d), -128, np.int8)
+    vc_i = kc_i.copy()
+    orc.reshape_and_cache(_bits(key), _bits(val), kc_i, vc_i, slots.numpy(), h_kv=h_kv, d=d, bs=bs,
+                          num_blocks=nb, cache="int8", k_scale=kh, v_scale=vh)
+    eik = torch.full((nb, h_kv, bs, d), -128, dtype=torch.int8)
+    eiv = eik.clone()
+    for t, s_ in enumerate(slots.tolist()):
+        if s_ >= 0:
+            qk = torch.round(key[t].float() / torch.from_numpy(kh)[:, None]).clamp(-127, 127)
+            qv = torch.round(val[t].float() / torch.from_numpy(vh)[:, None]).clamp(-127, 127)
+            eik[s_ // bs, :, s_ % bs, :] = qk.to(torch.int8)
+            eiv[s_ // bs, :, s_ % bs, :] = qv.to(torch.int8)
+    assert np.array_equal(kc_i, eik.numpy()) and np.array_equal(vc_i, eiv.numpy())
+    assert (np.abs(key.float().numpy()) / kh[None, :, None] > 127).any()     # saturation exercised
 
 
 def pin_copy_blocks(orc):
@@ -458,10 +592,11 @@ def test_copy_blocks(orc):
 # the pins bite: planted mistakes in copies of the oracle must fail a pin
 # ----------------------------------------------------------------------------
 
-ALL_PINS = [pin_closed_forms, pin_bf16_codec, pin_e4m3_codec, pin_div_f32, pin_decode_vs_sdpa,
-            pin_decode_brute_force, pin_decode_special_cases, pin_worked_block_table_example,
-            pin_permutation_invariance, pin_fp8_decode, pin_decode_rows_subset, pin_reshape_and_cache,
-            pin_copy_blocks]
+ALL_PINS = [pin_closed_forms, pin_bf16_codec, pin_e4m3_codec, pin_int8_codec, pin_div_f32,
+            pin_decode_vs_sdpa, pin_decode_brute_force, pin_decode_special_cases,
+            pin_worked_block_table_example, pin_permutation_invariance, pin_fp8_decode,
+            pin_int8_decode_per_head, pin_fp8_decode_per_head, pin_decode_rows_subset,
+            pin_reshape_and_cache, pin_copy_blocks]
 
 MUTANTS = {
     "gqa_mapping": ("int kvh = h / g;", "int kvh = h % h_kv;"),
@@ -482,6 +617,14 @@ MUTANTS = {
     "copy_direction": ("k_caches[l][(uint64_t)dst * block_bytes + b] = k_caches[l][(uint64_t)src * block_bytes + b];",
                        "k_caches[l][(uint64_t)src * block_bytes + b] = k_caches[l][(uint64_t)dst * block_bytes + b];"),
     "closed_form_factor": ("return 2ull * (uint64_t)layers", "return 1ull * (uint64_t)layers"),
+    "int8_round_half_up": ("else r = (fmod(f, 2.0) == 0.0) ? f : f + 1.0;", "else r = f + 1.0;"),
+    "int8_asymmetric_range": ("if (x <= -127.0f) return -127;", "if (x <= -128.0f) return -128;"),
+    "int8_decode_unsigned": ("double or_int8_decode(int8_t c) { return (double)c; }",
+                             "double or_int8_decode(int8_t c) { return (double)(uint8_t)c; }"),
+    "per_head_scale_index": ("double k_scale = cache_dtype ? (double)k_scales[kvh] : 1.0;",
+                             "double k_scale = cache_dtype ? (double)k_scales[0] : 1.0;"),
+    "per_head_encode_index": ("or_int8_encode_sat(or_div_f32(vx, v_scales[h]))",
+                              "or_int8_encode_sat(or_div_f32(vx, v_scales[0]))"),
 }
 
 

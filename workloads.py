@@ -20,6 +20,8 @@ shared_prefix_4x8      4 prompts x 2048 tokens, each shared by 8 samples through
                        identical physical ids; private tails ~ U{0..256}
 fp8_mha_b32_bs{16,32,64}  32 seqs, 32 q / 32 kv heads, d 128, E4M3 cache with a
                        per-tensor fp32 scale max|x|/448, ctx 4096
+int8_mha_b32_bs{16,32,64} the same shape with an INT8 cache, per-tensor scale max|x|/127
+int8_mha_b32_bs16_head  INT8, bs 16, one scale per KV head: max over that head's values / 127
 =====================  ==========================================================
 
 Values: q, K, V ~ N(0, 1) drawn in fp32 by ``torch.Generator(device).manual_seed(seed)``
@@ -38,6 +40,8 @@ import torch
 
 BF16_NAN = 0x7FC1          # bf16 quiet NaN with a payload: the "never read this" sentinel
 E4M3_NAN = 0x7F            # E4M3 NaN code
+INT8_UNUSED = -128         # an INT8 code the symmetric encoder never writes
+QUANT_MAX = {"e4m3": 448.0, "int8": 127.0}   # largest code magnitude: scale = max|x| / QUANT_MAX
 
 CONFIGS = {
     "tiny_gqa2_d64": dict(B=2, h_q=4, h_kv=2, d=64, bs=16, cache="bf16", ctx_cached=(37, 80),
@@ -54,6 +58,14 @@ CONFIGS = {
                              pool_factor=1.0, partition=512),
     "fp8_mha_b32_bs64": dict(B=32, h_q=32, h_kv=32, d=128, bs=64, cache="e4m3", ctx_fixed=4096,
                              pool_factor=1.0, partition=512),
+    "int8_mha_b32_bs16": dict(B=32, h_q=32, h_kv=32, d=128, bs=16, cache="int8", ctx_fixed=4096,
+                              pool_factor=1.0, partition=512),
+    "int8_mha_b32_bs32": dict(B=32, h_q=32, h_kv=32, d=128, bs=32, cache="int8", ctx_fixed=4096,
+                              pool_factor=1.0, partition=512),
+    "int8_mha_b32_bs64": dict(B=32, h_q=32, h_kv=32, d=128, bs=64, cache="int8", ctx_fixed=4096,
+                              pool_factor=1.0, partition=512),
+    "int8_mha_b32_bs16_head": dict(B=32, h_q=32, h_kv=32, d=128, bs=16, cache="int8", ctx_fixed=4096,
+                                   pool_factor=1.0, partition=512, scales="head"),
 }
 
 
@@ -68,7 +80,7 @@ class DecodeCase:
     d: int
     bs: int
     num_blocks: int
-    cache: str                      # "bf16" or "e4m3"
+    cache: str                      # "bf16", "e4m3" or "int8"
     partition: int
     scale: float
     q: torch.Tensor                 # bf16 [B, h_q, d]
@@ -77,16 +89,24 @@ class DecodeCase:
     slot_mapping: torch.Tensor      # int64 [B]
     block_tables: torch.Tensor      # int32 [B, max_blocks]
     context_lens: torch.Tensor      # int32 [B], including the appended token
-    # bf16 caches: filled directly [NB, h_kv, bs, d]; e4m3 caches: None (each side fills its
-    # own from fill_rows / fill_slots with its own quantiser)
+    # bf16 caches: filled directly [NB, h_kv, bs, d]; quantised caches: None (each side fills
+    # its own from fill_rows / fill_slots with its own quantiser)
     k_cache: Optional[torch.Tensor] = None
     v_cache: Optional[torch.Tensor] = None
     fill_k_rows: Optional[torch.Tensor] = None   # bf16 [n_fill, h_kv, d]
     fill_v_rows: Optional[torch.Tensor] = None
     fill_slots: Optional[torch.Tensor] = None    # int64 [n_fill]
-    k_scale: float = 1.0
+    k_scale: float = 1.0            # per-tensor scales, or (scales="head") fp32 [h_kv] CPU tensors
     v_scale: float = 1.0
     meta: dict = field(default_factory=dict)
+
+    @property
+    def quantised(self) -> bool:
+        return self.cache in QUANT_MAX
+
+    @property
+    def per_head_scales(self) -> bool:
+        return isinstance(self.k_scale, torch.Tensor)
 
     @property
     def max_context_len(self) -> int:
@@ -94,7 +114,7 @@ class DecodeCase:
 
     @property
     def elem_bytes(self) -> int:
-        return 1 if self.cache == "e4m3" else 2
+        return 1 if self.quantised else 2
 
     def kv_bytes(self) -> int:
         """K+V bytes the step must read: sum of ctx * h_kv * d * elem * 2."""
@@ -194,27 +214,46 @@ def make_case(name: str, seed: int = 0, device="cpu", **over) -> DecodeCase:
         case.k_cache = torch.where(hole, nan, pool_k)
         case.v_cache = torch.where(hole, nan, pool_v)
     else:
-        # E4M3: each side quantises the owned rows itself (pool layout -> rows + slot ids).
+        # quantised: each side quantises the owned rows itself (pool layout -> rows + slot ids).
         ids = owned.reshape(-1).nonzero().flatten()                 # slot ids of owned tokens
         blk, off = ids // bs, ids % bs
         kr = pool_k.permute(0, 2, 1, 3)[blk.to(device), off.to(device)]   # [n, h_kv, d]
         vr = pool_v.permute(0, 2, 1, 3)[blk.to(device), off.to(device)]
         case.fill_k_rows, case.fill_v_rows = kr.contiguous(), vr.contiguous()
         case.fill_slots = ids.to(torch.int64).to(device)
-        # per-tensor scale over every K (resp. V) value of the workload, appended tokens included
-        kmax = torch.maximum(kr.float().abs().max(), k_new.float().abs().max())
-        vmax = torch.maximum(vr.float().abs().max(), v_new.float().abs().max())
-        case.k_scale = float((kmax / 448.0).item())
-        case.v_scale = float((vmax / 448.0).item())
+        set_scales(case, cfg.get("scales", "tensor"))
     return case
 
 
-def empty_e4m3_pool(case: DecodeCase, device=None) -> tuple[torch.Tensor, torch.Tensor]:
-    """Two uint8 pools [NB, h_kv, bs, d] filled with the E4M3 NaN sentinel."""
+def set_scales(case: DecodeCase, granularity: str = "tensor") -> DecodeCase:
+    """Scales of a quantised case from its fill rows and appended rows: max|x| / QUANT_MAX over
+    every K (resp. V) value of the workload ("tensor", floats) or over each KV head's values
+    ("head", fp32 [h_kv] CPU tensors)."""
+    qmax = QUANT_MAX[case.cache]
+    out = []
+    for rows, new in ((case.fill_k_rows, case.key_new), (case.fill_v_rows, case.value_new)):
+        a = torch.cat([rows.float().abs().reshape(-1, case.h_kv, case.d),
+                       new.float().abs().reshape(-1, case.h_kv, case.d)]).cpu()
+        if granularity == "head":
+            out.append((a.amax(dim=(0, 2)) / qmax).to(torch.float32))
+        elif granularity == "tensor":
+            out.append(float((a.max() / qmax).item()))
+        else:
+            raise ValueError(granularity)
+    case.k_scale, case.v_scale = out
+    return case
+
+
+def empty_quant_pool(case: DecodeCase, device=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """Two code pools [NB, h_kv, bs, d] filled with a code the cache write never produces:
+    uint8 E4M3 NaN for "e4m3", int8 -128 for "int8"."""
     device = device if device is not None else case.q.device
     shape = (case.num_blocks, case.h_kv, case.bs, case.d)
-    return (torch.full(shape, E4M3_NAN, dtype=torch.uint8, device=device),
-            torch.full(shape, E4M3_NAN, dtype=torch.uint8, device=device))
+    if case.cache == "int8":
+        fill, dt = INT8_UNUSED, torch.int8
+    else:
+        fill, dt = E4M3_NAN, torch.uint8
+    return (torch.full(shape, fill, dtype=dt, device=device), torch.full(shape, fill, dtype=dt, device=device))
 
 
 def _make_shared_prefix(name, cfg, seed, device, gc) -> DecodeCase:
