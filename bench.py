@@ -38,8 +38,8 @@ if ROOT not in sys.path:
 METRIC = "paged decode attention KV GB/s & % of B200 HBM peak; decode tokens/s"
 FALLBACK_HBM_GBS = 6650.0
 KERNEL_SOURCES = [os.path.join(ROOT, "paged_kv_cache_428_b200", "csrc", f)
-                  for f in ("common.cuh", "decode.cuh", "decode_mma.cuh")]
-TRAFFIC_SUMMARY = os.path.join(ROOT, "profiles", "ncu_decode_partition_llama3_8b_b64.md")
+                  for f in ("common.cuh", "decode.cuh", "decode_mma.cuh", "decode_q8.cuh", "decode_balanced.cuh")]
+PROFILES = os.path.join(ROOT, "profiles")
 
 
 def parse_args(argv=None):
@@ -143,17 +143,24 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def ncu_traffic_per_launch():
-    """DRAM bytes (read + write) of one partition-kernel launch from the committed ncu summary,
-    or None when the summary is missing or the kernel source changed since it was taken."""
-    if not os.path.exists(TRAFFIC_SUMMARY):
+def ncu_traffic_per_launch(workload: str, partition: int):
+    """DRAM bytes (read + write) of one decode-kernel launch from a committed ncu summary under
+    profiles/ that names this workload and partition size, or None when there is none or the
+    kernel sources changed since the counters were taken."""
+    if not os.path.isdir(PROFILES):
         return None
-    text = open(TRAFFIC_SUMMARY).read()
-    m = re.search(r"traffic_bytes_per_launch:\s*([0-9]+)", text)
-    h = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
-    if not m or not h or h.group(1) != kernel_source_hash():
-        return None
-    return int(m.group(1))
+    want = kernel_source_hash()
+    for name in sorted(os.listdir(PROFILES)):
+        if not name.endswith(".md"):
+            continue
+        text = open(os.path.join(PROFILES, name)).read()
+        w = re.search(r"^workload:\s*(\S+)", text, re.M)
+        p = re.search(r"^partition:\s*(-?[0-9]+)", text, re.M)
+        m = re.search(r"^traffic_bytes_per_launch:\s*([0-9]+)", text, re.M)
+        h = re.search(r"^kernel_source_sha256_16:\s*([0-9a-f]+)", text, re.M)
+        if w and p and m and h and w.group(1) == workload and int(p.group(1)) == partition and h.group(1) == want:
+            return int(m.group(1))
+    return None
 
 
 # -------------------------------------------------------------------------------------- clocks
@@ -443,7 +450,7 @@ def run_ours(args):
         "roofline": {"bound": "hbm", "kernel": kernel, "achieved": round(achieved, 1),
                      "peak": peak, "peak_kind": peak_kind + " (hbm_gbs copy bandwidth)", "unit": "GB/s",
                      "frac": round(achieved / peak, 4),
-                     "traffic": ncu_traffic_per_launch() if (args.workload, P) == ("llama3_8b_b64", 512) else None,
+                     "traffic": ncu_traffic_per_launch(args.workload, P),
                      "algorithmic_bytes_per_launch": part_bytes},
         "gpu_launches": K * (2 + (1 if P > 0 and -(-mcl // P) > 16 else 0)),
         "clocks": clocks,

@@ -147,14 +147,21 @@ __device__ __forceinline__ void mma_consume_block(uint8_t *ktile, int valid, con
         // P^T as the B operand: b0 = P[head T/4][tokens 2tq, 2tq+1], b1 = tokens + 8
         const uint32_t pb0 = movmatrix_trans(pack_bf16x2(p0, p1));
         const uint32_t pb1 = movmatrix_trans(pack_bf16x2(p2, p3));
+        // rescale the accumulators only when a running max moved (after the first few
+        // sub-blocks it rarely does); the vote keeps the branch uniform over the warp
+        if (__any_sync(FULL, (al0 != 1.f) | (al1 != 1.f))) {
+#pragma unroll
+            for (int mt = 0; mt < C::MT; ++mt) {
+                o[mt][0] *= al0;
+                o[mt][1] *= al1;
+                o[mt][2] *= al0;
+                o[mt][3] *= al1;
+            }
+        }
         // ---- O^T += V^T . P^T (m-tiles of 16 head dims) ----
         const int tok = sub * 16 + (mat >> 1) * 8 + mrow;
 #pragma unroll
         for (int mt = 0; mt < C::MT; ++mt) {
-            o[mt][0] *= al0;
-            o[mt][1] *= al1;
-            o[mt][2] *= al0;
-            o[mt][3] *= al1;
             const int chunk = ((2 * mt) & 7) + (mat & 1);
             uint32_t a[4];
             ldmatrix_x4_trans(a, vbase + (mt >> 2) * C::HALF_BYTES + swz128(tok, chunk));

@@ -128,6 +128,37 @@ __device__ __forceinline__ float q8_load_q(uint32_t (&qb)[C::KS][2], const __nv_
     return exp2f((float)e);
 }
 
+// O^T += V^T . P^T for one 16-token sub-block, two m-tiles (chunks) per x4 load.  MASKED:
+// V values of tokens at or past `valid` are zeroed (this lane's tokens: u, u + 1, u + 8, u + 9).
+template <class C, int D, int QT, bool MASKED>
+__device__ __forceinline__ void q8_pv(uint32_t vbase, int tok, int mat, int u, int valid, uint32_t pb0, uint32_t pb1,
+                                      float (&o)[C::MT][4])
+{
+    uint32_t keep_lo = 0xffffffffu, keep_hi = 0xffffffffu;
+    if constexpr (MASKED) {
+        keep_lo = (u < valid ? 0x0000ffffu : 0u) | (u + 1 < valid ? 0xffff0000u : 0u);
+        keep_hi = (u + 8 < valid ? 0x0000ffffu : 0u) | (u + 9 < valid ? 0xffff0000u : 0u);
+    }
+#pragma unroll
+    for (int mt = 0; mt < C::MT; mt += 2) {
+        uint32_t w[4];
+        ldmatrix_x4_trans(w, vbase + swz_q8<D>(tok, mt + (mat >> 1)));
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            uint32_t a0, a1, a2, a3;
+            q8_cross_to_f16<QT>(w[2 * j], a0, a1);
+            q8_cross_to_f16<QT>(w[2 * j + 1], a2, a3);
+            if constexpr (MASKED) {
+                a0 &= keep_lo;
+                a1 &= keep_lo;
+                a2 &= keep_hi;
+                a3 &= keep_hi;
+            }
+            mma_f16_16816(o[mt + j], a0, a1, a2, a3, pb0, pb1);
+        }
+    }
+}
+
 // One physical block's code tiles (K at `ktile`, V right after it), already in shared memory,
 // folded into a warp's online-softmax state; `valid` tokens of the block count.
 // o[mt][0..1] are dim 16 mt + 2 (T/4), o[mt][2..3] dim 16 mt + 2 (T/4) + 1 (heads 2t, 2t+1).
@@ -182,39 +213,26 @@ __device__ __forceinline__ void q8_consume_block(const uint8_t *ktile, int valid
         l_run[1] = l_run[1] * al1 + (p1 + p3);
         const uint32_t pb0 = movmatrix_trans(pack_f16x2(p0, p1));
         const uint32_t pb1 = movmatrix_trans(pack_f16x2(p2, p3));
-        // V values of tokens past the context -> 0 (this lane's tokens: 2tq, 2tq+1 and + 8)
-        uint32_t keep_lo = 0xffffffffu, keep_hi = 0xffffffffu;
-        if (valid < sub * 16 + 16) {
-            const int u = sub * 16 + 2 * tq;
-            keep_lo = (u < valid ? 0x0000ffffu : 0u) | (u + 1 < valid ? 0xffff0000u : 0u);
-            keep_hi = (u + 8 < valid ? 0x0000ffffu : 0u) | (u + 9 < valid ? 0xffff0000u : 0u);
-        }
-        // ---- O^T += V^T . P^T, two m-tiles (chunks) per x4 load ----
+        // rescale the accumulators only when a running max moved (after the first few
+        // sub-blocks it rarely does); the vote keeps the branch uniform over the warp
+        if (__any_sync(FULL, (al0 != 1.f) | (al1 != 1.f))) {
 #pragma unroll
-        for (int mt = 0; mt < C::MT; mt += 2) {
-            uint32_t w[4];
-            ldmatrix_x4_trans(w, vbase + swz_q8<D>(tok, mt + (mat >> 1)));
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                o[mt + j][0] *= al0;
-                o[mt + j][1] *= al1;
-                o[mt + j][2] *= al0;
-                o[mt + j][3] *= al1;
-                uint32_t a0, a1, a2, a3;
-                q8_cross_to_f16<QT>(w[2 * j], a0, a1);
-                q8_cross_to_f16<QT>(w[2 * j + 1], a2, a3);
-                a0 &= keep_lo;
-                a1 &= keep_lo;
-                a2 &= keep_hi;
-                a3 &= keep_hi;
-                mma_f16_16816(o[mt + j], a0, a1, a2, a3, pb0, pb1);
+            for (int mt = 0; mt < C::MT; ++mt) {
+                o[mt][0] *= al0;
+                o[mt][1] *= al1;
+                o[mt][2] *= al0;
+                o[mt][3] *= al1;
             }
         }
+        if (valid < sub * 16 + 16)
+            q8_pv<C, D, QT, true>(vbase, tok, mat, sub * 16 + 2 * tq, valid, pb0, pb1, o);
+        else
+            q8_pv<C, D, QT, false>(vbase, tok, mat, 0, 0, pb0, pb1, o);
     }
 }
 
 template <int D, int BS, int G, int QT, int NW_ = 2, int RING_ = 32768>
-__global__ void __launch_bounds__(MmaQ8Config<D, BS, G, NW_, RING_>::THREADS)
+__global__ void __maxnreg__(96)
     paged_decode_partition_q8_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
                                      const __grid_constant__ CUtensorMap tmap_v)
 {

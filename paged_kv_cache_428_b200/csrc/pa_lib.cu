@@ -190,16 +190,25 @@ int launch_partition_mma(const DecodeParams &prm, int num_seqs, cudaStream_t st)
     return launch_status();
 }
 
+// Consumer warps and ring bytes of the one-byte-code kernel: 2 warps and a 32 KB ring (6 CTAs
+// per SM) measured best at every block size (against 1, 3 and 4 warps, 16 to 64 KB rings).
+template <int BS>
+struct Q8Tuning {
+    static constexpr int NW = 2;
+    static constexpr int RING = 32768;
+};
+
 template <int D, int BS, int G, int QT>
 int launch_partition_q8(const DecodeParams &prm, int num_seqs, cudaStream_t st)
 {
-    using C = MmaQ8Config<D, BS, G>;
+    constexpr int NW = Q8Tuning<BS>::NW, RING = Q8Tuning<BS>::RING;
+    using C = MmaQ8Config<D, BS, G, NW, RING>;
     static std::atomic<unsigned long long> smem_set{0};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
     const unsigned long long bit = 1ull << (dev & 63);
     if (!(smem_set.load(std::memory_order_acquire) & bit)) {
-        if (cudaFuncSetAttribute(paged_decode_partition_q8_kernel<D, BS, G, QT>,
+        if (cudaFuncSetAttribute(paged_decode_partition_q8_kernel<D, BS, G, QT, NW, RING>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
             return PA_ERR_CUDA;
         smem_set.fetch_or(bit, std::memory_order_release);
@@ -209,7 +218,7 @@ int launch_partition_q8(const DecodeParams &prm, int num_seqs, cudaStream_t st)
     if (rc == PA_OK) rc = cached_cache_map(&mv, prm.v_cache, prm.num_blocks, prm.h_kv, BS, D, 1);
     if (rc != PA_OK) return rc;
     const dim3 grid(prm.p_max, prm.h_kv, num_seqs);
-    paged_decode_partition_q8_kernel<D, BS, G, QT><<<grid, C::THREADS, C::SMEM, st>>>(prm, mk, mv);
+    paged_decode_partition_q8_kernel<D, BS, G, QT, NW, RING><<<grid, C::THREADS, C::SMEM, st>>>(prm, mk, mv);
     return launch_status();
 }
 
