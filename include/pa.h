@@ -81,6 +81,11 @@ int pa_version(void);
  * M_KV estimate).  Host only. */
 size_t pa_kv_bytes_per_token(int layers, int h_kv, int head_dim, int elem_bytes);
 
+/* Whole tokens whose KV fits in budget_bytes: budget_bytes / pa_kv_bytes_per_token(...) (0
+ * when the per-token size is 0).  "深度解构…" section 3.2: about 72k tokens of Llama-3-8B in
+ * the ~9 GB a 24 GB card leaves after the weights, twice that with an FP8 cache.  Host only. */
+size_t pa_kv_capacity_tokens(size_t budget_bytes, int layers, int h_kv, int head_dim, int elem_bytes);
+
 /* ---- cache write --------------------------------------------------------
  * Store the step's new K and V rows in their physical slots: for token t and
  * KV head h, cache[slot/bs][h][slot%bs][:] = row[t][h][:]

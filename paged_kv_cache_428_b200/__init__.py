@@ -60,6 +60,7 @@ def _load() -> ctypes.CDLL:
         "pa_status_str": (ctypes.c_char_p, [i32]),
         "pa_version": (i32, []),
         "pa_kv_bytes_per_token": (sz, [i32, i32, i32, i32]),
+        "pa_kv_capacity_tokens": (sz, [sz, i32, i32, i32, i32]),
         "pa_reshape_and_cache": (i32, [vp, vp, i64, i64, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, f32, vp]),
         "pa_reshape_and_cache_head_scales": (i32, [vp, vp, i64, i64, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp,
                                                    vp, vp]),
@@ -164,6 +165,10 @@ def _head_scales(k_scale, v_scale, h_kv: int):
 # ----------------------------------------------------------------------------------------------
 def pa_kv_bytes_per_token(layers: int, h_kv: int, head_dim: int, elem_bytes: int) -> int:
     return int(_lib.pa_kv_bytes_per_token(layers, h_kv, head_dim, elem_bytes))
+
+
+def pa_kv_capacity_tokens(budget_bytes: int, layers: int, h_kv: int, head_dim: int, elem_bytes: int) -> int:
+    return int(_lib.pa_kv_capacity_tokens(budget_bytes, layers, h_kv, head_dim, elem_bytes))
 
 
 def pa_version() -> int:

@@ -30,6 +30,12 @@ size_t pa_kv_bytes_per_token(int layers, int h_kv, int head_dim, int elem_bytes)
     return 2u * (size_t)layers * (size_t)h_kv * (size_t)head_dim * (size_t)elem_bytes;
 }
 
+size_t pa_kv_capacity_tokens(size_t budget_bytes, int layers, int h_kv, int head_dim, int elem_bytes)
+{
+    const size_t per_token = pa_kv_bytes_per_token(layers, h_kv, head_dim, elem_bytes);
+    return per_token ? budget_bytes / per_token : 0;
+}
+
 int pa_validate_block_tables(const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
                              int num_seqs, int block_size, int num_blocks)
 {

@@ -306,3 +306,39 @@ def random_rows(n: int, h_kv: int, d: int, seed: int, device="cpu") -> tuple[tor
     """K and V rows ~ N(0,1) in bf16, [n, h_kv, d] each (for cache-write cases)."""
     g = _gen(seed, torch.device(device))
     return _randn_bf16((n, h_kv, d), g, device), _randn_bf16((n, h_kv, d), g, device)
+
+
+# ---------------------------------------------------------------------------- serving traces
+# Request-length traces for the memory-utilisation measurement (host only).  Each request has a
+# prompt length and an output length; the context window bounds prompt + output.  The pages give
+# no length distribution, so the recipes are plain seeded uniforms whose names say what they are.
+TRACES = {
+    # a chat-like mix in a 2048-token window: prompts U{32..512}, outputs U{16..1024}
+    "chat_w2048_b64": dict(requests=512, slots=64, window=2048, prompt=(32, 512), output=(16, 1024), bs=16),
+    # the same mix, 8 concurrent requests (the pages' "8 concurrent requests" setting)
+    "chat_w2048_b8": dict(requests=64, slots=8, window=2048, prompt=(32, 512), output=(16, 1024), bs=16),
+    # long answers in a 4096-token window: prompts U{256..1024}, outputs U{512..3072}
+    "long_w4096_b32": dict(requests=128, slots=32, window=4096, prompt=(256, 1024), output=(512, 3072), bs=16),
+}
+
+
+@dataclass
+class Trace:
+    name: str
+    prompts: list           # prompt length of request i
+    outputs: list           # output length of request i (>= 1)
+    slots: int              # concurrent request slots (continuous batching)
+    window: int             # context window: the contiguous scheme reserves this per request
+    bs: int
+
+
+def make_trace(name: str, seed: int = 0, **over) -> Trace:
+    cfg = dict(TRACES[name])
+    cfg.update(over)
+    g = _cpu_gen(seed)
+    n = cfg["requests"]
+    p = torch.randint(cfg["prompt"][0], cfg["prompt"][1] + 1, (n,), generator=g).tolist()
+    o = torch.randint(cfg["output"][0], cfg["output"][1] + 1, (n,), generator=g).tolist()
+    if any(a + b > cfg["window"] for a, b in zip(p, o)):
+        raise ValueError("a request exceeds the window")
+    return Trace(name=name, prompts=p, outputs=o, slots=cfg["slots"], window=cfg["window"], bs=cfg["bs"])
