@@ -288,10 +288,43 @@ int  pa_alloc_free_seq(pa_alloc *a, int64_t seq);
 int  pa_alloc_block_table(const pa_alloc *a, const int64_t *seqs, int num_seqs, int32_t *table,
                           int max_blocks, int32_t *context_lens);
 int  pa_alloc_seq_len(const pa_alloc *a, int64_t seq, int64_t *len);
+/* free_blocks: blocks that can be handed out (free pool + evictable cached blocks);
+ * used_blocks: count > 0; shared_blocks: count > 1; frag_tokens: sum over sequences of
+ * allocated but unfilled slots. */
 int  pa_alloc_stats(const pa_alloc *a, int *free_blocks, int *used_blocks, int *shared_blocks,
                     int64_t *frag_tokens);
 /* Reference count of a block (>= 0), or PA_ERR_INVALID_ARG. */
 int  pa_alloc_refcount(const pa_alloc *a, int block);
+
+/* ---- prefix caching ------------------------------------------------------------
+ * "vLLM 推理原理…" section 前缀缓存能省掉哪部分工作: requests that begin with the same text
+ * reuse the KV of the common prefix, on an exact match only; the prefill of the cached part is
+ * skipped, the rest (and decoding) still runs.
+ * pa_alloc_new_seq_prefix creates a sequence holding the n prompt tokens `tokens` (host
+ * int32 token ids).  Its full blocks are looked up in order: block k matches a cached block
+ * registered with the same predecessor (the block this walk matched for k-1, or none for
+ * k = 0) and the same bs token ids; every match is shared (count + 1, an evictable block
+ * leaves the eviction list); the first miss ends the walk.  The remaining blocks are fresh,
+ * and each fresh FULL block is registered for later prompts.  A partly filled last block is
+ * never cached, so appends never write into a cached block.
+ *   slots          NULL or n entries: slot of every prompt token (cached ones included)
+ *   cached_tokens  tokens at the front whose KV is already in the cache (a multiple of
+ *                  block_size); the caller writes K/V only for tokens [cached_tokens, n)
+ * Cached blocks whose count drops to 0 stay cached and evictable; when the free pool is empty,
+ * taking a block evicts the least recently released one (its registration is dropped and
+ * entries naming it as predecessor can no longer match).  PA_ERR_OOM (state unchanged) when
+ * free + evictable blocks, minus those the walk hit, cannot hold the fresh blocks. */
+int  pa_alloc_new_seq_prefix(pa_alloc *a, const int32_t *tokens, int n, int64_t *seq_id, int64_t *slots,
+                             int *cached_tokens);
+/* Totals since creation: prompt tokens found cached / not cached by pa_alloc_new_seq_prefix;
+ * blocks registered in the cache now, and those of them with count 0 (evictable). */
+int  pa_alloc_prefix_stats(const pa_alloc *a, int64_t *hit_tokens, int64_t *miss_tokens, int *cached_blocks,
+                           int *evictable_blocks);
+/* An order of the batch `seqs` in which sequences that share physical blocks are adjacent:
+ * order[i] = index into seqs, sorted by the sequences' block lists (lexicographically by
+ * physical id; ties keep their input order).  Building the block tables in this order makes the
+ * decode kernels of sharers run close together in time, so shared blocks are read from L2. */
+int  pa_alloc_order_by_prefix(const pa_alloc *a, const int64_t *seqs, int n, int32_t *order);
 
 #ifdef __cplusplus
 }

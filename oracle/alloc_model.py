@@ -29,6 +29,18 @@ implement them, so block ids agree exactly):
   by one and the pair (old, new) is reported for the device copy.  The last
   holder (refcount 1) writes in place, so n sharers cause n - 1 copies;
 * sequence ids count up from 0.
+
+Prefix caching ("vLLM 推理原理…" section 前缀缓存能省掉哪部分工作: requests that begin with the
+same text reuse the common prefix's KV, on an exact match only):
+
+* each full block of a prompt inserted with ``new_seq_prefix`` is registered under the key
+  (predecessor block, predecessor's generation, the block's tokens); a new prompt walks its
+  full blocks from the first, sharing each block whose key is registered, and stops at the
+  first miss; the rest are fresh blocks, the full ones registered in turn;
+* a registered block whose count drops to zero stays registered and joins the end of an
+  eviction queue; when the free pool is empty a block is taken from the front of that queue,
+  its key is dropped and its generation incremented (keys naming it as predecessor can no
+  longer match); a hit on a queued block takes it out of the queue.
 """
 from __future__ import annotations
 
@@ -80,10 +92,24 @@ class AllocatorModel:
         self.refcnt = [0] * num_blocks
         self.seqs: dict[int, Seq] = {}
         self.next_id = 0
+        self.cache: dict = {}                   # (parent, parent_gen, tokens) -> block
+        self.key_of: dict = {}                  # block -> its key
+        self.gen = [0] * num_blocks
+        self.evict_queue: list = []             # registered blocks with count 0, oldest first
+        self.hit_tokens = 0
+        self.miss_tokens = 0
 
     # -- pool ----------------------------------------------------------------
+    def available(self) -> int:
+        return len(self.free) + len(self.evict_queue)
+
     def _take(self) -> int:
-        b = self.free.pop()
+        if self.free:
+            b = self.free.pop()
+        else:
+            b = self.evict_queue.pop(0)
+            del self.cache[self.key_of.pop(b)]
+            self.gen[b] += 1
         assert self.refcnt[b] == 0
         self.refcnt[b] = 1
         return b
@@ -91,7 +117,10 @@ class AllocatorModel:
     def _release(self, b: int) -> None:
         self.refcnt[b] -= 1
         if self.refcnt[b] == 0:
-            self.free.append(b)
+            if b in self.key_of:
+                self.evict_queue.append(b)
+            else:
+                self.free.append(b)
 
     # -- sequence operations -------------------------------------------------
     def new_seq(self) -> int:
@@ -111,7 +140,7 @@ class AllocatorModel:
         when no copy is needed."""
         s = self.seqs[sid]
         need, cow = self._blocks_needed(s, n)
-        if need > len(self.free):
+        if need > self.available():
             raise OutOfBlocks()
         pair = (-1, -1)
         if cow:
@@ -132,6 +161,56 @@ class AllocatorModel:
     def append_slot(self, sid: int):
         slots, pair = self.append_n(sid, 1)
         return slots[0], pair
+
+    def new_seq_prefix(self, tokens):
+        """A sequence holding the prompt `tokens`; returns (sid, slots, cached_tokens)."""
+        bs = self.bs
+        n = len(tokens)
+        full, total = n // bs, -(-n // bs)
+        hits = []
+        parent, pgen = -1, 0
+        for k in range(full):
+            key = (parent, pgen, tuple(tokens[k * bs:(k + 1) * bs]))
+            if key not in self.cache:
+                break
+            b = self.cache[key]
+            hits.append(b)
+            parent, pgen = b, self.gen[b]
+        queued_hits = sum(1 for b in hits if self.refcnt[b] == 0)
+        if total - len(hits) > self.available() - queued_hits:
+            raise OutOfBlocks()
+        s = Seq()
+        for b in hits:
+            if self.refcnt[b] == 0:
+                self.evict_queue.remove(b)
+            self.refcnt[b] += 1
+            s.blocks.append(b)
+        for k in range(len(hits), total):
+            b = self._take()
+            s.blocks.append(b)
+            if k < full:
+                prev = s.blocks[k - 1] if k > 0 else -1
+                key = (prev, self.gen[prev] if k > 0 else 0, tuple(tokens[k * bs:(k + 1) * bs]))
+                assert key not in self.cache
+                self.cache[key] = b
+                self.key_of[b] = key
+        s.length = n
+        sid = self.next_id
+        self.next_id += 1
+        self.seqs[sid] = s
+        cached = len(hits) * bs
+        self.hit_tokens += cached
+        self.miss_tokens += n - cached
+        slots = [s.blocks[t // bs] * bs + t % bs for t in range(n)]
+        return sid, slots, cached
+
+    def prefix_stats(self):
+        return {"hit_tokens": self.hit_tokens, "miss_tokens": self.miss_tokens, "cached_blocks": len(self.cache),
+                "evictable": len(self.evict_queue)}
+
+    def order_by_prefix(self, sids):
+        """Batch order with sharers adjacent: indices sorted by block list, ties in input order."""
+        return sorted(range(len(sids)), key=lambda i: (self.seqs[sids[i]].blocks, i))
 
     def fork(self, parent: int) -> int:
         p = self.seqs[parent]
@@ -164,7 +243,7 @@ class AllocatorModel:
         used = sum(1 for c in self.refcnt if c > 0)
         shared = sum(1 for c in self.refcnt if c > 1)
         frag = sum(len(s.blocks) * self.bs - s.length for s in self.seqs.values())
-        return {"free": len(self.free), "used": used, "shared": shared, "frag_tokens": frag}
+        return {"free": self.available(), "used": used, "shared": shared, "frag_tokens": frag}
 
     def check_invariants(self) -> None:
         """Conservation and refcount consistency (the properties the tests assert)."""
@@ -176,4 +255,7 @@ class AllocatorModel:
         assert holders == self.refcnt
         assert len(set(self.free)) == len(self.free)
         assert all(self.refcnt[b] == 0 for b in self.free)
-        assert len(self.free) + sum(1 for c in self.refcnt if c > 0) == self.num_blocks
+        assert all(self.refcnt[b] == 0 and b in self.key_of for b in self.evict_queue)
+        assert not set(self.free) & set(self.key_of)
+        assert all(self.cache[k] == b for b, k in self.key_of.items()) and len(self.cache) == len(self.key_of)
+        assert self.available() + sum(1 for c in self.refcnt if c > 0) == self.num_blocks

@@ -90,6 +90,9 @@ def _load() -> ctypes.CDLL:
         "pa_alloc_seq_len": (i32, [vp, i64, P64]),
         "pa_alloc_stats": (i32, [vp, PI, PI, PI, P64]),
         "pa_alloc_refcount": (i32, [vp, i32]),
+        "pa_alloc_new_seq_prefix": (i32, [vp, vp, i32, P64, vp, PI]),
+        "pa_alloc_prefix_stats": (i32, [vp, P64, P64, PI, PI]),
+        "pa_alloc_order_by_prefix": (i32, [vp, vp, i32, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -457,6 +460,33 @@ class BlockAllocator:
         _check(_lib.pa_alloc_stats(self._h, ctypes.byref(f), ctypes.byref(u), ctypes.byref(s), ctypes.byref(fr)),
                "pa_alloc_stats")
         return {"free": f.value, "used": u.value, "shared": s.value, "frag_tokens": fr.value}
+
+    def new_seq_prefix(self, tokens: Sequence[int]):
+        """A sequence holding the prompt `tokens`, sharing cached full blocks of an identical
+        prefix: returns (seq_id, slots, cached_tokens); write K/V only for tokens[cached:]."""
+        n = len(tokens)
+        tk = (ctypes.c_int32 * max(n, 1))(*tokens)
+        slots = (ctypes.c_int64 * max(n, 1))()
+        sid, cached = ctypes.c_int64(), ctypes.c_int()
+        _check(_lib.pa_alloc_new_seq_prefix(self._h, ctypes.cast(tk, ctypes.c_void_p), n, ctypes.byref(sid),
+                                            ctypes.cast(slots, ctypes.c_void_p), ctypes.byref(cached)),
+               "pa_alloc_new_seq_prefix")
+        return sid.value, list(slots)[:n], cached.value
+
+    def prefix_stats(self) -> dict:
+        h, m = ctypes.c_int64(), ctypes.c_int64()
+        c, e = ctypes.c_int(), ctypes.c_int()
+        _check(_lib.pa_alloc_prefix_stats(self._h, ctypes.byref(h), ctypes.byref(m), ctypes.byref(c),
+                                          ctypes.byref(e)), "pa_alloc_prefix_stats")
+        return {"hit_tokens": h.value, "miss_tokens": m.value, "cached_blocks": c.value, "evictable": e.value}
+
+    def order_by_prefix(self, seqs: Sequence[int]) -> list:
+        n = len(seqs)
+        sq = (ctypes.c_int64 * max(n, 1))(*seqs)
+        order = (ctypes.c_int32 * max(n, 1))()
+        _check(_lib.pa_alloc_order_by_prefix(self._h, ctypes.cast(sq, ctypes.c_void_p), n,
+                                             ctypes.cast(order, ctypes.c_void_p)), "pa_alloc_order_by_prefix")
+        return list(order)[:n]
 
     def refcount(self, block: int) -> int:
         rc = _lib.pa_alloc_refcount(self._h, block)

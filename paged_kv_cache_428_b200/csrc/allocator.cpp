@@ -7,9 +7,21 @@
 // 共享"); the first write into a partly filled shared block copies it ("深度解构…" section
 // 2.3; intelliparadigm section 3.1); a finished sequence releases its blocks ("vLLM 推理原理…"
 // generation flow).  Policy details the pages leave open are stated in pa.h.
+//
+// Prefix caching ("vLLM 推理原理…" section 前缀缓存能省掉哪部分工作: requests that start with the
+// same text reuse the KV of the common prefix, on an exact match only): every full block of a
+// prompt inserted with pa_alloc_new_seq_prefix is registered under (the physical block before it
+// and that block's generation, the block's token ids).  A later prompt walks its blocks from the
+// first one and shares every block found; the first miss ends the walk.  Cached blocks whose
+// count drops to zero stay cached and become evictable, least recently released first, when the
+// free pool runs dry; evicting a block bumps its generation, so entries that named it as their
+// predecessor can no longer match.
 #include <algorithm>
 #include <cstdint>
+#include <list>
+#include <map>
 #include <new>
+#include <numeric>
 #include <unordered_map>
 #include <unordered_set>
 #include <vector>
@@ -33,6 +45,20 @@ struct Sequence {
     int64_t len = 0;
 };
 
+// Identity of a cached block: its predecessor (physical id and generation; -1 for the first block
+// of a prompt) and its token ids.
+struct PrefixKey {
+    int32_t parent = -1;
+    uint32_t parent_gen = 0;
+    std::vector<int32_t> tokens;
+    bool operator<(const PrefixKey &o) const
+    {
+        if (parent != o.parent) return parent < o.parent;
+        if (parent_gen != o.parent_gen) return parent_gen < o.parent_gen;
+        return tokens < o.tokens;
+    }
+};
+
 }  // namespace
 
 struct pa_alloc {
@@ -42,18 +68,57 @@ struct pa_alloc {
     std::vector<int32_t> refcnt;
     std::unordered_map<int64_t, Sequence> seqs;
     int64_t next_id = 0;
+    // prefix cache
+    std::map<PrefixKey, int32_t> cache;                // key -> block
+    std::vector<const PrefixKey *> key_of;             // block -> its key in `cache`, or null
+    std::vector<uint32_t> gen;                         // block -> generation (bumped on eviction)
+    std::list<int32_t> evictable;                      // cached blocks with count 0, oldest first
+    std::vector<std::list<int32_t>::iterator> lru_pos; // block -> position in `evictable`
+    std::vector<char> in_lru;
+    int64_t hit_tokens = 0, miss_tokens = 0;
 
+    int64_t available() const { return (int64_t)free_stack.size() + (int64_t)evictable.size(); }
+
+    // A block for new data: the free pool first, else the least recently released cached block,
+    // which leaves the cache.  Caller has checked available() > 0.
     int32_t take()
     {
-        const int32_t b = free_stack.back();
-        free_stack.pop_back();
+        int32_t b;
+        if (!free_stack.empty()) {
+            b = free_stack.back();
+            free_stack.pop_back();
+        } else {
+            b = evictable.front();
+            evictable.pop_front();
+            in_lru[b] = 0;
+            cache.erase(cache.find(*key_of[b]));
+            key_of[b] = nullptr;
+            ++gen[b];
+        }
         refcnt[b] = 1;
         return b;
     }
 
     void release(int32_t b)
     {
-        if (--refcnt[b] == 0) free_stack.push_back(b);
+        if (--refcnt[b] == 0) {
+            if (key_of[b] != nullptr) {
+                lru_pos[b] = evictable.insert(evictable.end(), b);
+                in_lru[b] = 1;
+            } else {
+                free_stack.push_back(b);
+            }
+        }
+    }
+
+    // Another holder for block b (a prefix hit): an evictable block leaves the LRU list.
+    void retain(int32_t b)
+    {
+        if (refcnt[b] == 0 && in_lru[b]) {
+            evictable.erase(lru_pos[b]);
+            in_lru[b] = 0;
+        }
+        ++refcnt[b];
     }
 
     // Fresh blocks needed to grow `s` by n tokens, and whether the first write copies.
@@ -99,6 +164,10 @@ pa_alloc *pa_alloc_create(int num_blocks, int block_size, uint64_t seed)
     a->num_blocks = num_blocks;
     a->block_size = block_size;
     a->refcnt.assign(num_blocks, 0);
+    a->key_of.assign(num_blocks, nullptr);
+    a->gen.assign(num_blocks, 0);
+    a->lru_pos.resize(num_blocks);
+    a->in_lru.assign(num_blocks, 0);
     std::vector<int32_t> order(num_blocks);
     for (int i = 0; i < num_blocks; ++i) order[i] = i;
     if (seed != 0) {
@@ -129,7 +198,7 @@ int pa_alloc_append_n(pa_alloc *a, int64_t seq, int n, int64_t *slots, int64_t *
     auto it = a->seqs.find(seq);
     if (it == a->seqs.end()) return PA_ERR_NOT_FOUND;
     bool cow = false;
-    if (a->blocks_needed(it->second, n, cow) > (int64_t)a->free_stack.size()) return PA_ERR_OOM;
+    if (a->blocks_needed(it->second, n, cow) > a->available()) return PA_ERR_OOM;
     a->grow(it->second, n, slots, cow_src, cow_dst);
     return PA_OK;
 }
@@ -163,7 +232,7 @@ int pa_alloc_append_batch(pa_alloc *a, const int64_t *seqs, int n, int64_t *slot
             }
         }
     }
-    if (need > (int64_t)a->free_stack.size()) return PA_ERR_OOM;
+    if (need > a->available()) return PA_ERR_OOM;
     int ncow = 0;
     for (int i = 0; i < n; ++i) {
         int64_t src = -1, dst = -1;
@@ -242,7 +311,7 @@ int pa_alloc_stats(const pa_alloc *a, int *free_blocks, int *used_blocks, int *s
     int64_t frag = 0;
     for (const auto &kv : a->seqs)
         frag += (int64_t)kv.second.blocks.size() * a->block_size - kv.second.len;
-    if (free_blocks) *free_blocks = (int)a->free_stack.size();
+    if (free_blocks) *free_blocks = (int)a->available();
     if (used_blocks) *used_blocks = used;
     if (shared_blocks) *shared_blocks = shared;
     if (frag_tokens) *frag_tokens = frag;
@@ -253,6 +322,86 @@ int pa_alloc_refcount(const pa_alloc *a, int block)
 {
     if (!a || block < 0 || block >= a->num_blocks) return PA_ERR_INVALID_ARG;
     return a->refcnt[block];
+}
+
+int pa_alloc_new_seq_prefix(pa_alloc *a, const int32_t *tokens, int n, int64_t *seq_id, int64_t *slots,
+                            int *cached_tokens)
+{
+    if (!a || n < 0 || (n > 0 && !tokens) || !seq_id || !cached_tokens) return PA_ERR_INVALID_ARG;
+    const int bs = a->block_size;
+    const int full = n / bs, total = (n + bs - 1) / bs;
+    // walk the prompt's full blocks through the cache (no state change yet)
+    std::vector<int32_t> hits;
+    int64_t hit_evictable = 0;
+    PrefixKey key;
+    for (int k = 0; k < full; ++k) {
+        key.tokens.assign(tokens + (size_t)k * bs, tokens + (size_t)(k + 1) * bs);
+        auto it = a->cache.find(key);
+        if (it == a->cache.end()) break;
+        const int32_t b = it->second;
+        hits.push_back(b);
+        hit_evictable += a->refcnt[b] == 0;
+        key.parent = b;
+        key.parent_gen = a->gen[b];
+    }
+    const int64_t fresh = total - (int64_t)hits.size();
+    if (fresh > a->available() - hit_evictable) return PA_ERR_OOM;
+
+    Sequence s;
+    for (int32_t b : hits) {
+        a->retain(b);
+        s.blocks.push_back(b);
+    }
+    for (int k = (int)hits.size(); k < total; ++k) {
+        const int32_t b = a->take();
+        s.blocks.push_back(b);
+        if (k < full) {                           // a full prompt block: register it
+            PrefixKey nk;
+            nk.parent = k > 0 ? s.blocks[k - 1] : -1;
+            nk.parent_gen = k > 0 ? a->gen[s.blocks[k - 1]] : 0;
+            nk.tokens.assign(tokens + (size_t)k * bs, tokens + (size_t)(k + 1) * bs);
+            auto ins = a->cache.emplace(std::move(nk), b);
+            a->key_of[b] = &ins.first->first;
+        }
+    }
+    s.len = n;
+    if (slots)
+        for (int t = 0; t < n; ++t) slots[t] = (int64_t)s.blocks[t / bs] * bs + t % bs;
+    const int cached = (int)hits.size() * bs;
+    a->hit_tokens += cached;
+    a->miss_tokens += n - cached;
+    const int64_t id = a->next_id++;
+    a->seqs.emplace(id, std::move(s));
+    *seq_id = id;
+    *cached_tokens = cached;
+    return PA_OK;
+}
+
+int pa_alloc_prefix_stats(const pa_alloc *a, int64_t *hit_tokens, int64_t *miss_tokens, int *cached_blocks,
+                          int *evictable_blocks)
+{
+    if (!a) return PA_ERR_INVALID_ARG;
+    if (hit_tokens) *hit_tokens = a->hit_tokens;
+    if (miss_tokens) *miss_tokens = a->miss_tokens;
+    if (cached_blocks) *cached_blocks = (int)a->cache.size();
+    if (evictable_blocks) *evictable_blocks = (int)a->evictable.size();
+    return PA_OK;
+}
+
+int pa_alloc_order_by_prefix(const pa_alloc *a, const int64_t *seqs, int n, int32_t *order)
+{
+    if (!a || n < 0 || (n > 0 && (!seqs || !order))) return PA_ERR_INVALID_ARG;
+    std::vector<const Sequence *> sq(n);
+    for (int i = 0; i < n; ++i) {
+        auto it = a->seqs.find(seqs[i]);
+        if (it == a->seqs.end()) return PA_ERR_NOT_FOUND;
+        sq[i] = &it->second;
+    }
+    std::vector<int32_t> idx(n);
+    std::iota(idx.begin(), idx.end(), 0);
+    std::stable_sort(idx.begin(), idx.end(), [&](int32_t x, int32_t y) { return sq[x]->blocks < sq[y]->blocks; });
+    std::copy(idx.begin(), idx.end(), order);
+    return PA_OK;
 }
 
 }  // extern "C"

@@ -62,6 +62,15 @@ def test_shared_prefix_4x8(orc, seed):
     _full_parity(orc, case)
 
 
+@pytest.mark.parametrize("name", ["shared_prefix_16x8", "shared_prefix_16x8_interleaved"])
+def test_shared_prefix_16x8_sampled(orc, name):
+    case = workloads.make_case(name, 0, device=DEV)
+    g = torch.Generator().manual_seed(3)
+    seqs = sorted(set(torch.randint(0, case.B, (6,), generator=g).tolist()))
+    rows = [(s, h) for s in seqs for h in (0, 9, 31)]
+    _full_parity(orc, case, rows=rows)
+
+
 @pytest.mark.parametrize("bs", [16, 32, 64])
 def test_fp8_mha_b32_sampled_full_size(orc, bs):
     case = workloads.make_case("fp8_mha_b32_bs%d" % bs, 0, device=DEV)

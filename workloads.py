@@ -18,6 +18,8 @@ long_context_b8        8 seqs, 32 / 8 heads, d 128, bf16, bs 16, ctx ~ U{32768..
                        split-context partitions of 512 tokens
 shared_prefix_4x8      4 prompts x 2048 tokens, each shared by 8 samples through
                        identical physical ids; private tails ~ U{0..256}
+shared_prefix_16x8     16 prompts x 8 samples (unique prompt KV > L2), sharers adjacent;
+ _interleaved          the same batch with each prompt's sharers 16 rows apart
 fp8_mha_b32_bs{16,32,64}  32 seqs, 32 q / 32 kv heads, d 128, E4M3 cache with a
                        per-tensor fp32 scale max|x|/448, ctx 4096
 int8_mha_b32_bs{16,32,64} the same shape with an INT8 cache, per-tensor scale max|x|/127
@@ -52,6 +54,13 @@ CONFIGS = {
                             ctx_range=(32768, 131072), pool_factor=1.0, partition=512),
     "shared_prefix_4x8": dict(prompts=4, samples=8, prompt_len=2048, tail_range=(0, 256), h_q=32,
                               h_kv=8, d=128, bs=16, cache="bf16", partition=512),
+    # 16 prompts x 8 samples: ~134 MB of unique prompt KV, more than L2; sharers adjacent in the
+    # batch ("grouped", the order pa_alloc_order_by_prefix gives) or spread over it
+    "shared_prefix_16x8": dict(prompts=16, samples=8, prompt_len=2048, tail_range=(0, 256), h_q=32,
+                               h_kv=8, d=128, bs=16, cache="bf16", partition=512),
+    "shared_prefix_16x8_interleaved": dict(prompts=16, samples=8, prompt_len=2048, tail_range=(0, 256), h_q=32,
+                                           h_kv=8, d=128, bs=16, cache="bf16", partition=512,
+                                           order="interleaved"),
     "fp8_mha_b32_bs16": dict(B=32, h_q=32, h_kv=32, d=128, bs=16, cache="e4m3", ctx_fixed=4096,
                              pool_factor=1.0, partition=512),
     "fp8_mha_b32_bs32": dict(B=32, h_q=32, h_kv=32, d=128, bs=32, cache="e4m3", ctx_fixed=4096,
@@ -169,7 +178,7 @@ def make_case(name: str, seed: int = 0, device="cpu", **over) -> DecodeCase:
     device = torch.device(device)
     gc = _cpu_gen(seed)                    # structure (lengths, block order) always from the CPU stream
 
-    if name == "shared_prefix_4x8":
+    if "prompts" in cfg:
         return _make_shared_prefix(name, cfg, seed, device, gc)
 
     B, h_q, h_kv, d, bs = cfg["B"], cfg["h_q"], cfg["h_kv"], cfg["d"], cfg["bs"]
@@ -282,6 +291,10 @@ def _make_shared_prefix(name, cfg, seed, device, gc) -> DecodeCase:
             n = private[s]
             tables[s, pblocks:pblocks + n] = torch.tensor(order[pos:pos + n], dtype=torch.int32)
             pos += n
+    if cfg.get("order") == "interleaved":
+        # batch row r holds sample r // P of prompt r % P: a prompt's sharers are P rows apart
+        perm = torch.tensor([p * S + j for j in range(S) for p in range(P)])
+        tables, cached, ctx = tables[perm], cached[perm], ctx[perm]
     slots = torch.tensor([int(tables[s, int(cached[s]) // bs]) * bs + int(cached[s]) % bs
                           for s in range(B)], dtype=torch.int64)
     owned = _owned_slot_mask(tables, cached, nb, bs)
