@@ -2,6 +2,7 @@
 contiguous scheme that reserves the whole context window per request.
 
     python -m paged_kv_cache_428_b200.memory_report --trace chat_w2048_b64 [--seed 0] [--per-step]
+    python -m paged_kv_cache_428_b200.memory_report --prefix sys256_doc1536x4_q64_n64
 
 Contiguous pre-allocation keeps the window reserved for every request for its whole life
 ("深度解构 LLM 推理优化…" section 1.2, Internal Fragmentation / Reservation Gap; intelliparadigm
@@ -78,6 +79,24 @@ def summarise(records) -> dict:
             "max_seq_waste": max((r["worst_seq_waste"] for r in records), default=0)}
 
 
+def run_prefix_prompts(prompts, bs: int, seed: int = 0) -> dict:
+    """Insert every prompt with prefix caching (all requests alive together) and report the
+    prompt tokens found cached (prefill skipped), and the blocks held against the blocks the
+    same requests would hold without sharing (sum of ceil(len / bs))."""
+    pool = sum(-(-len(p) // bs) for p in prompts)
+    alloc = BlockAllocator(pool, bs, seed)
+    try:
+        cached = [alloc.new_seq_prefix(p)[2] for p in prompts]
+        used, ps = alloc.stats()["used"], alloc.prefix_stats()
+    finally:
+        alloc.close()
+    total = sum(len(p) for p in prompts)
+    return {"requests": len(prompts), "prompt_tokens": total, "cached_tokens": sum(cached),
+            "prefill_skipped": round(sum(cached) / total, 6), "blocks_shared": used, "blocks_private": pool,
+            "memory_saving": round(1.0 - used / pool, 6), "hit_tokens": ps["hit_tokens"],
+            "miss_tokens": ps["miss_tokens"]}
+
+
 def capacity_report(budget_bytes: int, layers: int, h_kv: int, head_dim: int) -> dict:
     return {"budget_bytes": budget_bytes,
             "tokens_bf16": pa_kv_capacity_tokens(budget_bytes, layers, h_kv, head_dim, 2),
@@ -90,7 +109,17 @@ def main(argv=None) -> int:
     ap.add_argument("--trace", default="chat_w2048_b64", choices=sorted(workloads.TRACES))
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--per-step", action="store_true")
+    ap.add_argument("--prefix", default=None, choices=sorted(workloads.PREFIX_TRACES),
+                    help="report prefix caching on prompts sharing a system prompt and documents")
     a = ap.parse_args(argv)
+    if a.prefix:
+        bs = workloads.PREFIX_TRACES[a.prefix]["bs"]
+        out = {"prefix_trace": a.prefix, "seed": a.seed, "block_size": bs,
+               "same_document_front": run_prefix_prompts(workloads.make_prefix_prompts(a.prefix, a.seed), bs, a.seed),
+               "document_front_changed": run_prefix_prompts(
+                   workloads.make_prefix_prompts(a.prefix, a.seed, front_changed=True), bs, a.seed)}
+        print(json.dumps(out))
+        return 0
     t = workloads.make_trace(a.trace, a.seed)
     rec = run_trace(t.prompts, t.outputs, t.slots, t.window, t.bs, a.seed)
     out = {"trace": a.trace, "seed": a.seed, "requests": len(t.prompts), "slots": t.slots, "window": t.window,

@@ -160,3 +160,28 @@ def test_order_by_prefix_groups_sharers():
     groups = [0 if i % 2 == 0 else 1 for i in order]
     assert groups in ([0, 0, 0, 1, 1, 1], [1, 1, 1, 0, 0, 0])
     assert sorted(order) == list(range(6))
+
+
+def test_prefix_report_matches_closed_form_and_model():
+    """System prompt (256) + one of 4 documents (1536) + a question: after the first request of
+    a document, each request finds system + document cached (1792 tokens, 112 whole blocks); the
+    first request of every other document finds the system prompt; changing each document's
+    first tokens leaves only the system prompt to hit."""
+    import workloads
+    from paged_kv_cache_428_b200 import memory_report
+    name = "sys256_doc1536x4_q64_n64"
+    bs = workloads.PREFIX_TRACES[name]["bs"]
+    prompts = workloads.make_prefix_prompts(name, 0)
+    docs_seen, want = set(), 0
+    for i, p in enumerate(prompts):
+        doc = tuple(p[256:256 + 1536])
+        want += 0 if i == 0 else (1792 if doc in docs_seen else 256)
+        docs_seen.add(doc)
+    rep = memory_report.run_prefix_prompts(prompts, bs)
+    assert rep["cached_tokens"] == want
+    m = AllocatorModel(sum(-(-len(p) // bs) for p in prompts), bs, 0)
+    assert [m.new_seq_prefix(p)[2] for p in prompts] and m.hit_tokens == rep["hit_tokens"]
+    assert m.stats()["used"] == rep["blocks_shared"]
+    changed = memory_report.run_prefix_prompts(workloads.make_prefix_prompts(name, 0, front_changed=True), bs)
+    assert changed["cached_tokens"] == 256 * (len(prompts) - 1)
+    assert rep["prefill_skipped"] > 0.9 and changed["prefill_skipped"] < 0.15

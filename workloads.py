@@ -355,3 +355,29 @@ def make_trace(name: str, seed: int = 0, **over) -> Trace:
     if any(a + b > cfg["window"] for a, b in zip(p, o)):
         raise ValueError("a request exceeds the window")
     return Trace(name=name, prompts=p, outputs=o, slots=cfg["slots"], window=cfg["window"], bs=cfg["bs"])
+
+
+# ------------------------------------------------------------------ prompts sharing a prefix
+# Prompt token ids for the prefix-caching measurement: a system prompt, then one of a few long
+# documents, then a short question ("vLLM 推理原理…" section 前缀缓存能省掉哪部分工作: fix the
+# system text and the document, vary only the final question).  With front_changed=True every
+# request's document gets its own first tokens, so only the system prompt can match.
+PREFIX_TRACES = {
+    "sys256_doc1536x4_q64_n64": dict(requests=64, system=256, docs=4, doc=1536, question=(16, 64), bs=16),
+}
+
+
+def make_prefix_prompts(name: str, seed: int = 0, front_changed: bool = False) -> list:
+    cfg = PREFIX_TRACES[name]
+    g = _cpu_gen(seed)
+    vocab = 32000
+    system = torch.randint(0, vocab, (cfg["system"],), generator=g).tolist()
+    docs = [torch.randint(0, vocab, (cfg["doc"],), generator=g).tolist() for _ in range(cfg["docs"])]
+    prompts = []
+    for i in range(cfg["requests"]):
+        doc = list(docs[int(torch.randint(0, cfg["docs"], (1,), generator=g))])
+        if front_changed:
+            doc[:8] = torch.randint(0, vocab, (8,), generator=g).tolist()
+        nq = int(torch.randint(cfg["question"][0], cfg["question"][1] + 1, (1,), generator=g))
+        prompts.append(system + doc + torch.randint(0, vocab, (nq,), generator=g).tolist())
+    return prompts
