@@ -99,6 +99,9 @@ class Oracle:
         L.or_paged_decode.restype = i32
         L.or_paged_decode.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32, i32,
                                       f64, i32, vp, vp]
+        L.or_paged_prefill_rows.restype = i32
+        L.or_paged_prefill_rows.argtypes = [vp, vp, i32, vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, i32, i32,
+                                            f64, i32, vp, vp]
         L.or_paged_decode_rows.restype = i32
         L.or_paged_decode_rows.argtypes = [vp, vp, i32, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32,
                                            i32, f64, i32, vp, vp]
@@ -223,6 +226,33 @@ class Oracle:
         if rc:
             raise ValueError("oracle paged_decode_rows failed with code %d" % rc)
         return out
+
+    # -- prefill (chunked) attention -----------------------------------------
+    def paged_prefill(self, q_bits, k_cache, v_cache, block_tables, query_start, context_lens, *, h_kv: int,
+                      bs: int, scale: float, rows=None, cache: str | None = None, k_scale=1.0,
+                      v_scale=1.0) -> np.ndarray:
+        """Causal attention of every chunk row over its sequence's paged cache.  q [T, h_q, d];
+        query_start [B+1]; context_lens [B] (including the chunk).  rows: (query row, head)
+        pairs -> [len(rows), d]; None -> all rows, [T, h_q, d]."""
+        dt = _cache_code(cache, False)
+        q = np.ascontiguousarray(q_bits, dtype=np.uint16)
+        T, h_q, d = q.shape
+        qs = np.ascontiguousarray(query_start, dtype=np.int32)
+        ctx = np.ascontiguousarray(context_lens, dtype=np.int32)
+        tab = np.ascontiguousarray(block_tables, dtype=np.int32)
+        full = rows is None
+        if full:
+            rows = [(t, h) for t in range(T) for h in range(h_q)]
+        pr = np.ascontiguousarray(rows, dtype=np.int32).reshape(-1, 2)
+        ks, vs = _head_scales(k_scale, h_kv), _head_scales(v_scale, h_kv)
+        out = np.empty((pr.shape[0], d), dtype=np.float64)
+        rc = self._L.or_paged_prefill_rows(out.ctypes.data, pr.ctypes.data, pr.shape[0], q.ctypes.data,
+                                           k_cache.ctypes.data, v_cache.ctypes.data, tab.ctypes.data, tab.shape[1],
+                                           qs.ctypes.data, ctx.ctypes.data, ctx.shape[0], h_q, h_kv, d, bs,
+                                           k_cache.shape[0], scale, dt, ks.ctypes.data, vs.ctypes.data)
+        if rc:
+            raise ValueError("oracle paged_prefill failed with code %d" % rc)
+        return out.reshape(T, h_q, d) if full else out
 
 
 def load(lib_path: os.PathLike | None = None) -> Oracle:

@@ -339,6 +339,87 @@ int or_paged_decode_rows(double *out, const int32_t *pairs, int npairs,
 }
 
 /* ------------------------------------------------------------------------ */
+/* Prefill / chunked-prefill attention                                        */
+/* ------------------------------------------------------------------------ */
+
+/* One prefill output row: query row `row` (of all chunks stacked: q[T][h_q][d]) belongs to
+ * sequence s, whose chunk holds rows query_start[s] .. query_start[s+1]-1 and ends at the
+ * sequence's last cached token, so row i of the chunk sits at absolute position
+ * p = context_lens[s] - chunk_len + i.  The row attends causally: tokens 0..p of sequence s,
+ * read through the block table, in fp64.
+ * "vLLM 推理原理…" section 一次生成有两个阶段 (prefill processes the input tokens and builds
+ * their KV; chunked prefill splits a long input into pieces scheduled with decoding);
+ * "现代 AI…" section 1 (attention formula); "深度解构…" section 2.1 (block table). */
+static int prefill_row(double *out_row, int s, int i, int h, const uint16_t *qrow,
+                       const void *k_cache, const void *v_cache, const int32_t *block_tables,
+                       int max_blocks_per_seq, int ctx, int chunk, int h_q, int h_kv, int d, int bs,
+                       int num_blocks, double scale, int cache_dtype, const float *k_scales,
+                       const float *v_scales)
+{
+    const int group = h_q / h_kv;
+    const int kh = h / group;                 /* KV head of query head h */
+    int p = ctx - chunk + i;                  /* absolute position of this query token */
+    int n = p + 1;                            /* tokens it attends to */
+    const double ks = cache_dtype ? (double)k_scales[kh] : 1.0;
+    const double vs = cache_dtype ? (double)v_scales[kh] : 1.0;
+    for (int e = 0; e < d; ++e) out_row[e] = 0.0;
+    if (p < 0) return -7;
+    if ((n + bs - 1) / bs > max_blocks_per_seq) return -2;
+    double *score = (double *)malloc(sizeof(double) * (size_t)n);
+    if (!score) return -3;
+    double top = -INFINITY;
+    for (int j = 0; j < n; ++j) {
+        const int32_t blk = block_tables[(size_t)s * max_blocks_per_seq + j / bs];
+        if (blk < 0 || blk >= num_blocks) { free(score); return -1; }
+        double acc = 0.0;
+        for (int e = 0; e < d; ++e)
+            acc += or_bf16_decode(qrow[e]) *
+                   cache_elem(k_cache, cache_index(blk, kh, j % bs, e, h_kv, bs, d), cache_dtype, ks);
+        score[j] = acc * scale;
+        if (score[j] > top) top = score[j];
+    }
+    double total = 0.0;
+    for (int j = 0; j < n; ++j) {
+        const double wj = exp(score[j] - top);
+        const int32_t blk = block_tables[(size_t)s * max_blocks_per_seq + j / bs];
+        total += wj;
+        for (int e = 0; e < d; ++e)
+            out_row[e] += wj * cache_elem(v_cache, cache_index(blk, kh, j % bs, e, h_kv, bs, d), cache_dtype, vs);
+    }
+    for (int e = 0; e < d; ++e) out_row[e] = out_row[e] / total;
+    free(score);
+    return 0;
+}
+
+/* Selected prefill rows: rows[2*r] = query row (0..T-1), rows[2*r+1] = query head;
+ * out[r][d] (fp64).  q: [T][h_q][d] bf16 bits; query_start: [B+1]; context_lens: [B] (each
+ * including its chunk).  Returns 0, -1 on a bad block id, -2 on a context longer than the
+ * table row, -4 on a bad head split, -5 on a bad type, -6 on a row outside every chunk, -7 on
+ * a chunk longer than its context. */
+int or_paged_prefill_rows(double *out, const int32_t *rows, int nrows, const uint16_t *q,
+                          const void *k_cache, const void *v_cache, const int32_t *block_tables,
+                          int max_blocks_per_seq, const int32_t *query_start, const int32_t *context_lens,
+                          int B, int h_q, int h_kv, int d, int bs, int num_blocks, double scale,
+                          int cache_dtype, const float *k_scales, const float *v_scales)
+{
+    if (h_kv <= 0 || h_q % h_kv != 0) return -4;
+    if (cache_dtype < 0 || cache_dtype > 2) return -5;
+    for (int r = 0; r < nrows; ++r) {
+        int row = rows[2 * r], h = rows[2 * r + 1];
+        int s = -1;
+        for (int b = 0; b < B; ++b)
+            if (row >= query_start[b] && row < query_start[b + 1]) { s = b; break; }
+        if (s < 0) return -6;
+        int chunk = query_start[s + 1] - query_start[s];
+        int rc = prefill_row(out + (size_t)r * d, s, row - query_start[s], h, q + ((size_t)row * h_q + h) * d,
+                             k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens[s], chunk,
+                             h_q, h_kv, d, bs, num_blocks, scale, cache_dtype, k_scales, v_scales);
+        if (rc) return rc;
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
 /* Array forms of the codecs (plain loops over the scalar definitions above). */
 /* ------------------------------------------------------------------------ */
 

@@ -456,6 +456,58 @@ def pin_fp8_decode_per_head(orc):
     np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-13)
 
 
+def _prefill_case(seed, B, h_q, h_kv, d, bs, cached_lens, chunk_lens):
+    """Contiguous K/V rows of each sequence (cached + chunk), scattered through tables, and the
+    chunk's query rows stacked as [T, h_q, d]."""
+    g = torch.Generator().manual_seed(seed)
+    ctxs = [c + n for c, n in zip(cached_lens, chunk_lens)]
+    ks = [torch.randn(n, h_kv, d, generator=g).to(torch.bfloat16) for n in ctxs]
+    vs = [torch.randn(n, h_kv, d, generator=g).to(torch.bfloat16) for n in ctxs]
+    q = torch.randn(sum(chunk_lens), h_q, d, generator=g).to(torch.bfloat16)
+    nb = sum(-(-n // bs) for n in ctxs) + 2
+    order = torch.randperm(nb, generator=g).tolist()
+    kp, vp, table = build_paged(ks, vs, order, bs, nb)
+    qstart = np.concatenate([[0], np.cumsum(chunk_lens)]).astype(np.int32)
+    return q, ks, vs, kp, vp, table, qstart, ctxs
+
+
+def pin_prefill_vs_masked_sdpa(orc):
+    """Chunked prefill: row i of a chunk of n rows ending at the sequence's last token attends
+    to tokens 0 .. ctx - n + i; against fp64 SDPA with that causal mask on contiguous rows
+    (a whole prompt, cached = 0, is plain causal attention)."""
+    for seed, (h_q, h_kv, d, bs, cached, chunk) in enumerate([
+            (4, 2, 64, 16, [0, 20, 37], [5, 17, 40]),
+            (8, 1, 128, 32, [64, 0], [1, 33]),
+            (4, 4, 64, 16, [3], [16])]):
+        q, ks, vs, kp, vp, table, qstart, ctxs = _prefill_case(seed, len(chunk), h_q, h_kv, d, bs, cached, chunk)
+        scale = 1.0 / math.sqrt(d)
+        got = orc.paged_prefill(_bits(q), _bits(kp), _bits(vp), table.numpy(), qstart, np.array(ctxs, np.int32),
+                                h_kv=h_kv, bs=bs, scale=scale)
+        for s_ in range(len(chunk)):
+            n, ctx = chunk[s_], ctxs[s_]
+            qq = q[qstart[s_]:qstart[s_ + 1]].to(torch.float64).transpose(0, 1)[None]      # [1, h_q, n, d]
+            kk = ks[s_].to(torch.float64).transpose(0, 1)[None]
+            vv = vs[s_].to(torch.float64).transpose(0, 1)[None]
+            mask = torch.arange(ctx)[None, :] <= (ctx - n + torch.arange(n))[:, None]   # [n, ctx]
+            want = F.scaled_dot_product_attention(qq, kk, vv, attn_mask=mask, scale=scale, enable_gqa=True)
+            np.testing.assert_allclose(got[qstart[s_]:qstart[s_ + 1]], want[0].transpose(0, 1).numpy(),
+                                       rtol=1e-12, atol=1e-13)
+            if cached[s_] == 0:
+                causal = F.scaled_dot_product_attention(qq, kk, vv, is_causal=True, scale=scale, enable_gqa=True)
+                np.testing.assert_allclose(got[qstart[s_]:qstart[s_ + 1]], causal[0].transpose(0, 1).numpy(),
+                                           rtol=1e-12, atol=1e-13)
+
+
+def pin_prefill_chunk_of_one_is_decode(orc):
+    """A one-token chunk is a decode step: the same row as or_paged_decode."""
+    h_q, h_kv, d, bs = 8, 2, 64, 16
+    q, ks, vs, kp, vp, table, qstart, ctxs = _prefill_case(41, 3, h_q, h_kv, d, bs, [10, 0, 47], [1, 1, 1])
+    kw = dict(h_kv=h_kv, bs=bs, scale=0.3)
+    pre = orc.paged_prefill(_bits(q), _bits(kp), _bits(vp), table.numpy(), qstart, np.array(ctxs, np.int32), **kw)
+    dec = orc.paged_decode(_bits(q), _bits(kp), _bits(vp), table.numpy(), np.array(ctxs, np.int32), **kw)
+    assert np.array_equal(pre, dec)
+
+
 def pin_decode_rows_subset(orc):
     B, h_q, h_kv, d, bs = 3, 8, 4, 64, 16
     q, ks, vs, order, nb, ctxs = _random_decode(31, B, h_q, h_kv, d, bs, ctxs=[20, 50, 3])
@@ -495,6 +547,14 @@ def test_fp8_decode(orc):
 
 def test_decode_rows_subset(orc):
     pin_decode_rows_subset(orc)
+
+
+def test_prefill_vs_masked_sdpa(orc):
+    pin_prefill_vs_masked_sdpa(orc)
+
+
+def test_prefill_chunk_of_one_is_decode(orc):
+    pin_prefill_chunk_of_one_is_decode(orc)
 
 
 def test_int8_decode_per_head(orc):
@@ -596,6 +656,7 @@ ALL_PINS = [pin_closed_forms, pin_bf16_codec, pin_e4m3_codec, pin_int8_codec, pi
             pin_decode_vs_sdpa, pin_decode_brute_force, pin_decode_special_cases,
             pin_worked_block_table_example, pin_permutation_invariance, pin_fp8_decode,
             pin_int8_decode_per_head, pin_fp8_decode_per_head, pin_decode_rows_subset,
+            pin_prefill_vs_masked_sdpa, pin_prefill_chunk_of_one_is_decode,
             pin_reshape_and_cache, pin_copy_blocks]
 
 MUTANTS = {
@@ -623,6 +684,16 @@ MUTANTS = {
                              "double or_int8_decode(int8_t c) { return (double)(uint8_t)c; }"),
     "per_head_scale_index": ("double k_scale = cache_dtype ? (double)k_scales[kvh] : 1.0;",
                              "double k_scale = cache_dtype ? (double)k_scales[0] : 1.0;"),
+    "prefill_causal_off_by_one": ("int n = p + 1;                            /* tokens it attends to */",
+                                  "int n = p;                                /* tokens it attends to */"),
+    "prefill_gqa_mapping": ("const int kh = h / group;", "const int kh = h % h_kv;"),
+    "prefill_dropped_scale": ("score[j] = acc * scale;", "score[j] = acc;"),
+    "prefill_softmax_sign": ("const double wj = exp(score[j] - top);", "const double wj = exp(top - score[j]);"),
+    "prefill_kv_swapped": ("out_row[e] += wj * cache_elem(v_cache", "out_row[e] += wj * cache_elem(k_cache"),
+    "prefill_table_index": ("const int32_t blk = block_tables[(size_t)s * max_blocks_per_seq + j / bs];\n        if (blk",
+                            "const int32_t blk = block_tables[(size_t)s * max_blocks_per_seq + j % bs];\n        if (blk"),
+    "prefill_chunk_position": ("int p = ctx - chunk + i;                  /* absolute position of this query token */",
+                               "int p = ctx - chunk;                      /* absolute position of this query token */"),
     "per_head_encode_index": ("or_int8_encode_sat(or_div_f32(vx, v_scales[h]))",
                               "or_int8_encode_sat(or_div_f32(vx, v_scales[0]))"),
 }
