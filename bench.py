@@ -577,9 +577,117 @@ def run_reference(args):
             "e2e": {"value": round(value, 5), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+# ---------------------------------------------------------------------------- prefill mode
+def measured_bf16_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured (cuBLAS bf16 burst)"
+    return 1590.0, "fallback"
+
+
+def run_prefill(args):
+    """--workload prefill_*: each step writes the chunks' K/V (pa_reshape_and_cache of every
+    chunk token) and runs pa_prefill; reported as attention TFLOP/s against the bf16 peak."""
+    import torch
+    import workloads
+    import paged_kv_cache_428_b200 as pa
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = init_dist(world, "nccl")
+    seed = shard_seeds(args.seed, world)[rank]
+    case = workloads.make_prefill_case(args.workload, seed, device=dev)
+    kc, vc = case.k_cache, case.v_cache
+    out = torch.empty_like(case.q)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    L, sp = pa.lib(), stream.cuda_stream
+    rargs = pa.reshape_call_args(case.key_new, case.value_new, kc, vc, case.slot_mapping)
+    pargs = pa.prefill_call_args(out, case.q, kc, vc, case.block_tables, case.query_start, case.context_lens,
+                                 case.max_query_len, case.scale)
+
+    def timed(calls, n_steps):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_steps)]
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        with torch.cuda.stream(stream):
+            for i in range(n_steps):
+                if not args.warm_l2:
+                    flush.zero_()
+                evs[i][0].record(stream)
+                rc = 0
+                for fn, a in calls:
+                    rc |= fn(*a, sp)
+                evs[i][1].record(stream)
+                if rc:
+                    raise SystemExit("library call failed: %d" % rc)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        return sum(a.elapsed_time(b) for a, b in evs)
+
+    step = [(L.pa_reshape_and_cache, rargs), (L.pa_prefill, pargs)]
+    timed(step, args.warmup)
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+    time.sleep(0.3)
+    t0 = time.time()
+    step_ms = timed(step, args.steps)
+    t1 = time.time()
+    kern_ms = timed([(L.pa_prefill, pargs)], args.steps)
+    t2 = time.time()
+    time.sleep(0.1)
+    sampler.stop()
+    errs = pa.pa_device_errors(clear=True)
+    if errs:
+        raise SystemExit("device error bits 0x%x during the benchmark" % errs)
+    flops = float(case.attention_flops())
+    T = float(case.q.shape[0])
+    step_ms, kern_ms = max_over_ranks([step_ms, kern_ms], world, dev)
+    tot_flops, tot_tok = sum_over_ranks([flops, T], world, dev)
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return None
+    K = args.steps
+    peak, kind = measured_bf16_peak()
+    achieved = flops / (kern_ms / 1e3 / K) / 1e12
+    line = {
+        "metric": "chunked-prefill attention TFLOP/s over the paged KV cache; prefill tokens/s",
+        "value": round(tot_flops / (step_ms / 1e3 / K) / 1e12, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(step_ms / K, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16 in, fp32 accumulate", "data": "synthetic",
+        "config": {"workload": args.workload, "num_seqs": case.B, "h_q": case.h_q, "h_kv": case.h_kv,
+                   "head_dim": case.d, "block_size": case.bs, "chunk_tokens": int(T),
+                   "cached_tokens": case.meta["cached"], "chunk_lens": case.meta["chunk"],
+                   "attention_flops_per_step": int(flops),
+                   "step": "reshape_and_cache(all chunk tokens) + pa_prefill",
+                   "l2": ("warm: no flush between steps" if args.warm_l2 else
+                          "flushed between steps (2x L2 write, outside the events)")},
+        "tokens_per_s": round(tot_tok / (step_ms / 1e3 / K), 1),
+        "kernels_ms_alone": {"prefill": round(kern_ms / K, 5)},
+        "roofline": {"bound": "tensor", "kernel": "paged_prefill_kernel (mma.sync bf16)", "achieved": round(achieved, 1),
+                     "peak": peak, "peak_kind": kind, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "traffic": None, "algorithmic_flops_per_launch": int(flops)},
+        "gpu_launches": 2 * K,
+        "clocks": sampler.summary(t0, t1),
+        "clocks_kernel_loops": sampler.summary(t1, t2),
+    }
+    if world > 1:
+        dist.destroy_process_group()
+    return line
+
+
 def main(argv=None):
     args = parse_args(argv)
-    line = run_reference(args) if args.impl == "reference" else run_ours(args)
+    if args.impl != "reference" and args.workload.startswith("prefill_"):
+        line = run_prefill(args)
+    else:
+        line = run_reference(args) if args.impl == "reference" else run_ours(args)
     if line is not None:
         print(json.dumps(line), flush=True)
 

@@ -64,6 +64,7 @@ extern "C" {
 #define PA_DEVERR_BAD_BLOCK 0x2u  /* a block-table entry outside the pool (or row) was skipped */
 #define PA_DEVERR_BAD_PAIR  0x4u  /* a copy pair outside the pool was skipped */
 #define PA_DEVERR_TIMEOUT   0x8u  /* a bounded in-kernel wait ran out */
+#define PA_DEVERR_BAD_CHUNK 0x10u /* a prefill chunk longer than its context was skipped */
 
 typedef enum { PA_CACHE_BF16 = 0, PA_CACHE_E4M3 = 1, PA_CACHE_INT8 = 2 } pa_cache_dtype;
 
@@ -205,6 +206,30 @@ int pa_decode_head_scales(void *out, const void *q, const void *k_cache, const v
                           int num_blocks, float scale, int cache_dtype, const float *k_scales,
                           const float *v_scales, int partition_size, void *workspace, size_t workspace_bytes,
                           void *stream);
+
+/* ---- chunked-prefill attention ---------------------------------------------------
+ * Causal attention of a chunk of new query rows per sequence over the paged cache
+ * ("vLLM 推理原理…" section 一次生成有两个阶段: prefill processes the input tokens and builds
+ * their KV; chunked prefill splits a long input into pieces).  The chunk of sequence s is query
+ * rows query_start[s] .. query_start[s+1]-1 and ends at the sequence's last token: row i of a
+ * chunk of n rows sits at position p = context_lens[s] - n + i and
+ *   out[row][h] = softmax(scale * q[row][h] . K_s[0..p]^T) . V_s[0..p]
+ * with token t of sequence s read from block block_tables[s][t / bs] at offset t % bs and
+ * query head h reading KV head h / (h_q / h_kv).  The chunk's own K/V rows must be in the cache
+ * (pa_reshape_and_cache of the chunk's tokens, e.g. with slots from pa_alloc_append_n).
+ *   out, q         device bf16 [T][h_q][head_dim], T = query_start[num_seqs]
+ *   query_start    device int32 [num_seqs + 1], non-decreasing, query_start[0] = 0
+ *   context_lens   device int32 [num_seqs], each including its chunk (>= the chunk length; a
+ *                  longer chunk leaves its rows unwritten and flags PA_DEVERR_BAD_CHUNK)
+ *   max_query_len  host-known upper bound of the chunk lengths (sizes the grid)
+ *   cache_dtype    PA_CACHE_BF16 (other types: PA_ERR_UNSUPPORTED)
+ * A block-table entry outside the pool is skipped, flags PA_DEVERR_BAD_BLOCK and turns the
+ * affected rows into NaN.  Tensor cores (mma.sync bf16, fp32 accumulate); accuracy as
+ * pa_decode for bf16 caches.  Allocates nothing; needs no workspace. */
+int pa_prefill(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
+               int max_blocks_per_seq, const int32_t *query_start, const int32_t *context_lens, int num_seqs,
+               int max_query_len, int h_q, int h_kv, int head_dim, int block_size, int num_blocks, float scale,
+               int cache_dtype, void *stream);
 
 /* ---- decode without any allocation (static scratch) ---------------------------
  * The pages have no counterpart for this call; it exists for callers that cannot

@@ -35,6 +35,7 @@ PA_DEVERR_BAD_SLOT = 0x1
 PA_DEVERR_BAD_BLOCK = 0x2
 PA_DEVERR_BAD_PAIR = 0x4
 PA_DEVERR_TIMEOUT = 0x8
+PA_DEVERR_BAD_CHUNK = 0x10
 
 STATUS = {0: "PA_OK", -1: "PA_ERR_INVALID_ARG", -2: "PA_ERR_UNSUPPORTED", -3: "PA_ERR_WORKSPACE",
           -4: "PA_ERR_OOM", -5: "PA_ERR_CUDA", -6: "PA_ERR_NOT_FOUND"}
@@ -75,6 +76,7 @@ def _load() -> ctypes.CDLL:
         "pa_decode_static_ws": (i32, [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32, i32, i32, f32, i32,
                                       f32, f32, i32, vp]),
         "pa_copy_blocks": (i32, [vp, vp, i32, vp, i32, sz, i32, vp]),
+        "pa_prefill": (i32, [vp, vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, i32, i32, i32, f32, i32, vp]),
         "pa_device_errors": (i32, [ctypes.POINTER(ctypes.c_uint), i32]),
         "pa_validate_block_tables": (i32, [vp, i32, vp, i32, i32, i32]),
         "pa_validate_slots": (i32, [vp, i32, i32, i32]),
@@ -331,6 +333,37 @@ def pa_decode_static_ws(out, q, k_cache, v_cache, block_tables, context_lens, ma
     args = _decode_args(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len, scale,
                         partition_size, k_scale, v_scale, None)
     _check(_lib.pa_decode_static_ws(*args[:-2], _stream_ptr(stream)), "pa_decode_static_ws")
+    return out
+
+
+def prefill_call_args(out, q, k_cache, v_cache, block_tables, query_start, context_lens, max_query_len: int,
+                      scale: float = None) -> tuple:
+    """Checked raw arguments of pa_prefill (all but the stream)."""
+    _need(out, "out", (torch.bfloat16,), 3)
+    _need(q, "q", (torch.bfloat16,), 3)
+    _need(k_cache, "k_cache", CACHE_DTYPES, 4)
+    _need(v_cache, "v_cache", (k_cache.dtype,), 4)
+    _need(block_tables, "block_tables", (torch.int32,), 2)
+    _need(query_start, "query_start", (torch.int32,), 1)
+    _need(context_lens, "context_lens", (torch.int32,), 1)
+    T, h_q, d = q.shape
+    NB, h_kv, bs, d2 = k_cache.shape
+    B = context_lens.shape[0]
+    if tuple(out.shape) != (T, h_q, d) or d2 != d or tuple(v_cache.shape) != tuple(k_cache.shape) \
+            or block_tables.shape[0] != B or query_start.shape[0] != B + 1:
+        raise ValueError("shape mismatch between out, q, caches, block_tables, query_start and context_lens")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    return (out.data_ptr(), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_tables.data_ptr(),
+            block_tables.shape[1], query_start.data_ptr(), context_lens.data_ptr(), B, int(max_query_len), h_q, h_kv,
+            d, bs, NB, float(scale), cache_dtype_code(k_cache))
+
+
+def pa_prefill(out, q, k_cache, v_cache, block_tables, query_start, context_lens, max_query_len: int,
+               scale: float = None, stream=None) -> torch.Tensor:
+    """Causal attention of each sequence's chunk of query rows over the paged cache; returns out."""
+    args = prefill_call_args(out, q, k_cache, v_cache, block_tables, query_start, context_lens, max_query_len, scale)
+    _check(_lib.pa_prefill(*args, _stream_ptr(stream)), "pa_prefill")
     return out
 
 

@@ -87,6 +87,14 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first()
     return pol;
 }
 
+// L2 policy for tiles that other CTAs will read again soon.
+__device__ __forceinline__ uint64_t l2_policy_evict_last()
+{
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
 // dst and src 16-byte aligned, bytes a multiple of 16; completion counted on `bar`.
 __device__ __forceinline__ void bulk_copy_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar,
                                               uint64_t policy)

@@ -12,6 +12,7 @@
 #include "decode.cuh"
 #include "decode_mma.cuh"
 #include "decode_q8.cuh"
+#include "prefill.cuh"
 #include "decode_balanced.cuh"
 
 using namespace pa;
@@ -563,6 +564,50 @@ int reshape_impl(const void *key, const void *value, int64_t key_stride, int64_t
     return launch_status();
 }
 
+// ---- chunked prefill ------------------------------------------------------------------------
+template <int D, int BS, int G>
+int launch_prefill(const PrefillParams &pp, int num_seqs, int max_query_len, cudaStream_t st)
+{
+    using C = PrefillConfig<D, BS, G>;
+    static std::atomic<unsigned long long> smem_set{0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (!(smem_set.load(std::memory_order_acquire) & bit)) {
+        if (cudaFuncSetAttribute(paged_prefill_kernel<D, BS, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::SMEM) != cudaSuccess)
+            return PA_ERR_CUDA;
+        smem_set.fetch_or(bit, std::memory_order_release);
+    }
+    CUtensorMap mk, mv;
+    int rc = cached_cache_map(&mk, pp.k_cache, pp.num_blocks, pp.h_kv, BS, D);
+    if (rc == PA_OK) rc = cached_cache_map(&mv, pp.v_cache, pp.num_blocks, pp.h_kv, BS, D);
+    if (rc != PA_OK) return rc;
+    const dim3 grid(prefill_tiles<C::TQ>(max_query_len), pp.h_kv, num_seqs);
+    paged_prefill_kernel<D, BS, G><<<grid, C::THREADS, C::SMEM, st>>>(pp, mk, mv);
+    return launch_status();
+}
+
+template <int D, int BS>
+int dispatch_prefill_group(int g, const PrefillParams &pp, int n, int mql, cudaStream_t st)
+{
+    return switch_group(g, [&](auto gc) { return launch_prefill<D, BS, decltype(gc)::value>(pp, n, mql, st); });
+}
+
+int dispatch_prefill(int d, int bs, int g, const PrefillParams &pp, int n, int mql, cudaStream_t st)
+{
+    if (d == 64) {
+        if (bs == 16) return dispatch_prefill_group<64, 16>(g, pp, n, mql, st);
+        if (bs == 32) return dispatch_prefill_group<64, 32>(g, pp, n, mql, st);
+        if (bs == 64) return dispatch_prefill_group<64, 64>(g, pp, n, mql, st);
+    } else if (d == 128) {
+        if (bs == 16) return dispatch_prefill_group<128, 16>(g, pp, n, mql, st);
+        if (bs == 32) return dispatch_prefill_group<128, 32>(g, pp, n, mql, st);
+        if (bs == 64) return dispatch_prefill_group<128, 64>(g, pp, n, mql, st);
+    }
+    return PA_ERR_UNSUPPORTED;
+}
+
 }  // namespace
 
 // Scratch of pa_decode_static_ws: one array per device in global memory (no allocation).
@@ -728,6 +773,39 @@ int pa_reshape_and_cache_head_scales(const void *key, const void *value, int64_t
     if (cache_dtype == PA_CACHE_BF16 || k_scales == nullptr || v_scales == nullptr) return PA_ERR_INVALID_ARG;
     return reshape_impl(key, value, key_stride, value_stride, k_cache, v_cache, slot_mapping, num_tokens, h_kv,
                         head_dim, block_size, num_blocks, cache_dtype, 1.f, 1.f, k_scales, v_scales, stream);
+}
+
+int pa_prefill(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
+               int max_blocks_per_seq, const int32_t *query_start, const int32_t *context_lens, int num_seqs,
+               int max_query_len, int h_q, int h_kv, int head_dim, int block_size, int num_blocks, float scale,
+               int cache_dtype, void *stream)
+{
+    if (num_seqs < 0 || max_query_len < 0 || h_q <= 0 || h_kv <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0)
+        return PA_ERR_INVALID_ARG;
+    if (h_q % h_kv != 0 || !std::isfinite(scale) || !valid_cache_dtype(cache_dtype)) return PA_ERR_INVALID_ARG;
+    if (cache_dtype != PA_CACHE_BF16) return PA_ERR_UNSUPPORTED;
+    if (!supported_head_dim(head_dim) || !supported_block_size(block_size) || !supported_group(h_q / h_kv))
+        return PA_ERR_UNSUPPORTED;
+    if (h_kv > 65535 || num_seqs > 65535) return PA_ERR_UNSUPPORTED;
+    if (num_seqs == 0 || max_query_len == 0) return PA_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !query_start || !context_lens)
+        return PA_ERR_INVALID_ARG;
+    if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return PA_ERR_INVALID_ARG;
+    PrefillParams pp{};
+    pp.out = static_cast<__nv_bfloat16 *>(out);
+    pp.q = static_cast<const __nv_bfloat16 *>(q);
+    pp.k_cache = static_cast<const uint8_t *>(k_cache);
+    pp.v_cache = static_cast<const uint8_t *>(v_cache);
+    pp.block_tables = block_tables;
+    pp.query_start = query_start;
+    pp.context_lens = context_lens;
+    pp.max_blocks_per_seq = max_blocks_per_seq;
+    pp.h_q = h_q;
+    pp.h_kv = h_kv;
+    pp.num_blocks = num_blocks;
+    pp.qk_scale = scale * kLog2e;
+    return dispatch_prefill(head_dim, block_size, h_q / h_kv, pp, num_seqs, max_query_len,
+                            static_cast<cudaStream_t>(stream));
 }
 
 int pa_copy_blocks(void *const *k_caches, void *const *v_caches, int num_layers, const int64_t *block_pairs,

@@ -381,3 +381,91 @@ def make_prefix_prompts(name: str, seed: int = 0, front_changed: bool = False) -
         nq = int(torch.randint(cfg["question"][0], cfg["question"][1] + 1, (1,), generator=g))
         prompts.append(system + doc + torch.randint(0, vocab, (nq,), generator=g).tolist())
     return prompts
+
+
+# ---------------------------------------------------------------------------- prefill chunks
+# Chunked prefill: every sequence already holds `cached` tokens and appends a chunk of new
+# tokens whose query rows attend causally to the whole prefix (the chunk included).
+PREFILL_CONFIGS = {
+    # 8 sequences, each appending a 512-token chunk to a cached prefix of U{0..3584} tokens
+    "prefill_llama3_8b_b8_chunk512": dict(B=8, h_q=32, h_kv=8, d=128, bs=16, cached=(0, 3584), chunk=(512, 512),
+                                          pool_factor=1.1),
+    # whole prompts of U{256..2048} tokens, nothing cached
+    "prefill_llama3_8b_b8_prompt": dict(B=8, h_q=32, h_kv=8, d=128, bs=16, cached=(0, 0), chunk=(256, 2048),
+                                        pool_factor=1.1),
+}
+
+
+@dataclass
+class PrefillCase:
+    name: str
+    B: int
+    h_q: int
+    h_kv: int
+    d: int
+    bs: int
+    num_blocks: int
+    scale: float
+    q: torch.Tensor                 # bf16 [T, h_q, d]: the chunks' query rows, stacked
+    key_new: torch.Tensor           # bf16 [T, h_kv, d]: the chunks' K rows
+    value_new: torch.Tensor
+    slot_mapping: torch.Tensor      # int64 [T]
+    query_start: torch.Tensor       # int32 [B + 1]
+    context_lens: torch.Tensor      # int32 [B], including the chunk
+    block_tables: torch.Tensor      # int32 [B, max_blocks]
+    k_cache: torch.Tensor           # bf16 [NB, h_kv, bs, d] holding the cached prefixes (NaN elsewhere)
+    v_cache: torch.Tensor
+    meta: dict = field(default_factory=dict)
+
+    @property
+    def max_query_len(self) -> int:
+        return int((self.query_start[1:] - self.query_start[:-1]).max().item()) if self.B else 0
+
+    def attention_flops(self) -> int:
+        """4 d (p + 1) per query row and head (Q K^T and P V over the p + 1 visible tokens)."""
+        qs = self.query_start.cpu().tolist()
+        ctx = self.context_lens.cpu().tolist()
+        tot = 0
+        for s in range(self.B):
+            n = qs[s + 1] - qs[s]
+            first = ctx[s] - n + 1                  # tokens seen by the chunk's first row
+            tot += n * first + n * (n - 1) // 2
+        return 4 * self.d * self.h_q * tot
+
+
+def make_prefill_case(name: str, seed: int = 0, device="cpu", **over) -> PrefillCase:
+    cfg = dict(PREFILL_CONFIGS[name])
+    cfg.update(over)
+    device = torch.device(device)
+    gc = _cpu_gen(seed)
+    B, h_q, h_kv, d, bs = cfg["B"], cfg["h_q"], cfg["h_kv"], cfg["d"], cfg["bs"]
+    cached = torch.randint(cfg["cached"][0], cfg["cached"][1] + 1, (B,), generator=gc, dtype=torch.int64)
+    chunk = torch.randint(cfg["chunk"][0], cfg["chunk"][1] + 1, (B,), generator=gc, dtype=torch.int64)
+    ctx = cached + chunk
+    blocks_per_seq = [int(-(-int(c) // bs)) for c in ctx]
+    nb = max(1, int(math.ceil(cfg.get("pool_factor", 1.0) * sum(blocks_per_seq))))
+    order = torch.randperm(nb, generator=gc).tolist()
+    tables = _tables_from_order(order, blocks_per_seq, max(blocks_per_seq) if blocks_per_seq else 1)
+    qs = torch.zeros(B + 1, dtype=torch.int64)
+    qs[1:] = torch.cumsum(chunk, 0)
+    slots = []
+    for s in range(B):
+        for t in range(int(cached[s]), int(ctx[s])):
+            slots.append(int(tables[s, t // bs]) * bs + t % bs)
+    T = int(qs[-1])
+    g = _gen(seed, device)
+    q = _randn_bf16((T, h_q, d), g, device)
+    k_new = _randn_bf16((T, h_kv, d), g, device)
+    v_new = _randn_bf16((T, h_kv, d), g, device)
+    pool_k = _randn_bf16((nb, h_kv, bs, d), g, device)
+    pool_v = _randn_bf16((nb, h_kv, bs, d), g, device)
+    owned = _owned_slot_mask(tables, cached, nb, bs)
+    hole = (~owned).to(device)[:, None, :, None].expand(nb, h_kv, bs, d)
+    nan = torch.tensor(BF16_NAN, dtype=torch.int16).view(torch.bfloat16).to(device)
+    return PrefillCase(name=name, B=B, h_q=h_q, h_kv=h_kv, d=d, bs=bs, num_blocks=nb, scale=1.0 / math.sqrt(d),
+                       q=q, key_new=k_new, value_new=v_new,
+                       slot_mapping=torch.tensor(slots, dtype=torch.int64).to(device),
+                       query_start=qs.to(torch.int32).to(device), context_lens=ctx.to(torch.int32).to(device),
+                       block_tables=tables.to(device), k_cache=torch.where(hole, nan, pool_k),
+                       v_cache=torch.where(hole, nan, pool_v),
+                       meta=dict(seed=seed, cached=cached.tolist(), chunk=chunk.tolist()))
