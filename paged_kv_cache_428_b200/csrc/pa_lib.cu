@@ -13,6 +13,7 @@
 #include "decode_mma.cuh"
 #include "decode_q8.cuh"
 #include "prefill.cuh"
+#include "prefill_tc.cuh"
 #include "decode_balanced.cuh"
 
 using namespace pa;
@@ -588,10 +589,45 @@ int launch_prefill(const PrefillParams &pp, int num_seqs, int max_query_len, cud
     return launch_status();
 }
 
+template <int D, int BS, int G>
+int launch_prefill_tc(const PrefillParams &pp, int num_seqs, int max_query_len, cudaStream_t st)
+{
+    using C = PrefillTcConfig<D, BS, G>;
+    static std::atomic<unsigned long long> smem_set{0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (!(smem_set.load(std::memory_order_acquire) & bit)) {
+        if (cudaFuncSetAttribute(paged_prefill_tc_kernel<D, BS, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::SMEM) != cudaSuccess)
+            return PA_ERR_CUDA;
+        smem_set.fetch_or(bit, std::memory_order_release);
+    }
+    CUtensorMap mk, mv;
+    int rc = cached_cache_map(&mk, pp.k_cache, pp.num_blocks, pp.h_kv, BS, D);
+    if (rc == PA_OK) rc = cached_cache_map(&mv, pp.v_cache, pp.num_blocks, pp.h_kv, BS, D);
+    if (rc != PA_OK) return rc;
+    const int pairs = (prefill_tiles<C::TQ>(max_query_len) + C::NQ - 1) / C::NQ;
+    const dim3 grid(pairs, pp.h_kv, num_seqs);
+    paged_prefill_tc_kernel<D, BS, G><<<grid, C::THREADS, C::SMEM, st>>>(pp, mk, mv);
+    return launch_status();
+}
+
+// The tcgen05 kernel by default; PA_PREFILL_MMA_SYNC=1 selects the mma.sync kernel (A/B runs).
+bool prefill_on_mma_sync()
+{
+    static const bool v = env_flag("PA_PREFILL_MMA_SYNC");
+    return v;
+}
+
 template <int D, int BS>
 int dispatch_prefill_group(int g, const PrefillParams &pp, int n, int mql, cudaStream_t st)
 {
-    return switch_group(g, [&](auto gc) { return launch_prefill<D, BS, decltype(gc)::value>(pp, n, mql, st); });
+    return switch_group(g, [&](auto gc) {
+        constexpr int G = decltype(gc)::value;
+        if (prefill_on_mma_sync()) return launch_prefill<D, BS, G>(pp, n, mql, st);
+        return launch_prefill_tc<D, BS, G>(pp, n, mql, st);
+    });
 }
 
 int dispatch_prefill(int d, int bs, int g, const PrefillParams &pp, int n, int mql, cudaStream_t st)

@@ -1,5 +1,6 @@
 """The CUDA-core decode kernels (selected by PA_DECODE_BF16_CUDA_CORES=1 and
-PA_DECODE_E4M3_CUDA_CORES=1, read once per process) against the oracle: the shape-grid
+PA_DECODE_E4M3_CUDA_CORES=1, read once per process) and the mma.sync prefill kernel
+(PA_PREFILL_MMA_SYNC=1) against the oracle: the shape-grid
 parity tests run again in a child process with both switches set."""
 import os
 import subprocess
@@ -17,5 +18,15 @@ def test_cuda_core_kernels_every_variant():
     r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-m", "gpu", "-p", "no:cacheprovider",
                         str(HERE / "test_gpu_decode.py"), "-k", "every_kernel_variant or fp8_mha_reduced"],
                        env=env, cwd=HERE.parent, capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stdout[-4000:] + r.stderr[-2000:]
+    assert " passed" in r.stdout
+
+
+def test_prefill_mma_sync_kernel():
+    """The mma.sync prefill kernel (PA_PREFILL_MMA_SYNC=1) on the prefill parity tests."""
+    env = dict(os.environ, PA_PREFILL_MMA_SYNC="1")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-m", "gpu", "-p", "no:cacheprovider",
+                        str(HERE / "test_gpu_prefill.py")], env=env, cwd=HERE.parent, capture_output=True, text=True,
+                       timeout=900)
     assert r.returncode == 0, r.stdout[-4000:] + r.stderr[-2000:]
     assert " passed" in r.stdout
