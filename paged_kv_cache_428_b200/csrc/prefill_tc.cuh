@@ -21,7 +21,7 @@
 //              the S products that read it finish, so K runs 4 tiles ahead; V (2 stages) is
 //              needed only after the softmax.
 // Q is copied into a swizzled shared tile once.  S_{j+1} is computed while the softmax works on
-// S_j (two S buffers); P is double-buffered.  V rows past the context are zeroed in shared memory
+// S_j (two S buffers per query tile); P is double-buffered.  V rows past the context are zeroed in shared memory
 // before the P V step (an unwritten NaN slot times a zero probability would poison O).  Every
 // wait is bounded; on a timeout or a bad block the CTA records the error, stops, drains its
 // MMAs and frees its tensor memory; its rows come out NaN.
@@ -231,36 +231,48 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
                 umma_commit(&o_done[2 * q + (i & 1)]);
                 return true;
             };
+            // S_q,j for tile q into S buffer j % 2 (K tile j must have landed); the last tile to
+            // read K tile j releases it
+            auto s_mma = [&](int q, int j) -> bool {
+                const int st = j % KST;
+                if (!mbar_wait_bounded(&k_full[st], (j / KST) & 1) || *abort_flag) return false;
+                if (j >= 2 && (!mbar_wait_bounded(&s_free[2 * q + (j & 1)], ((j - 2) >> 1) & 1) || *abort_flag))
+                    return false;
+                tc_fence_after_sync();
+                const uint32_t kbase = smem_addr(smem + C::OFF_K + st * C::KV_TILE);
+                const uint32_t qbase = smem_addr(smem + C::OFF_Q + q * C::Q_BYTES);
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks)
+                    umma_bf16_ss(tmem + q * C::TMEM_PER_Q + (uint32_t)((j & 1) * 64),
+                                 umma_desc_sw128(qbase + (ks >> 2) * C::Q_HALF + (ks & 3) * 32, 16, 1024),
+                                 umma_desc_sw128(kbase + (ks >> 2) * C::KV_HALF + (ks & 3) * 32, 16, 1024),
+                                 C::IDESC_S, ks > 0);
+                umma_commit(&s_full[2 * q + (j & 1)]);
+                bool last_reader = true;
+#pragma unroll
+                for (int r = q + 1; r < NQ; ++r)
+                    if (j < nkvq[r]) last_reader = false;
+                if (last_reader) umma_commit(&k_empty[st]);
+                return true;
+            };
+            // Schedule: S for the first two KV tiles of every query tile, then per KV tile j and
+            // query tile q: O += P V_j as soon as that tile's softmax has produced P_j, then
+            // S_q,j+2 into the S buffer P_j's softmax has just released.  Each query tile keeps
+            // one S product in flight while its softmax works on the other.
             bool ok = true;
-            for (int j = 0; j <= nkv && ok; ++j) {
-                if (j < nkv) {
-                    const int st = j % KST;
-                    ok = mbar_wait_bounded(&k_full[st], (j / KST) & 1) && !*abort_flag;
-                    const uint32_t kbase = smem_addr(smem + C::OFF_K + st * C::KV_TILE);
+            for (int j = 0; j < 2 && ok; ++j)
 #pragma unroll
-                    for (int q = 0; q < NQ; ++q) {
-                        if (!ok || j >= nkvq[q]) continue;
-                        if (j >= 2) ok = mbar_wait_bounded(&s_free[2 * q + (j & 1)], ((j - 2) >> 1) & 1) && !*abort_flag;
-                        if (!ok) break;
-                        tc_fence_after_sync();
-                        const uint32_t qbase = smem_addr(smem + C::OFF_Q + q * C::Q_BYTES);
+                for (int q = 0; q < NQ; ++q)
+                    if (ok && j < nkvq[q]) ok = s_mma(q, j);
+            for (int j = 0; j < nkv && ok; ++j) {
+                ok = mbar_wait_bounded(&v_full[j % VST], (j / VST) & 1) && !*abort_flag;
 #pragma unroll
-                        for (int ks = 0; ks < D / 16; ++ks)
-                            umma_bf16_ss(tmem + q * C::TMEM_PER_Q + (uint32_t)((j & 1) * 64),
-                                         umma_desc_sw128(qbase + (ks >> 2) * C::Q_HALF + (ks & 3) * 32, 16, 1024),
-                                         umma_desc_sw128(kbase + (ks >> 2) * C::KV_HALF + (ks & 3) * 32, 16, 1024),
-                                         C::IDESC_S, ks > 0);
-                        umma_commit(&s_full[2 * q + (j & 1)]);
-                    }
-                    if (ok) umma_commit(&k_empty[st]);          // K tile j free once these S finish
+                for (int q = 0; q < NQ; ++q) {
+                    if (!ok || j >= nkvq[q]) continue;
+                    ok = pv(q, j);
+                    if (ok && j + 2 < nkvq[q]) ok = s_mma(q, j + 2);
                 }
-                if (ok && j >= 1) {
-                    ok = mbar_wait_bounded(&v_full[(j - 1) % VST], ((j - 1) / VST) & 1) && !*abort_flag;
-#pragma unroll
-                    for (int q = 0; q < NQ; ++q)
-                        if (ok && j - 1 < nkvq[q]) ok = pv(q, j - 1);
-                    if (ok) umma_commit(&v_empty[(j - 1) % VST]);
-                }
+                if (ok) umma_commit(&v_empty[j % VST]);
             }
             if (!ok) {
                 if (!*abort_flag) record_error(PA_DEVERR_TIMEOUT);
@@ -298,19 +310,22 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
             __syncwarp();
             if (lane == 0) mbar_arrive(&my_s_free[j & 1]);
 
+            // raw scores s; the log2-domain logit is s * qk_scale (qk_scale > 0, so the max of
+            // the logits is the scaled max of the scores), p = 2^(s * qk_scale - m) by one FMA
             const int kv0 = j * BN;
-            const bool need_mask = kv0 + BN - 1 > first_pos;
+            if (kv0 + BN - 1 > first_pos) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int c = 0; c < 32; ++c)
+                        if (kv0 + 32 * h + c > pos) sr[h][c] = 0xff800000u;        // -inf
+            }
             float mx = -INFINITY;
 #pragma unroll
             for (int h = 0; h < 2; ++h)
 #pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    float x = __uint_as_float(sr[h][c]) * p.qk_scale;
-                    if (need_mask && kv0 + 32 * h + c > pos) x = -INFINITY;
-                    sr[h][c] = __float_as_uint(x);
-                    mx = fmaxf(mx, x);
-                }
-            const float mn = fmaxf(m_run, mx);
+                for (int c = 0; c < 32; ++c) mx = fmaxf(mx, __uint_as_float(sr[h][c]));
+            const float mn = fmaxf(m_run, mx * p.qk_scale);
             const float alpha = ex2_approx(m_run - mn);
             m_run = mn;
             float rs = 0.f;
@@ -319,8 +334,8 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
             for (int h = 0; h < 2; ++h)
 #pragma unroll
                 for (int c = 0; c < 32; c += 2) {
-                    const float a = ex2_approx(__uint_as_float(sr[h][c]) - mn);
-                    const float b = ex2_approx(__uint_as_float(sr[h][c + 1]) - mn);
+                    const float a = ex2_approx(fmaf(__uint_as_float(sr[h][c]), p.qk_scale, -mn));
+                    const float b = ex2_approx(fmaf(__uint_as_float(sr[h][c + 1]), p.qk_scale, -mn));
                     rs += a + b;
                     pk[16 * h + c / 2] = pack_bf16x2(a, b);
                 }
