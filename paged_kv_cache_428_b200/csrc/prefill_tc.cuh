@@ -325,9 +325,21 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
             for (int h = 0; h < 2; ++h)
 #pragma unroll
                 for (int c = 0; c < 32; ++c) mx = fmaxf(mx, __uint_as_float(sr[h][c]));
-            const float mn = fmaxf(m_run, mx * p.qk_scale);
-            const float alpha = ex2_approx(m_run - mn);
-            m_run = mn;
+            // m_run is the reference the exponentials are taken against.  It moves (and O and
+            // l are rescaled) only when the tile's max exceeds it by more than 8, so p <= 2^8;
+            // O / l does not depend on the reference, and rescaling becomes rare, which keeps
+            // the softmax from waiting for the previous P V.
+            const float m_tile = mx * p.qk_scale;
+            float alpha = 1.f;
+            bool moved = false;
+            if (j == 0) {
+                m_run = m_tile;
+            } else if (m_tile > m_run + 8.f) {
+                alpha = ex2_approx(m_run - m_tile);
+                m_run = m_tile;
+                moved = true;
+            }
+            const float mn = m_run;
             float rs = 0.f;
             uint32_t pk[32];
 #pragma unroll
@@ -341,7 +353,7 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
                 }
             l_run = l_run * alpha + rs;
             // rescale this warp's rows of O when any of their maxima moved (PV_{j-1} must be done)
-            if (j > 0 && __any_sync(FULL, alpha != 1.f)) {
+            if (__any_sync(FULL, moved)) {
                 ok = __all_sync(FULL, mbar_wait_bounded(&my_o_done[(j - 1) & 1], ((j - 1) >> 1) & 1));
                 if (!ok || *abort_flag) {
                     failed = true;
