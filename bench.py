@@ -276,12 +276,20 @@ def run_ours(args):
         part_call = lambda da, s_: L.pa_decode_partitions(*da, s_)
         decode_call = lambda da, s_: L.pa_decode(*da, s_)
 
+    # the step: pa_decode_step (the decode overlaps the cache write) for per-tensor scales, the
+    # separate calls for per-head scales
+    sargs = None if per_head else pa.step_call_args(k_new, v_new, slots, out, q, kc, vc, tables, ctx, mcl, case.scale,
+                                                    P, ks_arg, vs_arg, workspace=ws)
+
     def step(evs=None):
         if evs:
             evs[0].record(stream)
-        rc = write_call(rargs, sp)
-        rc |= part_call(dargs, sp)
-        rc |= L.pa_decode_merge(*margs, sp)
+        if sargs is not None:
+            rc = L.pa_decode_step(*sargs, sp)
+        else:
+            rc = write_call(rargs, sp)
+            rc |= part_call(dargs, sp)
+            rc |= L.pa_decode_merge(*margs, sp)
         if evs:
             evs[1].record(stream)
         if rc:
@@ -363,10 +371,17 @@ def run_ours(args):
         e_dargs = pa.decode_call_args(out, dv["q"], kc, vc, dv["tables"], dv["ctx"], mcl, case.scale, P,
                                       ks_arg, vs_arg, workspace=ws)
 
+        e_sargs = None if per_head else pa.step_call_args(dv["k_new"], dv["v_new"], dv["slots"], out, dv["q"], kc, vc,
+                                                          dv["tables"], dv["ctx"], mcl, case.scale, P, ks_arg, vs_arg,
+                                                          workspace=ws)
+
         def e2e_step():
             dev_buf.copy_(host_buf, non_blocking=True)
-            rc = write_call(e_rargs, sp)
-            rc |= decode_call(e_dargs, sp)
+            if e_sargs is not None:
+                rc = L.pa_decode_step(*e_sargs, sp)
+            else:
+                rc = write_call(e_rargs, sp)
+                rc |= decode_call(e_dargs, sp)
             out_host.copy_(out, non_blocking=True)
             if rc:
                 raise SystemExit("library call failed: %d" % rc)
@@ -436,7 +451,10 @@ def run_ours(args):
         "config": {"workload": args.workload, "num_seqs": B, "h_q": h_q, "h_kv": case.h_kv, "head_dim": d,
                    "block_size": case.bs, "ctx": ctx_desc(case), "partition": P,
                    "num_blocks": case.num_blocks, "kv_bytes_per_step_per_gpu": my_bytes,
-                   "step": "reshape_and_cache(%d new tokens) + split-context decode with in-kernel merge" % B,
+                   "step": ("pa_decode_step: reshape_and_cache(%d new tokens) + split-context decode with in-kernel "
+                            "merge, the decode launched as a programmatic dependent of the write" % B
+                            if not per_head else
+                            "reshape_and_cache(%d new tokens) + split-context decode with in-kernel merge" % B),
                    "scales": ("per KV head" if case.per_head_scales else "per tensor") if case.quantised else None,
                    "l2": ("warm: no flush between steps" if args.warm_l2 else
                           "flushed between steps (2x L2 write, outside the events)"),

@@ -207,6 +207,25 @@ int pa_decode_head_scales(void *out, const void *q, const void *k_cache, const v
                           const float *v_scales, int partition_size, void *workspace, size_t workspace_bytes,
                           void *stream);
 
+/* ---- one decode step: append, then attend --------------------------------------------
+ * pa_reshape_and_cache of one appended token per sequence followed by pa_decode, as one call:
+ *   key, value     device bf16 rows of the appended tokens, row s = sequence s (strides as in
+ *                  pa_reshape_and_cache; num_tokens = num_seqs)
+ *   slot_mapping   device int64 [num_seqs]: the slot of sequence s's appended token, which
+ *                  must be its position context_lens[s] - 1 (so it lies in the sequence's last
+ *                  block); negative = nothing appended for that sequence
+ *   everything else as pa_decode (per-tensor scales).
+ * The decode grid is launched as a programmatic dependent of the cache write: it starts while
+ * the write runs, and only the loads of each sequence's last block wait for the write to
+ * finish, so the write's latency is hidden behind the decode.  Results are identical to the two
+ * calls made separately.  All argument checks happen before anything is launched. */
+int pa_decode_step(const void *key, const void *value, int64_t key_stride, int64_t value_stride,
+                   const int64_t *slot_mapping, void *out, const void *q, void *k_cache, void *v_cache,
+                   const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens, int num_seqs,
+                   int max_context_len, int h_q, int h_kv, int head_dim, int block_size, int num_blocks, float scale,
+                   int cache_dtype, float k_scale, float v_scale, int partition_size, void *workspace,
+                   size_t workspace_bytes, void *stream);
+
 /* ---- chunked-prefill attention ---------------------------------------------------
  * Causal attention of a chunk of new query rows per sequence over the paged cache
  * ("vLLM 推理原理…" section 一次生成有两个阶段: prefill processes the input tokens and builds

@@ -31,6 +31,7 @@ LIB_PATH = _PKG / "libpa.so"
 PA_CACHE_BF16 = 0
 PA_CACHE_E4M3 = 1
 PA_CACHE_INT8 = 2
+PA_PARTITION_AUTO = -1
 PA_DEVERR_BAD_SLOT = 0x1
 PA_DEVERR_BAD_BLOCK = 0x2
 PA_DEVERR_BAD_PAIR = 0x4
@@ -76,6 +77,8 @@ def _load() -> ctypes.CDLL:
         "pa_decode_static_ws": (i32, [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32, i32, i32, f32, i32,
                                       f32, f32, i32, vp]),
         "pa_copy_blocks": (i32, [vp, vp, i32, vp, i32, sz, i32, vp]),
+        "pa_decode_step": (i32, [vp, vp, i64, i64, vp, vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32, i32, i32,
+                                 f32, i32, f32, f32, i32, vp, sz, vp]),
         "pa_prefill": (i32, [vp, vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, i32, i32, i32, f32, i32, vp]),
         "pa_device_errors": (i32, [ctypes.POINTER(ctypes.c_uint), i32]),
         "pa_validate_block_tables": (i32, [vp, i32, vp, i32, i32, i32]),
@@ -316,6 +319,33 @@ def pa_decode_merge(out, context_lens, max_context_len: int, partition_size: int
     ws_ptr, ws_bytes = (workspace.data_ptr(), workspace.numel()) if workspace is not None else (0, 0)
     _check(_lib.pa_decode_merge(out.data_ptr(), context_lens.data_ptr(), B, int(max_context_len), h_q, d,
                                 int(partition_size), ws_ptr, ws_bytes, _stream_ptr(stream)), "pa_decode_merge")
+
+
+def step_call_args(key, value, slot_mapping, out, q, k_cache, v_cache, block_tables, context_lens,
+                   max_context_len: int, scale: float = None, partition_size: int = 512, k_scale: float = 1.0,
+                   v_scale: float = 1.0, workspace: Optional[torch.Tensor] = None) -> tuple:
+    """Checked raw arguments of pa_decode_step (all but the stream)."""
+    r = reshape_call_args(key, value, k_cache, v_cache, slot_mapping, k_scale, v_scale)
+    d = _decode_args(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len, scale, partition_size,
+                     k_scale, v_scale, workspace)
+    if key.shape[0] != q.shape[0]:
+        raise ValueError("pa_decode_step appends one token per sequence: key has %d rows for %d sequences"
+                         % (key.shape[0], q.shape[0]))
+    # key, value, key_stride, value_stride, slot_mapping, then pa_decode's arguments
+    return (r[0], r[1], r[2], r[3], r[6]) + d[:2] + (k_cache.data_ptr(), v_cache.data_ptr()) + d[4:]
+
+
+def pa_decode_step(key, value, slot_mapping, out, q, k_cache, v_cache, block_tables, context_lens,
+                   max_context_len: int, scale: float = None, partition_size: int = 512, k_scale: float = 1.0,
+                   v_scale: float = 1.0, workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """One decode step: write each sequence's appended token (row s of key/value, slot_mapping[s]),
+    then attend; the decode overlaps the write (programmatic dependent launch).  Returns out."""
+    if workspace is None:
+        workspace = make_workspace(q.shape[0], q.shape[1], q.shape[2], max_context_len, partition_size, q.device)
+    args = step_call_args(key, value, slot_mapping, out, q, k_cache, v_cache, block_tables, context_lens,
+                          max_context_len, scale, partition_size, k_scale, v_scale, workspace)
+    _check(_lib.pa_decode_step(*args, _stream_ptr(stream)), "pa_decode_step")
+    return out
 
 
 PA_STATIC_WS_BYTES = 16 * 1024 * 1024

@@ -40,6 +40,7 @@ __device__ __forceinline__ float head_scale(const float *per_head, float per_ten
 template <int D>
 __global__ void __launch_bounds__(256) reshape_and_cache_bf16_kernel(CacheWriteParams p)
 {
+    pdl_launch_dependents();                           // a decode launched after this may start
     constexpr int CHUNKS = D * 2 / 16;                 // 16-byte chunks per row
     const long long tid = blockIdx.x * (long long)blockDim.x + threadIdx.x;
     const long long per_token = (long long)p.h_kv * 2 * CHUNKS;
@@ -74,6 +75,7 @@ __global__ void __launch_bounds__(256) reshape_and_cache_bf16_kernel(CacheWriteP
 template <int D, int QT>
 __global__ void __launch_bounds__(256) reshape_and_cache_quant_kernel(CacheWriteParams p)
 {
+    pdl_launch_dependents();                           // a decode launched after this may start
     constexpr int CHUNKS = D / 8;
     const long long tid = blockIdx.x * (long long)blockDim.x + threadIdx.x;
     const long long per_token = (long long)p.h_kv * 2 * CHUNKS;

@@ -87,6 +87,13 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first()
     return pol;
 }
 
+// Programmatic dependent launch.  launch_dependents lets the next grid on the stream (launched
+// with programmatic stream serialization) start before this one ends; pdl_wait blocks the
+// calling thread until the grid before this one has completed and its writes are visible (a
+// no-op when this grid was launched normally).
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // L2 policy for tiles that other CTAs will read again soon.
 __device__ __forceinline__ uint64_t l2_policy_evict_last()
 {

@@ -56,6 +56,8 @@ struct DecodeParams {
     float v_scale;                 // per-tensor V scale (1 for bf16)
     const float *k_scales;         // per-KV-head scales [h_kv] of a quantised cache, or null
     const float *v_scales;         //   (then qk_scale holds no K scale and v_scale is unused)
+    int pdl_wait_last;             // launched right after the cache write of each sequence's
+                                   // appended token: wait for it before loading a sequence's last block
 };
 
 // Factors of KV head kvh: the K scale folded into the logit scale and the V scale.
@@ -334,6 +336,7 @@ __global__ void __launch_bounds__(DecodeConfig<D, BS, G, FP8>::THREADS)
     const int tok_end = (part == n_part - 1) ? ctx : tok_begin + p.partition_size;
     const int nblk = tok_end > tok_begin ? ceil_div(tok_end - tok_begin, BS) : 0;
     const int blk0 = tok_begin / BS;
+    const int last_blk = ctx > 0 ? (ctx - 1) / BS : -1;    // holds the appended token
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
@@ -391,6 +394,7 @@ __global__ void __launch_bounds__(DecodeConfig<D, BS, G, FP8>::THREADS)
                     if (ii >= STAGES) ok = mbar_wait_bounded(&empty_bar[st], ((ii / STAGES) - 1) & 1);
                     if (ok && *abort_flag) ok = false;
                     if (ok) {
+                        if (p.pdl_wait_last && blk0 + ii == last_blk) pdl_wait();
                         if (ph >= 0) {
                             stage_bad[st] = 0;
                             mbar_arrive_expect_tx(&full_bar[st], 2 * S::TILE);

@@ -45,6 +45,7 @@ struct BalancedParams {
     int num_blocks;
     int num_ctas;                  // C: gridDim.x
     float qk_scale;                // scale * log2(e)
+    int pdl_wait;                  // launched right after the cache write: wait for it before loading
 };
 
 // NW_ consumer warps, RING_ bytes of stage ring, MINB_ = CTAs per SM the register budget
@@ -204,6 +205,7 @@ __global__ void __launch_bounds__(BalancedConfig<D, BS, G, NW_, RING_, MINB_>::T
         if (lane == 0) {
             prefetch_tensormap(&tmap_k);
             prefetch_tensormap(&tmap_v);
+            if (p.pdl_wait) pdl_wait();
         }
         const uint64_t pol = l2_policy_evict_first();
         int issued = 0;

@@ -257,6 +257,7 @@ __global__ void __maxnreg__(96)
     const int tok_end = (part == n_part - 1) ? ctx : tok_begin + p.partition_size;
     const int nblk = tok_end > tok_begin ? ceil_div(tok_end - tok_begin, BS) : 0;
     const int blk0 = tok_begin / BS;
+    const int last_blk = ctx > 0 ? (ctx - 1) / BS : -1;    // holds the appended token
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
@@ -305,6 +306,7 @@ __global__ void __maxnreg__(96)
                     if (ii >= STAGES) ok = mbar_wait_bounded(&empty_bar[st], ((ii / STAGES) - 1) & 1);
                     if (ok && *abort_flag) ok = false;
                     if (ok) {
+                        if (p.pdl_wait_last && blk0 + ii == last_blk) pdl_wait();
                         if (ph >= 0) {
                             stage_bad[st] = 0;
                             mbar_arrive_expect_tx(&full_bar[st], C::STAGE_BYTES);

@@ -6,6 +6,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <type_traits>
+#include <utility>
 
 #include "common.cuh"
 #include "cache_ops.cuh"
@@ -27,6 +28,25 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 int launch_status()
 {
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+// Launch `kernel`; with `pdl`, as a programmatic dependent of the grid before it on the stream
+// (it may start while that grid runs; the kernel waits for it where it reads its results).
+template <typename... KArgs, typename... Args>
+int launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl,
+              Args &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = pdl ? attr : nullptr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 bool supported_head_dim(int d) { return d == 64 || d == 128; }
@@ -87,8 +107,8 @@ int launch_partition(const DecodeParams &prm, int num_seqs, cudaStream_t st)
         smem_set.fetch_or(bit, std::memory_order_release);
     }
     const dim3 grid(prm.p_max, prm.h_kv, num_seqs);
-    paged_decode_partition_kernel<D, BS, G, FP8><<<grid, C::THREADS, C::SMEM, st>>>(prm);
-    return launch_status();
+    return launch_ex(paged_decode_partition_kernel<D, BS, G, FP8>, grid, dim3(C::THREADS), C::SMEM, st,
+                     prm.pdl_wait_last != 0, prm);
 }
 
 // ---- tensor maps of the bf16 caches (2-D: rows of head_dim elements, 128B swizzle) -----
@@ -188,8 +208,8 @@ int launch_partition_mma(const DecodeParams &prm, int num_seqs, cudaStream_t st)
     if (rc == PA_OK) rc = cached_cache_map(&mv, prm.v_cache, prm.num_blocks, prm.h_kv, BS, D);
     if (rc != PA_OK) return rc;
     const dim3 grid(prm.p_max, prm.h_kv, num_seqs);
-    paged_decode_partition_mma_kernel<D, BS, G><<<grid, C::THREADS, C::SMEM, st>>>(prm, mk, mv);
-    return launch_status();
+    return launch_ex(paged_decode_partition_mma_kernel<D, BS, G>, grid, dim3(C::THREADS), C::SMEM, st,
+                     prm.pdl_wait_last != 0, prm, mk, mv);
 }
 
 // Consumer warps and ring bytes of the one-byte-code kernel: 2 warps and a 32 KB ring (6 CTAs
@@ -220,8 +240,8 @@ int launch_partition_q8(const DecodeParams &prm, int num_seqs, cudaStream_t st)
     if (rc == PA_OK) rc = cached_cache_map(&mv, prm.v_cache, prm.num_blocks, prm.h_kv, BS, D, 1);
     if (rc != PA_OK) return rc;
     const dim3 grid(prm.p_max, prm.h_kv, num_seqs);
-    paged_decode_partition_q8_kernel<D, BS, G, QT, NW, RING><<<grid, C::THREADS, C::SMEM, st>>>(prm, mk, mv);
-    return launch_status();
+    return launch_ex(paged_decode_partition_q8_kernel<D, BS, G, QT, NW, RING>, grid, dim3(C::THREADS), C::SMEM, st,
+                     prm.pdl_wait_last != 0, prm, mk, mv);
 }
 
 bool env_flag(const char *name)
@@ -400,8 +420,9 @@ int launch_balanced(const DecodeParams &prm, int num_seqs, const BalLayout &lay,
     bp.num_blocks = prm.num_blocks;
     bp.num_ctas = ctas;
     bp.qk_scale = prm.qk_scale;
-    paged_decode_balanced_kernel<D, BS, G><<<ctas, BC::THREADS, smem, st>>>(bp, mk, mv);
-    return launch_status();
+    bp.pdl_wait = prm.pdl_wait_last;
+    return launch_ex(paged_decode_balanced_kernel<D, BS, G>, dim3(ctas), dim3(BC::THREADS), (size_t)smem, st,
+                     prm.pdl_wait_last != 0, bp, mk, mv);
 }
 
 template <int D, int BS>
@@ -499,7 +520,7 @@ int decode_partitions_impl(void *out, const void *q, const void *k_cache, const 
                            int num_seqs, int max_context_len, int h_q, int h_kv, int head_dim, int block_size,
                            int num_blocks, float scale, int cache_dtype, float k_scale, float v_scale,
                            const float *k_scales, const float *v_scales, int partition_size, void *workspace,
-                           size_t workspace_bytes, void *stream)
+                           size_t workspace_bytes, void *stream, bool after_append = false)
 {
     DecodeParams prm{};
     int rc = prepare_decode(prm, out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
@@ -507,6 +528,7 @@ int decode_partitions_impl(void *out, const void *q, const void *k_cache, const 
                             cache_dtype, k_scale, v_scale, k_scales, v_scales, partition_size, workspace,
                             workspace_bytes);
     if (rc != PA_OK || num_seqs == 0) return rc;
+    prm.pdl_wait_last = after_append ? 1 : 0;
     if (partition_size == PA_PARTITION_AUTO && balanced_applies(num_seqs, h_q, h_kv, cache_dtype))
         return dispatch_balanced(head_dim, block_size, h_q / h_kv, prm, num_seqs, bal_layout(num_seqs, h_q, head_dim),
                                  workspace, static_cast<cudaStream_t>(stream));
@@ -790,6 +812,33 @@ int pa_decode_head_scales(void *out, const void *q, const void *k_cache, const v
     if (rc != PA_OK) return rc;
     return pa_decode_merge(out, context_lens, num_seqs, max_context_len, h_q, head_dim, partition_size,
                            workspace, workspace_bytes, stream);
+}
+
+int pa_decode_step(const void *key, const void *value, int64_t key_stride, int64_t value_stride,
+                   const int64_t *slot_mapping, void *out, const void *q, void *k_cache, void *v_cache,
+                   const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens, int num_seqs,
+                   int max_context_len, int h_q, int h_kv, int head_dim, int block_size, int num_blocks, float scale,
+                   int cache_dtype, float k_scale, float v_scale, int partition_size, void *workspace,
+                   size_t workspace_bytes, void *stream)
+{
+    if (num_seqs < 0) return PA_ERR_INVALID_ARG;
+    if (num_seqs == 0) return PA_OK;
+    // the decode's argument checks first, so that nothing is launched on a bad call
+    DecodeParams chk{};
+    int rc = prepare_decode(chk, out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                            max_context_len, h_q, h_kv, head_dim, block_size, num_blocks, scale, cache_dtype,
+                            k_scale, v_scale, nullptr, nullptr, partition_size, workspace, workspace_bytes);
+    if (rc != PA_OK) return rc;
+    rc = reshape_impl(key, value, key_stride, value_stride, k_cache, v_cache, slot_mapping, num_seqs, h_kv, head_dim,
+                      block_size, num_blocks, cache_dtype, k_scale, v_scale, nullptr, nullptr, stream);
+    if (rc != PA_OK) return rc;
+    rc = decode_partitions_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                                max_context_len, h_q, h_kv, head_dim, block_size, num_blocks, scale, cache_dtype,
+                                k_scale, v_scale, nullptr, nullptr, partition_size, workspace, workspace_bytes, stream,
+                                true);
+    if (rc != PA_OK) return rc;
+    return pa_decode_merge(out, context_lens, num_seqs, max_context_len, h_q, head_dim, partition_size, workspace,
+                           workspace_bytes, stream);
 }
 
 int pa_reshape_and_cache(const void *key, const void *value, int64_t key_stride, int64_t value_stride,
