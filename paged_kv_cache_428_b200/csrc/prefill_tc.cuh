@@ -3,27 +3,30 @@
 //
 // Same computation and masking rules as paged_prefill_kernel (prefill.cuh).  One CTA per (pair
 // of query tiles, KV head, sequence); a query tile is 128 rows = 128 / G tokens x the G heads of
-// the KV head, and both tiles of a CTA share every K/V tile it streams.  Roles:
+// the KV head, and both tiles of a CTA share every K/V tile it streams.  Tensor memory per query
+// tile (256 of the 512 columns): S [0,64) fp32, P0 / P1 [64,128) bf16 pairs, O [128,128+D) fp32.
+// Roles:
 //   warps 0-7  two softmax warpgroups, one per query tile: thread t of a warpgroup owns row t of
-//              its tile (= tensor-memory lane t of the tile's columns).  It reads its row of S
-//              from tensor memory, applies the causal / context mask, keeps the running max
-//              and sum (log2 domain), writes its row of P (bf16) into a 128-byte-swizzled
-//              shared tile, rescales its row of O in tensor memory when its max moved, and
-//              finally normalises O and writes the output row.
-//   warp 8     tensor-memory allocation (all 512 columns: per tile two 64-column S buffers and
-//              the O accumulator); lane 0 issues every tcgen05.mma: S = Q K_j^T (M 128, N 64,
-//              K = D) for both tiles, then O += P V_{j-1} (M 128, N D, K 64) for both, with P
-//              from shared memory and V read N-major, so one tile's S runs on the tensor core
-//              while the other tile's softmax works; tcgen05.commit signals each step.
-//   warp 9     lane 0 streams the 64-token K tiles, lane 1 the V tiles, per physical block with
-//              2-D TMA (the decode tensor maps, 128-byte swizzle), so the tiles are the MMA
-//              operands as they land.  K and V have separate rings: a K tile is free as soon as
-//              the S products that read it finish, so K runs 4 tiles ahead; V (2 stages) is
-//              needed only after the softmax.
-// Q is copied into a swizzled shared tile once.  S_{j+1} is computed while the softmax works on
-// S_j (two S buffers per query tile); P is double-buffered.  V rows past the context are zeroed in shared memory
-// before the P V step (an unwritten NaN slot times a zero probability would poison O).  Every
-// wait is bounded; on a timeout or a bad block the CTA records the error, stops, drains its
+//              its tile (= tensor-memory lane t).  It loads its row of S_j from tensor memory
+//              (which frees S for S_{j+1}), applies the causal / context mask, keeps the running
+//              max and sum (log2 domain), stores its row of P_j (bf16) into tensor memory,
+//              rescales its row of O when its max moved, and finally normalises O and writes the
+//              output row.
+//   warps 8-9  one MMA warp per query tile: lane 0 issues S_{j+1} = Q K_{j+1}^T (M 128, N 64,
+//              K = D, both operands in shared memory) as soon as the softmax has loaded S_j, and
+//              O += P_j V_j (M 128, N = D, K 64) with P read from tensor memory and V read N-major
+//              from shared memory; tcgen05.commit signals each step.  With one issuing thread per
+//              tile, one tile's barrier waits overlap the other tile's MMAs on the tensor core.
+//              Warp 8 also allocates the 512 tensor-memory columns.
+//   warps 10-11 K and V producers: 2-D TMA copies per physical block (the decode tensor maps,
+//              128-byte swizzle), so the tiles are the MMA operands as they land.  Each warp
+//              reads the block table 32 entries at a time, the next 32 in flight meanwhile, and
+//              its lanes issue the copies of one tile.  K and V have rings of their own; a slot
+//              is free when both query tiles have released it (their MMAs that read it finished,
+//              or the tile's KV range ended before it).
+// Q is copied into a swizzled shared tile once.  V rows past the context are zeroed in shared
+// memory before the P V step (an unwritten NaN slot times a zero probability would poison O).
+// Every wait is bounded; on a timeout or a bad block the CTA records the error, stops, drains its
 // MMAs and frees its tensor memory; its rows come out NaN.
 #pragma once
 
@@ -40,11 +43,11 @@ __device__ __forceinline__ float ex2_approx(float x)
     return y;
 }
 
-template <int D, int BS, int G, int NQ_ = 2, int KST_ = 4, int VST_ = 2>
+template <int D, int BS, int G, int NQ_ = 2, int KST_ = 4, int VST_ = 4>
 struct PrefillTcConfig {
     static constexpr int NQ = NQ_;                        // 128-row query tiles per CTA
-    static constexpr int THREADS = 128 * NQ + 64;         // softmax warpgroups, MMA warp, TMA warp
-    static constexpr int MMA_WARP = 4 * NQ, TMA_WARP = 4 * NQ + 1;
+    static constexpr int THREADS = 128 * NQ + 32 * NQ + 64; // softmax warpgroups, one MMA warp per query tile, K and V TMA warps
+    static constexpr int MMA_WARP = 4 * NQ, TMA_WARP = 5 * NQ;
     static constexpr int BM = 128;                        // rows per query tile = tensor-memory lanes
     static constexpr int TQ = BM / G;                     // query tokens per query tile
     static constexpr int BN = 64;                         // KV tokens per tile
@@ -56,16 +59,15 @@ struct PrefillTcConfig {
     static constexpr int BLOCKS_PER_TILE = BN / BS;
     static constexpr int Q_HALF = BM * 128;               // [128 rows][64 elements]
     static constexpr int Q_BYTES = HALVES * Q_HALF;
-    static constexpr int P_BYTES = BM * 128;              // [128 rows][64 tokens] bf16
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = NQ * Q_BYTES;
     static constexpr int OFF_V = OFF_K + KST * KV_TILE;
-    static constexpr int OFF_P = OFF_V + VST * KV_TILE;
-    static constexpr int OFF_BARS = OFF_P + NQ * 2 * P_BYTES;
-    static constexpr int NBARS = 2 * KST + 2 * VST + NQ * 8 + 1; // k, v full/empty; per tile s full/free, p full, o done; drain
+    static constexpr int OFF_BARS = OFF_V + VST * KV_TILE;
+    static constexpr int NBARS = 2 * KST + 2 * VST + NQ * 7; // k, v full/empty; per tile s full, s free, p full x2, o done x2, drain
     static constexpr int OFF_MISC = OFF_BARS + NBARS * 8; // tensor-memory base, abort flag
     static constexpr int SMEM = OFF_MISC + 16 + 1024;
-    static constexpr int TMEM_PER_Q = 256;                // S0 [0,64), S1 [64,128), O [128, 128 + D)
+    static constexpr int TMEM_PER_Q = 256;                // S [0,64), P0 [64,96), P1 [96,128), O [128, 128 + D)
+    static constexpr int COL_P = 64;
     static constexpr int TMEM_COLS = NQ * TMEM_PER_Q;
     static constexpr int COL_O = 128;
     static constexpr uint32_t IDESC_S = umma_idesc_bf16(BM, BN, false);
@@ -77,7 +79,7 @@ struct PrefillTcConfig {
     static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
-template <int D, int BS, int G, int NQ_ = 2, int KST_ = 4, int VST_ = 2>
+template <int D, int BS, int G, int NQ_ = 2, int KST_ = 4, int VST_ = 4>
 __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::THREADS, 1)
     paged_prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmap_k,
                             const __grid_constant__ CUtensorMap tmap_v)
@@ -91,8 +93,8 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BARS);
     uint64_t *k_full = bars, *k_empty = bars + KST, *v_full = bars + 2 * KST, *v_empty = v_full + VST;
     // per query tile q and buffer b: index 2 q + b
-    uint64_t *s_full = bars + 2 * KST + 2 * VST, *s_free = s_full + 2 * NQ, *p_full = s_free + 2 * NQ, *o_done = p_full + 2 * NQ;
-    uint64_t *drain = o_done + 2 * NQ;
+    uint64_t *s_full = bars + 2 * KST + 2 * VST, *s_free = s_full + NQ, *p_full = s_free + NQ, *o_done = p_full + 2 * NQ;
+    uint64_t *drain = o_done + 2 * NQ;                          // one per query tile
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
 
@@ -124,19 +126,21 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
     if (threadIdx.x == 0) {
         for (int i = 0; i < KST; ++i) {
             mbar_init(&k_full[i], 1);
-            mbar_init(&k_empty[i], 1);
+            mbar_init(&k_empty[i], NQ);
         }
         for (int i = 0; i < VST; ++i) {
             mbar_init(&v_full[i], 1);
-            mbar_init(&v_empty[i], 1);
+            mbar_init(&v_empty[i], NQ);
+        }
+        for (int q = 0; q < NQ; ++q) {
+            mbar_init(&s_full[q], 1);
+            mbar_init(&s_free[q], 4);
         }
         for (int b = 0; b < 2 * NQ; ++b) {
-            mbar_init(&s_full[b], 1);
-            mbar_init(&s_free[b], 4);
             mbar_init(&p_full[b], 4);
             mbar_init(&o_done[b], 1);
         }
-        mbar_init(drain, 1);
+        for (int q = 0; q < NQ; ++q) mbar_init(&drain[q], 1);
         *abort_flag = 0;
         mbar_init_fence();
     }
@@ -163,123 +167,116 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == C::TMA_WARP) {
+    if (warp == C::TMA_WARP || warp == C::TMA_WARP + 1) {
         // ------------------------------ TMA producers ------------------------------
-        // lane 0 streams the K tiles (ring of KST, freed once S is computed), lane 1 the V tiles
-        // (ring of VST, freed after P V); each checks the block-table entries of its tiles.
-        if (lane < 2) {
-            const bool is_v = lane == 1;
-            const int nst = is_v ? VST : KST;
-            uint64_t *full = is_v ? v_full : k_full;
-            uint64_t *empty = is_v ? v_empty : k_empty;
-            const CUtensorMap *map = is_v ? &tmap_v : &tmap_k;
-            prefetch_tensormap(map);
-            const uint64_t pol = l2_policy_evict_last();
-            const int32_t *trow = p.block_tables + (size_t)seq * p.max_blocks_per_seq;
-            for (int it = 0; it < nkv; ++it) {
-                const int st = it % nst;
+        // one warp per operand: the warp reads the block table 32 entries at a time (the next
+        // 32 are in flight meanwhile), lane 0 waits for the ring slot, and lane l issues the copy
+        // of block l / HALVES, half l % HALVES of the tile
+        const bool is_v = warp != C::TMA_WARP;
+        const int nst = is_v ? VST : KST;
+        uint64_t *full = is_v ? v_full : k_full;
+        uint64_t *empty = is_v ? v_empty : k_empty;
+        const CUtensorMap *map = is_v ? &tmap_v : &tmap_k;
+        if (lane == 0) prefetch_tensormap(map);
+        const uint64_t pol = l2_policy_evict_last();
+        const int32_t *trow = p.block_tables + (size_t)seq * p.max_blocks_per_seq;
+        constexpr int BPT = C::BLOCKS_PER_TILE, TPB = 32 / BPT;
+        auto entry = [&](int lb) -> int {
+            return (lb < nblk_seq && lb < p.max_blocks_per_seq) ? __ldg(trow + lb) : -1;
+        };
+        int cur = entry(lane), nxt = entry(32 + lane);
+        const int k = lane / C::HALVES, hf = lane % C::HALVES;
+        for (int it = 0; it < nkv; ++it) {
+            if (it > 0 && it % TPB == 0) {
+                cur = nxt;
+                nxt = entry((it / TPB + 1) * 32 + lane);
+            }
+            const int st = it % nst;
+            int go = 1;
+            if (lane == 0) {
                 if (it >= nst && !mbar_wait_bounded(&empty[st], ((it / nst) - 1) & 1)) {
                     if (!*abort_flag) record_error(PA_DEVERR_TIMEOUT);
                     *abort_flag = 1;
-                    break;
                 }
-                if (*abort_flag) break;
-                const int b0 = it * C::BLOCKS_PER_TILE;
-                const int nb = min(C::BLOCKS_PER_TILE, nblk_seq - b0);
-                int phys[C::BLOCKS_PER_TILE];
-                bool bad = false;
-#pragma unroll
-                for (int k = 0; k < C::BLOCKS_PER_TILE; ++k) {
-                    phys[k] = -1;
-                    if (k < nb) {
-                        const int lb = b0 + k;
-                        phys[k] = lb < p.max_blocks_per_seq ? trow[lb] : -1;
-                        if (phys[k] < 0 || phys[k] >= p.num_blocks) bad = true;
-                    }
-                }
-                if (bad) {
+                go = *abort_flag ? 0 : 1;
+            }
+            if (!__shfl_sync(FULL, go, 0)) break;
+            const int nb = min(BPT, nblk_seq - it * BPT);
+            const int phys = __shfl_sync(FULL, cur, (it % TPB) * BPT + min(k, BPT - 1));
+            const bool mine = lane < nb * C::HALVES;
+            if (__any_sync(FULL, mine && (phys < 0 || phys >= p.num_blocks))) {
+                if (lane == 0) {
                     record_error(PA_DEVERR_BAD_BLOCK);
                     *abort_flag = 1;
                     mbar_arrive(&full[st]);                    // wake the MMA thread
-                    break;
                 }
-                mbar_arrive_expect_tx(&full[st], (uint32_t)(nb * C::HALVES * BS * 128));
-                uint8_t *dst = smem + (is_v ? C::OFF_V : C::OFF_K) + st * C::KV_TILE;
-                for (int k = 0; k < nb; ++k) {
-                    const int row = (phys[k] * p.h_kv + kvh) * BS;
-#pragma unroll
-                    for (int hf = 0; hf < C::HALVES; ++hf)
-                        tma_load_2d(dst + hf * C::KV_HALF + k * BS * 128, map, hf * 64, row, &full[st], pol);
-                }
+                break;
             }
+            if (lane == 0) mbar_arrive_expect_tx(&full[st], (uint32_t)(nb * C::HALVES * BS * 128));
+            __syncwarp();
+            if (mine)
+                tma_load_2d(smem + (is_v ? C::OFF_V : C::OFF_K) + st * C::KV_TILE + hf * C::KV_HALF + k * BS * 128, map,
+                            hf * 64, (phys * p.h_kv + kvh) * BS, &full[st], pol);
         }
-    } else if (warp == C::MMA_WARP) {
-        // ------------------------------ MMA issue ------------------------------
+    } else if (warp >= C::MMA_WARP && warp < C::MMA_WARP + NQ) {
+        // ------------------------------ MMA issue, one warp per query tile ------------------------------
+        // Lane 0 issues S_j = Q K_j^T and O += P_j V_j for its tile.  Every query tile releases
+        // every K and V slot once per KV tile: a tile that reads the slot commits after its MMAs,
+        // a tile whose range ended arrives as soon as the slot's data has landed (so the
+        // arrival falls into that tile's phase of the empty barrier).
+        const int q = warp - C::MMA_WARP;
         if (lane == 0) {
-            int nkvq[NQ];
-#pragma unroll
-            for (int q = 0; q < NQ; ++q) nkvq[q] = nkv_of(q);
-            auto pv = [&](int q, int i) -> bool {
-                if (!mbar_wait_bounded(&p_full[2 * q + (i & 1)], (i >> 1) & 1) || *abort_flag) return false;
-                tc_fence_after_sync();
-                const uint32_t vbase = smem_addr(smem + C::OFF_V + (i % VST) * C::KV_TILE);
-                const uint32_t pbase = smem_addr(smem + C::OFF_P + (2 * q + (i & 1)) * C::P_BYTES);
-#pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk)
-                    umma_bf16_ss(tmem + q * C::TMEM_PER_Q + C::COL_O, umma_desc_sw128(pbase + kk * 32, 16, 1024),
-                                 umma_desc_sw128(vbase + kk * 2048, C::KV_HALF, 1024), C::IDESC_O, i > 0 || kk > 0);
-                umma_commit(&o_done[2 * q + (i & 1)]);
-                return true;
-            };
-            // S_q,j for tile q into S buffer j % 2 (K tile j must have landed); the last tile to
-            // read K tile j releases it
-            auto s_mma = [&](int q, int j) -> bool {
+            const int nkq = nkv_of(q);
+            const uint32_t d_s = tmem + q * C::TMEM_PER_Q, d_o = d_s + C::COL_O, d_p = d_s + C::COL_P;
+            const uint64_t qdesc = umma_desc_sw128(smem_addr(smem + C::OFF_Q + q * C::Q_BYTES), 16, 1024);
+            const uint64_t kdesc = umma_desc_sw128(smem_addr(smem + C::OFF_K), 16, 1024);
+            const uint64_t vdesc = umma_desc_sw128(smem_addr(smem + C::OFF_V), C::KV_HALF, 1024);
+            auto s_mma = [&](int j) -> bool {
                 const int st = j % KST;
                 if (!mbar_wait_bounded(&k_full[st], (j / KST) & 1) || *abort_flag) return false;
-                if (j >= 2 && (!mbar_wait_bounded(&s_free[2 * q + (j & 1)], ((j - 2) >> 1) & 1) || *abort_flag))
-                    return false;
+                if (j >= 1 && (!mbar_wait_bounded(&s_free[q], (j - 1) & 1) || *abort_flag)) return false;
                 tc_fence_after_sync();
-                const uint32_t kbase = smem_addr(smem + C::OFF_K + st * C::KV_TILE);
-                const uint32_t qbase = smem_addr(smem + C::OFF_Q + q * C::Q_BYTES);
+                const uint64_t kd = kdesc + (uint64_t)((st * C::KV_TILE) >> 4);
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks)
-                    umma_bf16_ss(tmem + q * C::TMEM_PER_Q + (uint32_t)((j & 1) * 64),
-                                 umma_desc_sw128(qbase + (ks >> 2) * C::Q_HALF + (ks & 3) * 32, 16, 1024),
-                                 umma_desc_sw128(kbase + (ks >> 2) * C::KV_HALF + (ks & 3) * 32, 16, 1024),
-                                 C::IDESC_S, ks > 0);
-                umma_commit(&s_full[2 * q + (j & 1)]);
-                bool last_reader = true;
-#pragma unroll
-                for (int r = q + 1; r < NQ; ++r)
-                    if (j < nkvq[r]) last_reader = false;
-                if (last_reader) umma_commit(&k_empty[st]);
+                    umma_bf16_ss(d_s, qdesc + (uint64_t)(((ks >> 2) * C::Q_HALF + (ks & 3) * 32) >> 4),
+                                 kd + (uint64_t)(((ks >> 2) * C::KV_HALF + (ks & 3) * 32) >> 4), C::IDESC_S, ks > 0);
+                umma_commit(&s_full[q]);
+                umma_commit(&k_empty[st]);
                 return true;
             };
-            // Schedule: S for the first two KV tiles of every query tile, then per KV tile j and
-            // query tile q: O += P V_j as soon as that tile's softmax has produced P_j, then
-            // S_q,j+2 into the S buffer P_j's softmax has just released.  Each query tile keeps
-            // one S product in flight while its softmax works on the other.
+            auto pv = [&](int i) -> bool {
+                if (!mbar_wait_bounded(&v_full[i % VST], (i / VST) & 1) || *abort_flag) return false;
+                if (!mbar_wait_bounded(&p_full[2 * q + (i & 1)], (i >> 1) & 1) || *abort_flag) return false;
+                tc_fence_after_sync();
+                const uint64_t vd = vdesc + (uint64_t)(((i % VST) * C::KV_TILE) >> 4);
+                const uint32_t pt = d_p + 32 * (i & 1);
+#pragma unroll
+                for (int kk = 0; kk < BN / 16; ++kk)
+                    umma_bf16_ts(d_o, pt + 8 * kk, vd + (uint64_t)((kk * 2048) >> 4), C::IDESC_O, i > 0 || kk > 0);
+                umma_commit(&o_done[2 * q + (i & 1)]);
+                umma_commit(&v_empty[i % VST]);
+                return true;
+            };
             bool ok = true;
-            for (int j = 0; j < 2 && ok; ++j)
-#pragma unroll
-                for (int q = 0; q < NQ; ++q)
-                    if (ok && j < nkvq[q]) ok = s_mma(q, j);
-            for (int j = 0; j < nkv && ok; ++j) {
-                ok = mbar_wait_bounded(&v_full[j % VST], (j / VST) & 1) && !*abort_flag;
-#pragma unroll
-                for (int q = 0; q < NQ; ++q) {
-                    if (!ok || j >= nkvq[q]) continue;
-                    ok = pv(q, j);
-                    if (ok && j + 2 < nkvq[q]) ok = s_mma(q, j + 2);
-                }
-                if (ok) umma_commit(&v_empty[j % VST]);
+            if (nkq > 0) ok = s_mma(0);
+            for (int j = 0; j < nkq && ok; ++j) {
+                if (j + 1 < nkq) ok = s_mma(j + 1);
+                if (ok) ok = pv(j);
+            }
+            // the KV tiles past this query tile's range: release their slots as they land
+            for (int j = nkq; j < nkv && ok; ++j) {
+                ok = mbar_wait_bounded(&k_full[j % KST], (j / KST) & 1) && !*abort_flag;
+                if (ok) mbar_arrive(&k_empty[j % KST]);
+                ok = ok && mbar_wait_bounded(&v_full[j % VST], (j / VST) & 1) && !*abort_flag;
+                if (ok) mbar_arrive(&v_empty[j % VST]);
             }
             if (!ok) {
                 if (!*abort_flag) record_error(PA_DEVERR_TIMEOUT);
                 *abort_flag = 1;
             }
-            umma_commit(drain);                                 // every MMA issued so far has finished
-            mbar_wait_bounded(drain, 0);
+            umma_commit(&drain[q]);                             // every MMA this thread issued has finished
+            mbar_wait_bounded(&drain[q], 0);
         }
         __syncwarp();
     } else {
@@ -291,24 +288,24 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
         const int pos = row_ok ? ctx - chunk + tok : 0;
         const int first_pos = ctx - chunk + tok0;
         const uint32_t lane_tm = tmem + q * C::TMEM_PER_Q + ((uint32_t)(32 * (warp & 3)) << 16);
-        uint64_t *my_s_full = s_full + 2 * q, *my_s_free = s_free + 2 * q;
+        uint64_t *my_s_full = s_full + q, *my_s_free = s_free + q;
         uint64_t *my_p_full = p_full + 2 * q, *my_o_done = o_done + 2 * q;
         float m_run = -INFINITY, l_run = 0.f;
         bool failed = false;
         for (int j = 0; j < nkv_q; ++j) {
-            bool ok = __all_sync(FULL, mbar_wait_bounded(&my_s_full[j & 1], (j >> 1) & 1));
+            bool ok = __all_sync(FULL, mbar_wait_bounded(my_s_full, j & 1));
             if (!ok || *abort_flag) {
                 failed = true;
                 break;
             }
             tc_fence_after_sync();
             uint32_t sr[2][32];
-            tmem_ld32(lane_tm + (uint32_t)((j & 1) * 64), sr[0]);
-            tmem_ld32(lane_tm + (uint32_t)((j & 1) * 64 + 32), sr[1]);
+            tmem_ld32(lane_tm, sr[0]);
+            tmem_ld32(lane_tm + 32u, sr[1]);
             tmem_wait_ld();
             tc_fence_before_sync();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&my_s_free[j & 1]);
+            if (lane == 0) mbar_arrive(my_s_free);
 
             // raw scores s; the log2-domain logit is s * qk_scale (qk_scale > 0, so the max of
             // the logits is the scaled max of the scores), p = 2^(s * qk_scale - m) by one FMA
@@ -386,6 +383,7 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
                     *reinterpret_cast<uint4 *>(vt + hf * C::KV_HALF + (r0 + rem / 8) * 128 + (rem % 8) * 16) =
                         make_uint4(0u, 0u, 0u, 0u);
                 }
+                fence_proxy_async_smem();
             }
             // P buffer j % 2 is free once P V_{j-2} has finished
             if (j >= 2) {
@@ -395,12 +393,8 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
                     break;
                 }
             }
-            uint8_t *prow = smem + C::OFF_P + (2 * q + (j & 1)) * C::P_BYTES;
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-                *reinterpret_cast<uint4 *>(prow + swz128(t, c)) =
-                    make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-            fence_proxy_async_smem();
+            tmem_st32(lane_tm + (uint32_t)(C::COL_P + 32 * (j & 1)), pk);
+            tmem_wait_st();
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(&my_p_full[j & 1]);
