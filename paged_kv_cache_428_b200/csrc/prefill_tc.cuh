@@ -9,7 +9,8 @@
 //   warps 0-7  two softmax warpgroups, one per query tile: thread t of a warpgroup owns row t of
 //              its tile (= tensor-memory lane t).  It loads its row of S_j from tensor memory
 //              (which frees S for S_{j+1}), applies the causal / context mask, keeps the running
-//              max and sum (log2 domain), stores its row of P_j (bf16) into tensor memory,
+//              max and sum (log2 domain; a quarter of the exponentials by a polynomial on
+//              the FMA pipe, beside the MUFU unit), stores its row of P_j (bf16) into tensor memory,
 //              rescales its row of O when its max moved, and finally normalises O and writes the
 //              output row.
 //   warps 8-9  one MMA warp per query tile: lane 0 issues S_{j+1} = Q K_{j+1}^T (M 128, N 64,
@@ -43,6 +44,40 @@ __device__ __forceinline__ float ex2_approx(float x)
     return y;
 }
 
+// Coefficients of the cubic that interpolates 2^f at the four Chebyshev nodes of [-1/2, 1/2]
+// (relative error below 1.0e-4 there, i.e. under 2^-13, against the 2^-9 rounding of P to bf16).
+#define PA_EX2_C0 0.999924541f
+#define PA_EX2_C1 0.693136752f
+#define PA_EX2_C2 0.242639482f
+#define PA_EX2_C3 0.0558382832f
+
+// 2^x for a pair, on the FMA pipe instead of the MUFU unit: Cody-Waite style range reduction
+// x = n + f with n = round(x) (adding 1.5 * 2^23 leaves n in the low mantissa bits), f in
+// [-1/2, 1/2]; 2^f by the cubic above; 2^n added to the exponent field.  x is clamped to -125
+// first, so results below 2^-125 come out as about 2^-125 instead of 0 (x <= 8 here).
+__device__ __forceinline__ float2 ex2_poly2(float2 x)
+{
+    constexpr float R = 12582912.f;                       // 1.5 * 2^23
+    x.x = fmaxf(x.x, -125.f);
+    x.y = fmaxf(x.y, -125.f);
+    const float2 t = __fadd2_rn(x, make_float2(R, R));
+    const float2 n = __fadd2_rn(t, make_float2(-R, -R));
+    const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
+    float2 c = __ffma2_rn(make_float2(PA_EX2_C3, PA_EX2_C3), f, make_float2(PA_EX2_C2, PA_EX2_C2));
+    c = __ffma2_rn(c, f, make_float2(PA_EX2_C1, PA_EX2_C1));
+    c = __ffma2_rn(c, f, make_float2(PA_EX2_C0, PA_EX2_C0));
+    return make_float2(__int_as_float(__float_as_int(c.x) + (__float_as_int(t.x) << 23)),
+                       __int_as_float(__float_as_int(c.y) + (__float_as_int(t.y) << 23)));
+}
+
+// max(a, b, c) in one instruction
+__device__ __forceinline__ float max3f(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 template <int D, int BS, int G, int NQ_ = 2, int KST_ = 4, int VST_ = 4>
 struct PrefillTcConfig {
     static constexpr int NQ = NQ_;                        // 128-row query tiles per CTA
@@ -68,6 +103,7 @@ struct PrefillTcConfig {
     static constexpr int SMEM = OFF_MISC + 16 + 1024;
     static constexpr int TMEM_PER_Q = 256;                // S [0,64), P0 [64,96), P1 [96,128), O [128, 128 + D)
     static constexpr int COL_P = 64;
+    static constexpr int POLY_PAIRS = 2;                  // of every 8 pairs of P, on the FMA pipe
     static constexpr int TMEM_COLS = NQ * TMEM_PER_Q;
     static constexpr int COL_O = 128;
     static constexpr uint32_t IDESC_S = umma_idesc_bf16(BM, BN, false);
@@ -317,11 +353,17 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
                     for (int c = 0; c < 32; ++c)
                         if (kv0 + 32 * h + c > pos) sr[h][c] = 0xff800000u;        // -inf
             }
-            float mx = -INFINITY;
+            // pair i of the row tile = columns 2i, 2i + 1
+            auto pair_of = [&](int i) {
+                return make_float2(__uint_as_float(sr[i >> 4][2 * (i & 15)]), __uint_as_float(sr[i >> 4][2 * (i & 15) + 1]));
+            };
+            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
-#pragma unroll
-                for (int c = 0; c < 32; ++c) mx = fmaxf(mx, __uint_as_float(sr[h][c]));
+            for (int i = 0; i < 32; ++i) {
+                const float2 s2 = pair_of(i);
+                m4[i & 3] = max3f(m4[i & 3], s2.x, s2.y);
+            }
+            const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
             // m_run is the reference the exponentials are taken against.  It moves (and O and
             // l are rescaled) only when the tile's max exceeds it by more than 8, so p <= 2^8;
             // O / l does not depend on the reference, and rescaling becomes rare, which keeps
@@ -337,17 +379,21 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
                 moved = true;
             }
             const float mn = m_run;
-            float rs = 0.f;
+            // p = 2^(s * qk_scale - m) in pairs: one packed FMA, then the MUFU unit for most pairs
+            // and the FMA-pipe polynomial for POLY_PAIRS of every 8 (the two units run side by
+            // side); the row sum in two packed partial sums
             uint32_t pk[32];
+            const float2 sc2 = make_float2(p.qk_scale, p.qk_scale), nm2 = make_float2(-mn, -mn);
+            float2 rsa = make_float2(0.f, 0.f), rsb = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
-#pragma unroll
-                for (int c = 0; c < 32; c += 2) {
-                    const float a = ex2_approx(fmaf(__uint_as_float(sr[h][c]), p.qk_scale, -mn));
-                    const float b = ex2_approx(fmaf(__uint_as_float(sr[h][c + 1]), p.qk_scale, -mn));
-                    rs += a + b;
-                    pk[16 * h + c / 2] = pack_bf16x2(a, b);
-                }
+            for (int i = 0; i < 32; ++i) {
+                const float2 x2 = __ffma2_rn(pair_of(i), sc2, nm2);
+                const float2 e2 = (i & 7) < C::POLY_PAIRS ? ex2_poly2(x2) : make_float2(ex2_approx(x2.x), ex2_approx(x2.y));
+                if (i & 1) rsb = __fadd2_rn(rsb, e2);
+                else rsa = __fadd2_rn(rsa, e2);
+                pk[i] = pack_bf16x2(e2.x, e2.y);
+            }
+            const float rs = (rsa.x + rsb.x) + (rsa.y + rsb.y);
             l_run = l_run * alpha + rs;
             // rescale this warp's rows of O when any of their maxima moved (PV_{j-1} must be done)
             if (__any_sync(FULL, moved)) {
