@@ -604,6 +604,13 @@ def measured_bf16_peak():
     return 1590.0, "fallback"
 
 
+def prefill_kernel_name() -> str:
+    """The prefill kernel pa_prefill dispatches to (PA_PREFILL_MMA_SYNC=1 selects the mma.sync one)."""
+    if os.environ.get("PA_PREFILL_MMA_SYNC") == "1":
+        return "paged_prefill_kernel (mma.sync bf16)"
+    return "paged_prefill_tc_kernel (tcgen05.mma bf16, fp32 accumulators in tensor memory)"
+
+
 def run_prefill(args):
     """--workload prefill_*: each step writes the chunks' K/V (pa_reshape_and_cache of every
     chunk token) and runs pa_prefill; reported as attention TFLOP/s against the bf16 peak."""
@@ -688,7 +695,7 @@ def run_prefill(args):
                           "flushed between steps (2x L2 write, outside the events)")},
         "tokens_per_s": round(tot_tok / (step_ms / 1e3 / K), 1),
         "kernels_ms_alone": {"prefill": round(kern_ms / K, 5)},
-        "roofline": {"bound": "tensor", "kernel": "paged_prefill_kernel (mma.sync bf16)", "achieved": round(achieved, 1),
+        "roofline": {"bound": "tensor", "kernel": prefill_kernel_name(), "achieved": round(achieved, 1),
                      "peak": peak, "peak_kind": kind, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                      "traffic": None, "algorithmic_flops_per_launch": int(flops)},
         "gpu_launches": 2 * K,
