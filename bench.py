@@ -220,6 +220,15 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------------- our arm
+def percentiles_ms(xs):
+    """p10 / median / p90 of per-step times (ms), nearest-rank."""
+    if not xs:
+        return None
+    v = sorted(xs)
+    pick = lambda f: v[min(len(v) - 1, max(0, int(math.ceil(f * len(v))) - 1))]
+    return {"p10": round(pick(0.10), 5), "p50": round(pick(0.50), 5), "p90": round(pick(0.90), 5)}
+
+
 def run_ours(args):
     import torch
     import workloads
@@ -312,8 +321,10 @@ def run_ours(args):
         torch.cuda.nvtx.range_pop()
         if world > 1:
             dist.barrier()
+        per_step[:] = [e[0].elapsed_time(e[n_ev - 1]) for e in evs]
         return [sum(e[k].elapsed_time(e[k + 1]) for e in evs) for k in range(n_ev - 1)]
 
+    per_step = []                      # the last timed() call's per-step intervals (ms)
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
             flush.zero_()
@@ -326,6 +337,7 @@ def run_ours(args):
     t0 = time.time()
     # the timed region: K whole steps, each bracketed by two events
     step_ms = timed(step, 2, "timed")[0]
+    step_pct = percentiles_ms(per_step)
     t1 = time.time()
 
     # each kernel alone over K launches (for the roofline and the per-kernel split); an event
@@ -460,6 +472,8 @@ def run_ours(args):
                           "flushed between steps (2x L2 write, outside the events)"),
                    "parallelism": "replicas (weak scaling, no collective)" if world > 1 else "single GPU"},
         "tokens_per_s": round(tot_seqs / per_step_s, 1),
+        "tokens_per_s_32_layer_attention_only": round(tot_seqs / per_step_s / 32, 1),
+        "step_ms_rank0": step_pct,
         "pct_of_hbm_peak": round(value / world / peak, 4),
         "pct_of_nominal_8tbs": round(value / world / 8000.0, 4),
         "kernels_ms_alone": {"reshape_and_cache": round(write_ms / K, 5),
@@ -653,8 +667,10 @@ def run_prefill(args):
         torch.cuda.synchronize(dev)
         if world > 1:
             dist.barrier()
-        return sum(a.elapsed_time(b) for a, b in evs)
+        per_step[:] = [a.elapsed_time(b) for a, b in evs]
+        return sum(per_step)
 
+    per_step = []
     step = [(L.pa_reshape_and_cache, rargs), (L.pa_prefill, pargs)]
     timed(step, args.warmup)
     uuid = str(torch.cuda.get_device_properties(dev).uuid)
@@ -662,6 +678,7 @@ def run_prefill(args):
     time.sleep(0.3)
     t0 = time.time()
     step_ms = timed(step, args.steps)
+    step_pct = percentiles_ms(per_step)
     t1 = time.time()
     kern_ms = timed([(L.pa_prefill, pargs)], args.steps)
     t2 = time.time()
@@ -694,6 +711,7 @@ def run_prefill(args):
                    "l2": ("warm: no flush between steps" if args.warm_l2 else
                           "flushed between steps (2x L2 write, outside the events)")},
         "tokens_per_s": round(tot_tok / (step_ms / 1e3 / K), 1),
+        "step_ms_rank0": step_pct,
         "kernels_ms_alone": {"prefill": round(kern_ms / K, 5)},
         "roofline": {"bound": "tensor", "kernel": prefill_kernel_name(), "achieved": round(achieved, 1),
                      "peak": peak, "peak_kind": kind, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
