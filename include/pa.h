@@ -242,9 +242,13 @@ int pa_decode_step(const void *key, const void *value, int64_t key_stride, int64
  *                  longer chunk leaves its rows unwritten and flags PA_DEVERR_BAD_CHUNK)
  *   max_query_len  host-known upper bound of the chunk lengths (sizes the grid)
  *   cache_dtype    PA_CACHE_BF16 (other types: PA_ERR_UNSUPPORTED)
- * A block-table entry outside the pool is skipped, flags PA_DEVERR_BAD_BLOCK and turns the
- * affected rows into NaN.  Tensor cores (mma.sync bf16, fp32 accumulate); accuracy as
- * pa_decode for bf16 caches.  Allocates nothing; needs no workspace. */
+ * A block-table entry outside the pool is never dereferenced: it flags PA_DEVERR_BAD_BLOCK
+ * and turns the affected rows into NaN.  5th-generation tensor cores (tcgen05.mma, bf16 in,
+ * fp32 accumulators in tensor memory; the environment variable PA_PREFILL_MMA_SYNC=1 selects
+ * an mma.sync kernel instead); accuracy as pa_decode for bf16 caches (a quarter of the
+ * softmax exponentials use a cubic with relative error < 1e-4, and terms below 2^-125 of the
+ * row's running maximum come out as about that instead of 0).  Allocates nothing; needs no
+ * workspace. */
 int pa_prefill(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
                int max_blocks_per_seq, const int32_t *query_start, const int32_t *context_lens, int num_seqs,
                int max_query_len, int h_q, int h_kv, int head_dim, int block_size, int num_blocks, float scale,
