@@ -27,8 +27,9 @@
 //              or the tile's KV range ended before it).
 // Q is copied into a swizzled shared tile once.  V rows past the context are zeroed in shared
 // memory before the P V step (an unwritten NaN slot times a zero probability would poison O).
-// Every wait is bounded; on a timeout or a bad block the CTA records the error, stops, drains its
-// MMAs and frees its tensor memory; its rows come out NaN.
+// Every wait is bounded and also ends when another role has stopped the CTA; on a timeout or a
+// bad block the CTA records the error, stops, waits for its copies and MMAs in flight and frees
+// its tensor memory; its rows come out NaN.
 #pragma once
 
 #include "prefill.cuh"
@@ -68,6 +69,19 @@ __device__ __forceinline__ float2 ex2_poly2(float2 x)
     c = __ffma2_rn(c, f, make_float2(PA_EX2_C0, PA_EX2_C0));
     return make_float2(__int_as_float(__float_as_int(c.x) + (__float_as_int(t.x) << 23)),
                        __int_as_float(__float_as_int(c.y) + (__float_as_int(t.y) << 23)));
+}
+
+// As mbar_wait_bounded, but also gives up (false) as soon as *abort reads non-zero, so once one
+// role of the CTA has stopped the others do not sit out the full limit in each of their waits.
+__device__ __forceinline__ bool mbar_wait_or_abort(uint64_t *bar, uint32_t parity, const volatile int *abort)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (*abort) return false;
+        if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+    }
+    return true;
 }
 
 // max(a, b, c) in one instruction
@@ -222,6 +236,7 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
         };
         int cur = entry(lane), nxt = entry(32 + lane);
         const int k = lane / C::HALVES, hf = lane % C::HALVES;
+        int issued = 0;                                        // tiles whose copies were issued
         for (int it = 0; it < nkv; ++it) {
             if (it > 0 && it % TPB == 0) {
                 cur = nxt;
@@ -230,7 +245,7 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
             const int st = it % nst;
             int go = 1;
             if (lane == 0) {
-                if (it >= nst && !mbar_wait_bounded(&empty[st], ((it / nst) - 1) & 1)) {
+                if (it >= nst && !mbar_wait_or_abort(&empty[st], ((it / nst) - 1) & 1, abort_flag)) {
                     if (!*abort_flag) record_error(PA_DEVERR_TIMEOUT);
                     *abort_flag = 1;
                 }
@@ -243,8 +258,7 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
             if (__any_sync(FULL, mine && (phys < 0 || phys >= p.num_blocks))) {
                 if (lane == 0) {
                     record_error(PA_DEVERR_BAD_BLOCK);
-                    *abort_flag = 1;
-                    mbar_arrive(&full[st]);                    // wake the MMA thread
+                    *abort_flag = 1;                           // the MMA warps' waits see it
                 }
                 break;
             }
@@ -253,7 +267,15 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
             if (mine)
                 tma_load_2d(smem + (is_v ? C::OFF_V : C::OFF_K) + st * C::KV_TILE + hf * C::KV_HALF + k * BS * 128, map,
                             hf * 64, (phys * p.h_kv + kvh) * BS, &full[st], pol);
+            ++issued;
         }
+        // Every copy this warp issued has landed before the CTA can exit, also when it stopped
+        // early and nobody consumed the last tiles: wait (bounded) for each of the last nst
+        // tiles.  The tile nst before each was consumed before the slot was refilled, so each
+        // wait's phase is unambiguous; on the normal path these waits return at once.
+        if (lane == 0)
+            for (int i = max(0, issued - nst); i < issued; ++i) mbar_wait_bounded(&full[i % nst], (i / nst) & 1);
+        __syncwarp();
     } else if (warp >= C::MMA_WARP && warp < C::MMA_WARP + NQ) {
         // ------------------------------ MMA issue, one warp per query tile ------------------------------
         // Lane 0 issues S_j = Q K_j^T and O += P_j V_j for its tile.  Every query tile releases
@@ -269,8 +291,8 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
             const uint64_t vdesc = umma_desc_sw128(smem_addr(smem + C::OFF_V), C::KV_HALF, 1024);
             auto s_mma = [&](int j) -> bool {
                 const int st = j % KST;
-                if (!mbar_wait_bounded(&k_full[st], (j / KST) & 1) || *abort_flag) return false;
-                if (j >= 1 && (!mbar_wait_bounded(&s_free[q], (j - 1) & 1) || *abort_flag)) return false;
+                if (!mbar_wait_or_abort(&k_full[st], (j / KST) & 1, abort_flag) || *abort_flag) return false;
+                if (j >= 1 && (!mbar_wait_or_abort(&s_free[q], (j - 1) & 1, abort_flag) || *abort_flag)) return false;
                 tc_fence_after_sync();
                 const uint64_t kd = kdesc + (uint64_t)((st * C::KV_TILE) >> 4);
 #pragma unroll
@@ -282,8 +304,8 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
                 return true;
             };
             auto pv = [&](int i) -> bool {
-                if (!mbar_wait_bounded(&v_full[i % VST], (i / VST) & 1) || *abort_flag) return false;
-                if (!mbar_wait_bounded(&p_full[2 * q + (i & 1)], (i >> 1) & 1) || *abort_flag) return false;
+                if (!mbar_wait_or_abort(&v_full[i % VST], (i / VST) & 1, abort_flag) || *abort_flag) return false;
+                if (!mbar_wait_or_abort(&p_full[2 * q + (i & 1)], (i >> 1) & 1, abort_flag) || *abort_flag) return false;
                 tc_fence_after_sync();
                 const uint64_t vd = vdesc + (uint64_t)(((i % VST) * C::KV_TILE) >> 4);
                 const uint32_t pt = d_p + 32 * (i & 1);
@@ -302,9 +324,9 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
             }
             // the KV tiles past this query tile's range: release their slots as they land
             for (int j = nkq; j < nkv && ok; ++j) {
-                ok = mbar_wait_bounded(&k_full[j % KST], (j / KST) & 1) && !*abort_flag;
+                ok = mbar_wait_or_abort(&k_full[j % KST], (j / KST) & 1, abort_flag) && !*abort_flag;
                 if (ok) mbar_arrive(&k_empty[j % KST]);
-                ok = ok && mbar_wait_bounded(&v_full[j % VST], (j / VST) & 1) && !*abort_flag;
+                ok = ok && mbar_wait_or_abort(&v_full[j % VST], (j / VST) & 1, abort_flag) && !*abort_flag;
                 if (ok) mbar_arrive(&v_empty[j % VST]);
             }
             if (!ok) {
@@ -329,7 +351,7 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
         float m_run = -INFINITY, l_run = 0.f;
         bool failed = false;
         for (int j = 0; j < nkv_q; ++j) {
-            bool ok = __all_sync(FULL, mbar_wait_bounded(my_s_full, j & 1));
+            bool ok = __all_sync(FULL, mbar_wait_or_abort(my_s_full, j & 1, abort_flag));
             if (!ok || *abort_flag) {
                 failed = true;
                 break;
@@ -397,7 +419,7 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
             l_run = l_run * alpha + rs;
             // rescale this warp's rows of O when any of their maxima moved (PV_{j-1} must be done)
             if (__any_sync(FULL, moved)) {
-                ok = __all_sync(FULL, mbar_wait_bounded(&my_o_done[(j - 1) & 1], ((j - 1) >> 1) & 1));
+                ok = __all_sync(FULL, mbar_wait_or_abort(&my_o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag));
                 if (!ok || *abort_flag) {
                     failed = true;
                     break;
@@ -416,7 +438,7 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
             }
             // V rows past the context (last tile): zero them before the P V step reads the tile
             if (kv0 + BN > ctx) {
-                ok = __all_sync(FULL, mbar_wait_bounded(&v_full[j % VST], (j / VST) & 1));
+                ok = __all_sync(FULL, mbar_wait_or_abort(&v_full[j % VST], (j / VST) & 1, abort_flag));
                 if (!ok) {
                     failed = true;
                     break;
@@ -433,7 +455,7 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
             }
             // P buffer j % 2 is free once P V_{j-2} has finished
             if (j >= 2) {
-                ok = __all_sync(FULL, mbar_wait_bounded(&my_o_done[j & 1], ((j - 2) >> 1) & 1));
+                ok = __all_sync(FULL, mbar_wait_or_abort(&my_o_done[j & 1], ((j - 2) >> 1) & 1, abort_flag));
                 if (!ok || *abort_flag) {
                     failed = true;
                     break;
@@ -446,7 +468,7 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
             if (lane == 0) mbar_arrive(&my_p_full[j & 1]);
         }
         if (!failed && nkv_q > 0) {
-            const bool ok = __all_sync(FULL, mbar_wait_bounded(&my_o_done[(nkv_q - 1) & 1], ((nkv_q - 1) >> 1) & 1));
+            const bool ok = __all_sync(FULL, mbar_wait_or_abort(&my_o_done[(nkv_q - 1) & 1], ((nkv_q - 1) >> 1) & 1, abort_flag));
             failed = !ok || *abort_flag;
         }
         if (nkv_q > 0) {
