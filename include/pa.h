@@ -241,6 +241,7 @@ int pa_decode_step(const void *key, const void *value, int64_t key_stride, int64
  *   context_lens   device int32 [num_seqs], each including its chunk (>= the chunk length; a
  *                  longer chunk leaves its rows unwritten and flags PA_DEVERR_BAD_CHUNK)
  *   max_query_len  host-known upper bound of the chunk lengths (sizes the grid)
+ *   scale          finite and >= 0 (else PA_ERR_INVALID_ARG)
  *   cache_dtype    PA_CACHE_BF16 (other types: PA_ERR_UNSUPPORTED)
  * A block-table entry outside the pool is never dereferenced: it flags PA_DEVERR_BAD_BLOCK
  * and turns the affected rows into NaN.  5th-generation tensor cores (tcgen05.mma, bf16 in,

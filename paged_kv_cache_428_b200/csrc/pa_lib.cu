@@ -867,7 +867,9 @@ int pa_prefill(void *out, const void *q, const void *k_cache, const void *v_cach
 {
     if (num_seqs < 0 || max_query_len < 0 || h_q <= 0 || h_kv <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0)
         return PA_ERR_INVALID_ARG;
-    if (h_q % h_kv != 0 || !std::isfinite(scale) || !valid_cache_dtype(cache_dtype)) return PA_ERR_INVALID_ARG;
+    // scale >= 0: the kernel takes the row max of the raw scores and scales it afterwards
+    if (h_q % h_kv != 0 || !std::isfinite(scale) || scale < 0.f || !valid_cache_dtype(cache_dtype))
+        return PA_ERR_INVALID_ARG;
     if (cache_dtype != PA_CACHE_BF16) return PA_ERR_UNSUPPORTED;
     if (!supported_head_dim(head_dim) || !supported_block_size(block_size) || !supported_group(h_q / h_kv))
         return PA_ERR_UNSUPPORTED;

@@ -118,3 +118,46 @@ def test_host_validators():
     assert pa.pa_validate_block_tables(bt, torch.tensor([65, 20], dtype=torch.int32), 16, 6) == -1  # row too short
     assert pa.pa_validate_slots(torch.tensor([0, -1, 95]), 16, 6) == 0
     assert pa.pa_validate_slots(torch.tensor([96]), 16, 6) == -1
+
+
+def test_prefill_host_checks():
+    def rc(**kw):
+        a = dict(out=FAKE, q=FAKE, k=FAKE, v=FAKE, bt=FAKE, maxblk=8, qs=FAKE, ctx=FAKE, B=2, mql=64, hq=8, hkv=2,
+                 d=128, bs=16, nb=16, scale=0.088, dt=0)
+        a.update(kw)
+        return L.pa_prefill(a["out"], a["q"], a["k"], a["v"], a["bt"], a["maxblk"], a["qs"], a["ctx"], a["B"],
+                            a["mql"], a["hq"], a["hkv"], a["d"], a["bs"], a["nb"], a["scale"], a["dt"], None)
+    assert rc(hq=6, hkv=4) == -1                            # h_q % h_kv != 0
+    assert rc(d=96) == -2                                   # unsupported head dim
+    assert rc(bs=8) == -2                                   # unsupported block size
+    assert rc(hq=32, hkv=2) == -2                           # group 16 unsupported
+    assert rc(dt=1) == -2                                   # quantised caches: bf16 only
+    assert rc(dt=9) == -1                                   # not a cache type
+    assert rc(scale=float("nan")) == -1
+    assert rc(scale=-0.1) == -1                             # the kernel needs scale >= 0
+    assert rc(B=-1) == -1 and rc(mql=-1) == -1 and rc(nb=0) == -1
+    assert rc(qs=0) == -1 and rc(out=0) == -1               # null pointers
+    assert rc(q=FAKE + 4) == -1                             # misaligned rows
+    assert rc(B=0) == 0 and rc(mql=0) == 0                  # nothing to do, nothing launched
+
+
+def test_decode_step_host_checks():
+    def rc(**kw):
+        a = dict(key=FAKE, val=FAKE, kst=0, vst=0, slots=FAKE, out=FAKE, q=FAKE, kc=FAKE, vc=FAKE, bt=FAKE, maxblk=8,
+                 ctx=FAKE, B=2, maxctx=100, hq=4, hkv=2, d=64, bs=16, nb=16, scale=0.125, dt=0, ks=1.0, vs=1.0, P=0,
+                 ws=0, wsb=0)
+        a.update(kw)
+        return L.pa_decode_step(a["key"], a["val"], a["kst"], a["vst"], a["slots"], a["out"], a["q"], a["kc"], a["vc"],
+                                a["bt"], a["maxblk"], a["ctx"], a["B"], a["maxctx"], a["hq"], a["hkv"], a["d"],
+                                a["bs"], a["nb"], a["scale"], a["dt"], a["ks"], a["vs"], a["P"], a["ws"], a["wsb"],
+                                None)
+    # every rejection happens before the cache write is launched
+    assert rc(B=-1) == -1
+    assert rc(B=0) == 0
+    assert rc(hq=6, hkv=4) == -1
+    assert rc(d=96) == -2
+    assert rc(dt=1, ks=0.0) == -1                           # quantised caches need positive scales
+    assert rc(P=16, maxctx=1000) == -3                      # partials need a workspace
+    assert rc(q=0) == -1
+    assert rc(kst=100) == -1                                # key rows shorter than h_kv * d
+    assert rc(slots=0) == -1
