@@ -435,10 +435,13 @@ def run_ours(args):
 
     K = args.steps
     per_step_s = step_ms / 1e3 / K
+    # the kernel the library dispatches to for this cache type (the same switches as pa_lib.cu)
     if case.cache == "e4m3" and os.environ.get("PA_DECODE_E4M3_CUDA_CORES") == "1":
         kernel = "paged_decode_partition_kernel (E4M3, CUDA cores)"
     elif case.quantised:
-        kernel = "paged_decode_partition_mma_quant_kernel (%s codes -> fp16, tensor cores)" % case.cache.upper()
+        kernel = "paged_decode_partition_q8_kernel (%s codes converted in registers, tensor cores)" % case.cache.upper()
+    elif os.environ.get("PA_DECODE_BF16_CUDA_CORES") == "1":
+        kernel = "paged_decode_partition_kernel (bf16, CUDA cores)"
     elif P == -1:
         kernel = "paged_decode_balanced_kernel"
     else:
