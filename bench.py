@@ -220,6 +220,21 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------------- our arm
+def cow_pairs(case):
+    """(src, dst) block pairs of one copy-on-write event of a shared-prompt batch: each prompt's
+    last shared block copied into a private block of every sharer but the first."""
+    import torch
+    pb = case.meta["prompt_blocks"]
+    tab = case.block_tables.cpu()
+    seen, pairs = set(), []
+    for s in range(tab.shape[0]):
+        src = int(tab[s, pb - 1])
+        if src in seen and int(tab[s, pb]) >= 0:
+            pairs.append([src, int(tab[s, pb])])
+        seen.add(src)
+    return torch.tensor(pairs, dtype=torch.int64).reshape(-1, 2)
+
+
 def percentiles_ms(xs):
     """p10 / median / p90 of per-step times (ms), nearest-rank."""
     if not xs:
@@ -354,6 +369,19 @@ def run_ours(args):
     part_ms = timed(only(lambda *a: part_call(a[:-1], a[-1]), dargs), 2, "kernel_decode")[0]
     merge_launches = P > 0 and -(-mcl // P) > 16
     merge_ms = timed(only(L.pa_decode_merge, margs), 2, "kernel_merge")[0] if merge_launches else 0.0
+    # shared prompts: one copy-on-write event (pa_copy_blocks), timed alone on a scratch copy of
+    # the caches so that the attention workload above is untouched
+    cow = cow_pairs(case) if "prompt_blocks" in case.meta and not case.quantised else None
+    copy_ms = 0.0
+    if cow is not None and cow.shape[0] > 0:
+        kc_s, vc_s, cow_dev = kc.clone(), vc.clone(), cow.to(dev)
+
+        def copy_body(evs):
+            evs[0].record(stream)
+            pa.pa_copy_blocks([kc_s], [vc_s], cow_dev, stream=stream)
+            evs[1].record(stream)
+        copy_ms = timed(copy_body, 2, "kernel_copy_blocks")[0]
+        del kc_s, vc_s
     t2 = time.time()
     time.sleep(0.1)
     sampler.stop()
@@ -497,6 +525,12 @@ def run_ours(args):
     if "unique_tokens" in case.meta:      # shared prompts: bytes that are distinct in memory
         ub = case.meta["unique_tokens"] * case.h_kv * d * case.elem_bytes * 2
         line["unique_kv_GBs"] = round(ub * world / per_step_s / 1e9, 2)
+    if cow is not None and cow.shape[0] > 0:
+        moved = 2 * 2 * int(cow.shape[0]) * case.h_kv * case.bs * d * case.elem_bytes   # K and V, read + written
+        line["copy_blocks"] = {"pairs_per_event": int(cow.shape[0]), "us_per_event": round(copy_ms / K * 1e3, 2),
+                               "bytes_per_event": moved, "GBs": round(moved / (copy_ms / 1e3 / K) / 1e9, 1),
+                               "event": "each prompt's last shared block copied for every sharer but one",
+                               "note": "rank 0's time; an empty CUDA-event pair (~2.7 us) is included"}
     if e2e:
         line["e2e"] = {"value": round(tot_bytes / (e2e_ms / 1e3 / K) / 1e9, 2), "unit": "GB/s",
                        "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
