@@ -1,0 +1,37 @@
+"""Host-side pieces of bench.py that need no GPU: the copy-on-write event of the shared-prompt
+workloads and the per-step percentiles."""
+import pytest
+
+import bench
+import workloads
+
+
+@pytest.mark.parametrize("name,prompts,samples", [("shared_prefix_4x8", 4, 8),
+                                                   ("shared_prefix_16x8", 16, 8),
+                                                   ("shared_prefix_16x8_interleaved", 16, 8)])
+def test_cow_event_copies_each_prompts_last_shared_block_for_all_sharers_but_one(name, prompts, samples):
+    case = workloads.make_case(name, 0)
+    pairs = bench.cow_pairs(case).tolist()
+    assert len(pairs) == prompts * (samples - 1)
+    pb = case.meta["prompt_blocks"]
+    tab = case.block_tables.cpu()
+    last_shared = {int(tab[s, pb - 1]) for s in range(case.B)}
+    private = {int(tab[s, j]) for s in range(case.B) for j in range(pb, tab.shape[1]) if int(tab[s, j]) >= 0}
+    assert len(last_shared) == prompts
+    srcs = [p[0] for p in pairs]
+    dsts = [p[1] for p in pairs]
+    assert set(srcs) == last_shared and all(srcs.count(x) == samples - 1 for x in last_shared)
+    assert len(set(dsts)) == len(dsts) and set(dsts) <= private     # distinct private blocks
+    assert all(0 <= b < case.num_blocks for b in srcs + dsts)
+
+
+def test_no_cow_event_without_shared_prompts():
+    case = workloads.make_case("llama3_8b_b64", 0, B=4)
+    assert "prompt_blocks" not in case.meta
+
+
+def test_percentiles_nearest_rank():
+    xs = [float(i) for i in range(1, 101)]                # 1 .. 100
+    assert bench.percentiles_ms(xs) == {"p10": 10.0, "p50": 50.0, "p90": 90.0}
+    assert bench.percentiles_ms([3.0]) == {"p10": 3.0, "p50": 3.0, "p90": 3.0}
+    assert bench.percentiles_ms([]) is None
