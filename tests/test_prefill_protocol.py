@@ -1,0 +1,266 @@
+"""The tcgen05 prefill kernel's barrier protocol (prefill_tc.cuh), model-checked on the CPU.
+
+Roles, as the kernel runs them for one CTA (two 128-row query tiles q = 0, 1):
+  * K producer / V producer warps: tile it goes to slot it % ST after the slot's empty barrier
+    completed phase it / ST - 1; its data lands later (the full barrier completes then);
+  * one MMA thread per query tile: S_j needs K_j and (j > 0) s_free phase j - 1; P V_j needs V_j
+    and p_full phase j >> 1 of buffer j & 1; completions arrive on s_full / k_empty and o_done /
+    v_empty in issue order (tcgen05.commit); past its KV range the thread releases each K and V
+    slot as its data lands;
+  * four softmax warps per query tile: wait s_full phase j, load S_j, arrive s_free; sometimes
+    rescale O (wait o_done of P V_{j-1}); on the context's last tile wait V_j (zeroing rows);
+    before storing P_j wait o_done of P V_{j-2}; arrive p_full; at the end wait o_done of the
+    last P V and read O.
+An mbarrier parity wait for phase k passes when the number of completed phases has a parity
+other than k's, so it is only sound if that number is k or k + 1 whenever the wait is tried:
+k - 1 would pass early, k + 2 would never pass.  The model runs random interleavings and checks
+that every wait respects this, that every role finishes without deadlock, and that no shared
+buffer is overwritten while an operation still reads it or read before it holds the right tile
+(K / V slots, S, the two P buffers, O).
+
+One finding: the wait before storing P_j (for P V_{j-2}) is implied by the others.  S_j's
+commit is issued after P V_{j-2}'s on the same MMA thread and tcgen05.commit arrives only when
+all of that thread's earlier operations have finished, so a softmax that has S_j sees P V_{j-2}
+done; the kernel keeps the wait, which passes at once.
+"""
+import inspect
+import random
+import textwrap
+
+import pytest
+
+
+class Violation(AssertionError):
+    pass
+
+
+def check(cond, msg):
+    if not cond:
+        raise Violation(msg)
+
+
+class Bar:
+    def __init__(self, count):
+        self.count, self.pending, self.done = count, count, 0
+
+    def arrive(self):
+        self.pending -= 1
+        check(self.pending >= 0, "more arrivals than the barrier's count in one phase")
+        if self.pending == 0:
+            self.done += 1
+            self.pending = self.count
+
+
+def run(nkv_q, KST, VST, seed, ctx_last_tile=True, rescale_p=0.2):
+    """One CTA; nkv_q[q] = KV tiles of query tile q (as the kernel's nkv_of computes them)."""
+    rnd = random.Random(seed)
+    NQ = len(nkv_q)
+    nkv = max(nkv_q)
+    k_full = [Bar(1) for _ in range(KST)]
+    k_empty = [Bar(NQ) for _ in range(KST)]
+    v_full = [Bar(1) for _ in range(VST)]
+    v_empty = [Bar(NQ) for _ in range(VST)]
+    s_full = [Bar(1) for _ in range(NQ)]
+    s_free = [Bar(4) for _ in range(NQ)]
+    p_full = [Bar(4) for _ in range(2 * NQ)]
+    o_done = [Bar(1) for _ in range(2 * NQ)]
+    # data state
+    kslot, vslot = [None] * KST, [None] * VST              # tile whose data sits in the slot
+    kread, vread = [set() for _ in range(KST)], [set() for _ in range(VST)]   # pending MMA readers
+    sbuf = [None] * NQ                                     # tile of the completed S product
+    s_pending = [False] * NQ                               # an S product is writing S
+    sloaded = [[-1] * 4 for _ in range(NQ)]                # last S tile each softmax warp loaded
+    pbuf = [[[None] * 4 for _ in range(2)] for _ in range(NQ)]   # tile of P per buffer and warp
+    pread = [[0, 0] for _ in range(NQ)]                    # pending P V reading each P buffer
+    pv_pending = [0] * NQ                                  # pending P V (writes O)
+    inflight = []                                          # (kind, slot, tile) still landing
+    tc_queue = [[] for _ in range(NQ)]                     # per MMA thread: completions in order
+
+    def sound(bar, k):
+        check(bar.done in (k, k + 1), "wait for phase %d with %d phases completed" % (k, bar.done))
+        return bar.done == k + 1
+
+    def producer(is_v, ST):
+        full, empty = (v_full, v_empty) if is_v else (k_full, k_empty)
+        slot, readers = (vslot, vread) if is_v else (kslot, kread)
+        for it in range(nkv):
+            st = it % ST
+            if it >= ST:
+                yield (empty[st], it // ST - 1)
+            check(not readers[st], "slot %d refilled while an MMA still reads tile %s" % (st, slot[st]))
+            slot[st] = None                                # being overwritten
+            inflight.append((is_v, st, it))
+
+    def mma(q):
+        nkq = nkv_q[q]
+
+        def s_mma(j):
+            st = j % KST
+            yield (k_full[st], j // KST)
+            if j >= 1:
+                yield (s_free[q], j - 1)
+                check(all(x == j - 1 for x in sloaded[q]), "S_%d issued before every warp loaded S_%d" % (j, j - 1))
+            check(kslot[st] == j, "S_%d reads slot %d holding %s" % (j, st, kslot[st]))
+            kread[st].add((q, j))
+            s_pending[q] = True
+
+            def done():
+                kread[st].discard((q, j))
+                s_pending[q] = False
+                sbuf[q] = j
+                s_full[q].arrive()
+                k_empty[st].arrive()
+            tc_queue[q].append(done)
+
+        def pv(i):
+            st, b = i % VST, i & 1
+            yield (v_full[st], i // VST)
+            yield (p_full[2 * q + b], i >> 1)
+            check(vslot[st] == i, "P V_%d reads V slot %d holding %s" % (i, st, vslot[st]))
+            check(all(x == i for x in pbuf[q][b]), "P V_%d reads P buffer %d holding %s" % (i, b, pbuf[q][b]))
+            vread[st].add((q, i))
+            pread[q][b] += 1
+            pv_pending[q] += 1
+
+            def done():
+                vread[st].discard((q, i))
+                pread[q][b] -= 1
+                pv_pending[q] -= 1
+                o_done[2 * q + b].arrive()
+                v_empty[st].arrive()
+            tc_queue[q].append(done)
+
+        if nkq > 0:
+            yield from s_mma(0)
+        for j in range(nkq):
+            if j + 1 < nkq:
+                yield from s_mma(j + 1)
+            yield from pv(j)
+        for j in range(nkq, nkv):
+            yield (k_full[j % KST], j // KST)
+            k_empty[j % KST].arrive()
+            yield (v_full[j % VST], j // VST)
+            v_empty[j % VST].arrive()
+
+    def softmax(q, w):
+        n = nkv_q[q]
+        for j in range(n):
+            yield (s_full[q], j)
+            check(sbuf[q] == j and not s_pending[q], "warp loads S_%d while S holds %s" % (j, sbuf[q]))
+            sloaded[q][w] = j
+            s_free[q].arrive()
+            if j > 0 and rnd.random() < rescale_p:
+                yield (o_done[2 * q + ((j - 1) & 1)], (j - 1) >> 1)
+                check(pv_pending[q] == 0, "O rescaled while a P V is pending")
+            if ctx_last_tile and j == nkv - 1:
+                yield (v_full[j % VST], j // VST)
+                check(vslot[j % VST] == j, "zeroing rows of V_%d in the wrong slot contents" % j)
+            b = j & 1
+            if j >= 2:
+                yield (o_done[2 * q + b], (j - 2) >> 1)
+            check(pread[q][b] == 0, "P_%d stored into buffer %d while a P V reads it" % (j, b))
+            pbuf[q][b][w] = j
+            p_full[2 * q + b].arrive()
+        if n > 0:
+            yield (o_done[2 * q + ((n - 1) & 1)], (n - 1) >> 1)
+            check(pv_pending[q] == 0, "O read while a P V is pending")
+
+    roles = [producer(False, KST), producer(True, VST)]
+    roles += [mma(q) for q in range(NQ)]
+    roles += [softmax(q, w) for q in range(NQ) for w in range(4)]
+    waiting = [None] * len(roles)
+    alive = set(range(len(roles)))
+
+    def step(r):
+        """Advance role r until it blocks or ends; True if it made progress."""
+        progressed = False
+        while True:
+            if waiting[r] is not None:
+                if not sound(*waiting[r]):
+                    return progressed
+                waiting[r] = None
+                progressed = True
+            try:
+                waiting[r] = next(roles[r])
+                progressed = True
+            except StopIteration:
+                alive.discard(r)
+                return True
+
+    while alive or inflight or any(tc_queue):
+        choices = [("role", r) for r in sorted(alive)]
+        if inflight:
+            choices.append(("land", None))
+        choices += [("tc", q) for q in range(NQ) if tc_queue[q]]
+        kind, arg = rnd.choice(choices)
+        if kind == "role":
+            step(arg)
+        elif kind == "land":
+            is_v, st, it = inflight.pop(rnd.randrange(len(inflight)))
+            (vslot if is_v else kslot)[st] = it
+            (v_full if is_v else k_full)[st].arrive()
+        else:
+            tc_queue[arg].pop(0)()                          # one thread's completions in issue order
+        if not inflight and not any(tc_queue) and alive:
+            if not any(step(r) for r in sorted(alive)) and alive:
+                raise Violation("deadlock: %d roles blocked" % len(alive))
+    for b in k_empty + v_empty + s_free + p_full:
+        check(b.pending == b.count, "a barrier was left with partial arrivals")
+    return True
+
+
+def tile_counts(ctx, chunk, pair, TQ=32, BN=64, NQ=2):
+    """nkv_of(q) as the kernel computes it."""
+    out = []
+    for q in range(NQ):
+        t0 = (pair * NQ + q) * TQ
+        out.append(0 if t0 >= chunk else -(-(ctx - chunk + min(chunk, t0 + TQ)) // BN))
+    return out
+
+
+@pytest.mark.parametrize("KST,VST", [(4, 4), (3, 3), (2, 2), (5, 5), (4, 2)])
+def test_protocol_sound_race_free_and_deadlock_free(KST, VST):
+    rnd = random.Random(KST * 10 + VST)
+    cases = 0
+    while cases < 50:
+        chunk = rnd.randint(1, 300)
+        ctx = chunk + rnd.randint(0, 400)
+        npairs = (-(-chunk // 32) + 1) // 2
+        n = tile_counts(ctx, chunk, rnd.randrange(npairs))
+        if max(n) == 0:
+            continue
+        for seed in range(4):
+            assert run(n, KST, VST, seed=1000 * cases + seed)
+        cases += 1
+
+
+def test_second_tile_missing_and_short_ranges():
+    # an odd number of query tiles leaves the last pair with one tile (nkv_of(1) == 0)
+    for n in ([1, 0], [3, 0], [1, 1], [1, 2], [7, 8], [9, 9]):
+        for seed in range(20):
+            assert run(list(n), 4, 4, seed)
+
+
+def _mutant(old, new):
+    text = textwrap.dedent(inspect.getsource(run))
+    assert text.count(old) == 1, old
+    ns = {}
+    exec(compile(text.replace(old, new), "<mutant>", "exec"), run.__globals__, ns)
+    return ns["run"]
+
+
+@pytest.mark.parametrize("old,new", [
+    # the softmax stores P_j after waiting for P V_{j-1}'s buffer phase instead of P V_{j-2}'s
+    ("yield (o_done[2 * q + b], (j - 2) >> 1)", "yield (o_done[2 * q + b], (j - 0) >> 1)"),
+    # O rescaled after waiting for P V_{j-2} instead of P V_{j-1} (P V_{j-1} may still be adding)
+    ("yield (o_done[2 * q + ((j - 1) & 1)], (j - 1) >> 1)", "yield (o_done[2 * q + (j & 1)], max(j - 2, 0) >> 1)"),
+    # a K slot is released after one query tile's S instead of both
+    ("k_empty = [Bar(NQ) for _ in range(KST)]", "k_empty = [Bar(1) for _ in range(KST)]"),
+    # S_{j+1} issued without waiting for the softmax to have loaded S_j
+    ("            if j >= 1:\n                yield (s_free[q], j - 1)\n", "            if False:\n                pass\n"),
+])
+def test_model_catches_planted_mistakes(old, new):
+    bad = _mutant(old, new)
+    with pytest.raises(Violation):
+        for seed in range(200):
+            bad([6, 7], 4, 4, seed)
