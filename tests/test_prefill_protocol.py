@@ -51,11 +51,14 @@ class Bar:
             self.pending = self.count
 
 
-def run(nkv_q, KST, VST, seed, ctx_last_tile=True, rescale_p=0.2):
-    """One CTA; nkv_q[q] = KV tiles of query tile q (as the kernel's nkv_of computes them)."""
+def run(nkv_q, KST, VST, seed, ctx_last_tile=True, rescale_p=0.2, abort_p=0.0, bad=None):
+    """One CTA; nkv_q[q] = KV tiles of query tile q (as the kernel's nkv_of computes them).
+    abort_p: chance per scheduling step that some role raises the CTA's abort flag (a timeout);
+    bad = (is_v, tile): that producer finds a bad block-table entry there."""
     rnd = random.Random(seed)
     NQ = len(nkv_q)
     nkv = max(nkv_q)
+    abort = [False]
     k_full = [Bar(1) for _ in range(KST)]
     k_empty = [Bar(NQ) for _ in range(KST)]
     v_full = [Bar(1) for _ in range(VST)]
@@ -80,25 +83,40 @@ def run(nkv_q, KST, VST, seed, ctx_last_tile=True, rescale_p=0.2):
         check(bar.done in (k, k + 1), "wait for phase %d with %d phases completed" % (k, bar.done))
         return bar.done == k + 1
 
+    # a role yields (barrier, phase, ends_on_abort) and gets back True (passed) or False (the
+    # abort flag ended the wait); ("drain", q) waits until MMA thread q has nothing pending
     def producer(is_v, ST):
         full, empty = (v_full, v_empty) if is_v else (k_full, k_empty)
         slot, readers = (vslot, vread) if is_v else (kslot, kread)
+        issued = 0
         for it in range(nkv):
             st = it % ST
-            if it >= ST:
-                yield (empty[st], it // ST - 1)
+            if it >= ST and not (yield (empty[st], it // ST - 1, True)):
+                break
+            if abort[0]:
+                break
+            if bad == (is_v, it):
+                abort[0] = True                            # record, stop; no copy for this tile
+                break
             check(not readers[st], "slot %d refilled while an MMA still reads tile %s" % (st, slot[st]))
             slot[st] = None                                # being overwritten
             inflight.append((is_v, st, it))
+            issued += 1
+        # the kernel waits for its last ring's worth of tiles before leaving
+        for i in range(max(0, issued - ST), issued):
+            yield (full[i % ST], i // ST, False)
+        check(all(x[0] != is_v for x in inflight), "producer leaves with copies in flight")
 
     def mma(q):
         nkq = nkv_q[q]
 
         def s_mma(j):
             st = j % KST
-            yield (k_full[st], j // KST)
+            if not (yield (k_full[st], j // KST, True)) or abort[0]:
+                return False
             if j >= 1:
-                yield (s_free[q], j - 1)
+                if not (yield (s_free[q], j - 1, True)) or abort[0]:
+                    return False
                 check(all(x == j - 1 for x in sloaded[q]), "S_%d issued before every warp loaded S_%d" % (j, j - 1))
             check(kslot[st] == j, "S_%d reads slot %d holding %s" % (j, st, kslot[st]))
             kread[st].add((q, j))
@@ -111,11 +129,14 @@ def run(nkv_q, KST, VST, seed, ctx_last_tile=True, rescale_p=0.2):
                 s_full[q].arrive()
                 k_empty[st].arrive()
             tc_queue[q].append(done)
+            return True
 
         def pv(i):
             st, b = i % VST, i & 1
-            yield (v_full[st], i // VST)
-            yield (p_full[2 * q + b], i >> 1)
+            if not (yield (v_full[st], i // VST, True)) or abort[0]:
+                return False
+            if not (yield (p_full[2 * q + b], i >> 1, True)) or abort[0]:
+                return False
             check(vslot[st] == i, "P V_%d reads V slot %d holding %s" % (i, st, vslot[st]))
             check(all(x == i for x in pbuf[q][b]), "P V_%d reads P buffer %d holding %s" % (i, b, pbuf[q][b]))
             vread[st].add((q, i))
@@ -129,65 +150,97 @@ def run(nkv_q, KST, VST, seed, ctx_last_tile=True, rescale_p=0.2):
                 o_done[2 * q + b].arrive()
                 v_empty[st].arrive()
             tc_queue[q].append(done)
+            return True
 
+        ok = True
         if nkq > 0:
-            yield from s_mma(0)
+            ok = yield from s_mma(0)
         for j in range(nkq):
+            if not ok:
+                break
             if j + 1 < nkq:
-                yield from s_mma(j + 1)
-            yield from pv(j)
+                ok = yield from s_mma(j + 1)
+            if ok:
+                ok = yield from pv(j)
         for j in range(nkq, nkv):
-            yield (k_full[j % KST], j // KST)
-            k_empty[j % KST].arrive()
-            yield (v_full[j % VST], j // VST)
-            v_empty[j % VST].arrive()
+            if not ok:
+                break
+            ok = (yield (k_full[j % KST], j // KST, True)) and not abort[0]
+            if ok:
+                k_empty[j % KST].arrive()
+                ok = (yield (v_full[j % VST], j // VST, True)) and not abort[0]
+            if ok:
+                v_empty[j % VST].arrive()
+        if not ok:
+            abort[0] = True
+        yield ("drain", q)                                 # every MMA this thread issued finished
+        check(not tc_queue[q], "MMA thread leaves with products pending")
 
     def softmax(q, w):
         n = nkv_q[q]
         for j in range(n):
-            yield (s_full[q], j)
+            if not (yield (s_full[q], j, True)) or abort[0]:
+                return
             check(sbuf[q] == j and not s_pending[q], "warp loads S_%d while S holds %s" % (j, sbuf[q]))
             sloaded[q][w] = j
             s_free[q].arrive()
             if j > 0 and rnd.random() < rescale_p:
-                yield (o_done[2 * q + ((j - 1) & 1)], (j - 1) >> 1)
+                if not (yield (o_done[2 * q + ((j - 1) & 1)], (j - 1) >> 1, True)) or abort[0]:
+                    return
                 check(pv_pending[q] == 0, "O rescaled while a P V is pending")
             if ctx_last_tile and j == nkv - 1:
-                yield (v_full[j % VST], j // VST)
+                if not (yield (v_full[j % VST], j // VST, True)):
+                    return
                 check(vslot[j % VST] == j, "zeroing rows of V_%d in the wrong slot contents" % j)
             b = j & 1
             if j >= 2:
-                yield (o_done[2 * q + b], (j - 2) >> 1)
+                if not (yield (o_done[2 * q + b], (j - 2) >> 1, True)) or abort[0]:
+                    return
             check(pread[q][b] == 0, "P_%d stored into buffer %d while a P V reads it" % (j, b))
             pbuf[q][b][w] = j
             p_full[2 * q + b].arrive()
         if n > 0:
-            yield (o_done[2 * q + ((n - 1) & 1)], (n - 1) >> 1)
-            check(pv_pending[q] == 0, "O read while a P V is pending")
+            if (yield (o_done[2 * q + ((n - 1) & 1)], (n - 1) >> 1, True)) and not abort[0]:
+                check(pv_pending[q] == 0, "O read while a P V is pending")
 
     roles = [producer(False, KST), producer(True, VST)]
     roles += [mma(q) for q in range(NQ)]
     roles += [softmax(q, w) for q in range(NQ) for w in range(4)]
     waiting = [None] * len(roles)
+    started = [False] * len(roles)
     alive = set(range(len(roles)))
 
     def step(r):
         """Advance role r until it blocks or ends; True if it made progress."""
         progressed = False
         while True:
+            val = None
             if waiting[r] is not None:
-                if not sound(*waiting[r]):
-                    return progressed
+                if waiting[r][0] == "drain":
+                    if tc_queue[waiting[r][1]]:
+                        return progressed
+                    val = True
+                else:
+                    bar, k, ends_on_abort = waiting[r]
+                    if sound(bar, k):
+                        val = True
+                    elif ends_on_abort and abort[0]:
+                        val = False
+                    else:
+                        return progressed
                 waiting[r] = None
                 progressed = True
             try:
-                waiting[r] = next(roles[r])
+                waiting[r] = roles[r].send(val) if started[r] else next(roles[r])
+                started[r] = True
                 progressed = True
             except StopIteration:
                 alive.discard(r)
                 return True
 
     while alive or inflight or any(tc_queue):
+        if abort_p and not abort[0] and rnd.random() < abort_p:
+            abort[0] = True
         choices = [("role", r) for r in sorted(alive)]
         if inflight:
             choices.append(("land", None))
@@ -204,8 +257,9 @@ def run(nkv_q, KST, VST, seed, ctx_last_tile=True, rescale_p=0.2):
         if not inflight and not any(tc_queue) and alive:
             if not any(step(r) for r in sorted(alive)) and alive:
                 raise Violation("deadlock: %d roles blocked" % len(alive))
-    for b in k_empty + v_empty + s_free + p_full:
-        check(b.pending == b.count, "a barrier was left with partial arrivals")
+    if not abort[0]:
+        for b in k_empty + v_empty + s_free + p_full:
+            check(b.pending == b.count, "a barrier was left with partial arrivals")
     return True
 
 
@@ -251,16 +305,45 @@ def _mutant(old, new):
 
 @pytest.mark.parametrize("old,new", [
     # the softmax stores P_j after waiting for P V_{j-1}'s buffer phase instead of P V_{j-2}'s
-    ("yield (o_done[2 * q + b], (j - 2) >> 1)", "yield (o_done[2 * q + b], (j - 0) >> 1)"),
+    ("yield (o_done[2 * q + b], (j - 2) >> 1, True)", "yield (o_done[2 * q + b], (j - 0) >> 1, True)"),
     # O rescaled after waiting for P V_{j-2} instead of P V_{j-1} (P V_{j-1} may still be adding)
-    ("yield (o_done[2 * q + ((j - 1) & 1)], (j - 1) >> 1)", "yield (o_done[2 * q + (j & 1)], max(j - 2, 0) >> 1)"),
+    ("yield (o_done[2 * q + ((j - 1) & 1)], (j - 1) >> 1, True)",
+     "yield (o_done[2 * q + (j & 1)], max(j - 2, 0) >> 1, True)"),
     # a K slot is released after one query tile's S instead of both
     ("k_empty = [Bar(NQ) for _ in range(KST)]", "k_empty = [Bar(1) for _ in range(KST)]"),
     # S_{j+1} issued without waiting for the softmax to have loaded S_j
-    ("            if j >= 1:\n                yield (s_free[q], j - 1)\n", "            if False:\n                pass\n"),
+    ("            if j >= 1:\n                if not (yield (s_free[q], j - 1, True)) or abort[0]:\n                    return False\n",
+     "            if False:\n                pass\n"),
 ])
 def test_model_catches_planted_mistakes(old, new):
     bad = _mutant(old, new)
     with pytest.raises(Violation):
         for seed in range(200):
             bad([6, 7], 4, 4, seed)
+
+
+@pytest.mark.parametrize("KST,VST", [(4, 4), (3, 3), (2, 2)])
+def test_abort_paths_drain_and_end(KST, VST):
+    # a timeout raised at a random moment, or a bad block-table entry met by either producer at
+    # any tile: every role still finishes, the drains' parity waits are sound, no copy is in
+    # flight when a producer leaves and no MMA is pending when an MMA thread leaves
+    rnd = random.Random(7 * KST + VST)
+    for case in range(40):
+        chunk = rnd.randint(1, 300)
+        ctx = chunk + rnd.randint(0, 400)
+        npairs = (-(-chunk // 32) + 1) // 2
+        n = tile_counts(ctx, chunk, rnd.randrange(npairs))
+        if max(n) == 0:
+            continue
+        for seed in range(3):
+            assert run(n, KST, VST, seed=100 * case + seed, abort_p=0.01)
+            bad = (rnd.random() < 0.5, rnd.randrange(max(n)))
+            assert run(n, KST, VST, seed=100 * case + seed + 50, bad=bad)
+
+
+def test_model_catches_a_missing_drain():
+    # the producer leaves without waiting for its last tiles: copies may still be landing
+    bad = _mutant("        for i in range(max(0, issued - ST), issued):\n            yield (full[i % ST], i // ST, False)\n", "")
+    with pytest.raises(Violation):
+        for seed in range(300):
+            bad([6, 7], 4, 4, seed, abort_p=0.02)
