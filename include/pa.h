@@ -261,17 +261,23 @@ int pa_prefill(void *out, const void *q, const void *k_cache, const void *v_cach
  * inference engine's enqueue callback (plugins must not call cudaMalloc there, because it
  * can synchronise the device and is not allowed while the engine records work), hosts with
  * a fixed memory budget, and runtimes whose allocator belongs to someone else.
- * Same arguments and result as pa_decode, minus the workspace: the split-context partials
- * go to one library-owned array of PA_STATIC_WS_BYTES in device global memory.  Every GPU
- * on which the library's device code is loaded holds that array until the process exits.
+ * Same arguments and result as pa_decode (PA_PARTITION_AUTO included), minus the
+ * workspace: the split-context partials go to one library-owned array of
+ * PA_STATIC_WS_BYTES in device global memory.  Every GPU on which the library's device code
+ * is loaded holds that array until the process exits.
  *   - Returns PA_ERR_WORKSPACE, launching nothing, when pa_decode_workspace_size(...) for
  *     the arguments exceeds PA_STATIC_WS_BYTES (e.g. use a larger partition_size, or
- *     pa_decode with a caller workspace).
- *   - The first call on a device looks up the array's device address (once per device, with
- *     that device current); make that first call before any stream capture.
- *   - All calls share the one array and it keeps the previous call's contents (nothing in it
- *     needs to start at zero).  Calls that can overlap on the GPU -- on different streams
- *     without ordering between them -- race on it and must not be issued that way.
+ *     pa_decode with a caller workspace).  Every other argument error is also returned
+ *     before anything is queued.
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress,
+ *     with that device current) and keeps it for that device's CUDA context; make that first
+ *     call before any stream capture.  After cudaDeviceReset the next call sees a new context
+ *     and looks the address up again, so it too should come before any capture.
+ *   - All calls share the one array, and it keeps the previous call's contents.  The call
+ *     itself clears what must start at zero (the per-group counters at the front of the
+ *     array, one cudaMemsetAsync on `stream` before the decode); the caller clears nothing.
+ *   - Calls that can overlap on the GPU -- on different streams without ordering between
+ *     them -- race on the array (partials and counters) and must not be issued that way.
  *   - Calls no cudaMalloc, cudaFree or allocating library routine. */
 #define PA_STATIC_WS_BYTES (16u * 1024u * 1024u)
 

@@ -17,7 +17,7 @@ ROOT = PKG.parent
 CSRC = PKG / "csrc"
 LIB = PKG / "libpa.so"
 SOURCES = [CSRC / "pa_lib.cu", CSRC / "host.cpp", CSRC / "allocator.cpp"]
-HEADERS = [ROOT / "include" / "pa.h", CSRC / "common.cuh", CSRC / "cache_ops.cuh", CSRC / "decode.cuh", CSRC / "decode_mma.cuh", CSRC / "decode_balanced.cuh", CSRC / "decode_q8.cuh", CSRC / "prefill.cuh", CSRC / "prefill_tc.cuh", CSRC / "tc.cuh"]
+HEADERS = [ROOT / "include" / "pa.h", CSRC / "common.cuh", CSRC / "cache_ops.cuh", CSRC / "decode.cuh", CSRC / "decode_mma.cuh", CSRC / "decode_balanced.cuh", CSRC / "decode_allheads.cuh", CSRC / "decode_q8.cuh", CSRC / "prefill.cuh", CSRC / "prefill_tc.cuh", CSRC / "tc.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

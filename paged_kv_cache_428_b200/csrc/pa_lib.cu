@@ -16,6 +16,7 @@
 #include "prefill.cuh"
 #include "prefill_tc.cuh"
 #include "decode_balanced.cuh"
+#include "decode_allheads.cuh"
 
 using namespace pa;
 
@@ -133,14 +134,15 @@ EncodeTiledFn encode_tiled()
 // 64 elements (128 bytes) by block_size rows, swizzled in 128-byte atoms (two boxes per row at
 // head_dim 128).  One-byte codes: a box is a whole row (head_dim bytes) by block_size rows,
 // 128-byte swizzle for 128-byte rows, 64-byte swizzle for 64-byte rows.
+// box_rows: rows of one box (block_size for one KV head's tile; h_kv * block_size for a whole block).
 int make_cache_map(CUtensorMap *map, const void *cache, int num_blocks, int h_kv, int block_size, int head_dim,
-                   int elem_bytes)
+                   int elem_bytes, int box_rows)
 {
     EncodeTiledFn enc = encode_tiled();
     if (!enc) return PA_ERR_CUDA;
     const cuuint64_t dims[2] = {(cuuint64_t)head_dim, (cuuint64_t)num_blocks * h_kv * block_size};
     const cuuint64_t strides[1] = {(cuuint64_t)head_dim * elem_bytes};
-    const cuuint32_t box[2] = {elem_bytes == 2 ? 64u : (cuuint32_t)head_dim, (cuuint32_t)block_size};
+    const cuuint32_t box[2] = {elem_bytes == 2 ? 64u : (cuuint32_t)head_dim, (cuuint32_t)box_rows};
     const cuuint32_t estr[2] = {1, 1};
     const CUtensorMapDataType dt = elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
     const CUtensorMapSwizzle sw = (elem_bytes == 1 && head_dim == 64) ? CU_TENSOR_MAP_SWIZZLE_64B
@@ -155,26 +157,27 @@ int make_cache_map(CUtensorMap *map, const void *cache, int num_blocks, int h_kv
 // cache tensors call after call, and encoding costs host time on every launch otherwise.
 struct CachedMap {
     const void *base = nullptr;
-    int num_blocks = 0, h_kv = 0, block_size = 0, head_dim = 0, elem_bytes = 0;
+    int num_blocks = 0, h_kv = 0, block_size = 0, head_dim = 0, elem_bytes = 0, box_rows = 0;
     CUtensorMap map;
 };
 
 int cached_cache_map(CUtensorMap *map, const void *cache, int num_blocks, int h_kv, int block_size, int head_dim,
-                     int elem_bytes = 2)
+                     int elem_bytes = 2, int box_rows = 0)
 {
     constexpr int kSlots = 8;
     static thread_local CachedMap slots[kSlots];
     static thread_local int next = 0;
+    if (box_rows <= 0) box_rows = block_size;
     for (const CachedMap &c : slots) {
         if (c.base == cache && c.num_blocks == num_blocks && c.h_kv == h_kv && c.block_size == block_size &&
-            c.head_dim == head_dim && c.elem_bytes == elem_bytes) {
+            c.head_dim == head_dim && c.elem_bytes == elem_bytes && c.box_rows == box_rows) {
             *map = c.map;
             return PA_OK;
         }
     }
     CachedMap &c = slots[next];
     next = (next + 1) % kSlots;
-    const int rc = make_cache_map(&c.map, cache, num_blocks, h_kv, block_size, head_dim, elem_bytes);
+    const int rc = make_cache_map(&c.map, cache, num_blocks, h_kv, block_size, head_dim, elem_bytes, box_rows);
     if (rc != PA_OK) {
         c.base = nullptr;
         return rc;
@@ -185,6 +188,7 @@ int cached_cache_map(CUtensorMap *map, const void *cache, int num_blocks, int h_
     c.block_size = block_size;
     c.head_dim = head_dim;
     c.elem_bytes = elem_bytes;
+    c.box_rows = box_rows;
     *map = c.map;
     return PA_OK;
 }
@@ -452,6 +456,99 @@ int dispatch_balanced(int d, int bs, int g, const DecodeParams &prm, int n, cons
     return PA_ERR_UNSUPPORTED;
 }
 
+// ---- whole-block schedule (PA_PARTITION_AUTO, 8 KV heads) ------------------------------------
+// Workspace: [group counters][partial (m, l): kAllHeadsMaxCtas x 2 x h_q x 2][partial o].
+struct AllHeadsLayout {
+    size_t ml = 0, o = 0, total = 0;
+};
+
+AllHeadsLayout allheads_layout(int num_seqs, int h_q, int head_dim)
+{
+    AllHeadsLayout L;
+    L.ml = round256((size_t)num_seqs * h_q * sizeof(int));
+    L.o = L.ml + round256((size_t)kAllHeadsMaxCtas * 2 * h_q * 2 * sizeof(float));
+    L.total = L.o + (size_t)kAllHeadsMaxCtas * 2 * h_q * head_dim * sizeof(float);
+    return L;
+}
+
+// PA_DECODE_AUTO_PER_HEAD=1 keeps PA_PARTITION_AUTO on the per-KV-head balanced kernel (A/B runs).
+bool auto_per_head()
+{
+    static const bool v = env_flag("PA_DECODE_AUTO_PER_HEAD");
+    return v;
+}
+
+bool allheads_applies(int num_seqs, int h_kv, int head_dim, int block_size, int cache_dtype)
+{
+    return cache_dtype == PA_CACHE_BF16 && !bf16_on_cuda_cores() && !auto_per_head() && h_kv == kAllHeadsHkv &&
+           num_seqs <= kAllHeadsMaxSeqs && (block_size == 16 || block_size == 32) &&
+           (head_dim == 64 || head_dim == 128);
+}
+
+template <int D, int BS, int G>
+int launch_allheads(const DecodeParams &prm, int num_seqs, void *workspace, cudaStream_t st)
+{
+    constexpr int HKV = kAllHeadsHkv;
+    using AC = AllHeadsConfig<D, BS, G, HKV>;
+    static std::atomic<unsigned long long> smem_set{0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (!(smem_set.load(std::memory_order_acquire) & bit)) {
+        if (cudaFuncSetAttribute(paged_decode_allheads_kernel<D, BS, G, HKV>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, AC::smem_bytes(kAllHeadsMaxSeqs)) !=
+            cudaSuccess)
+            return PA_ERR_CUDA;
+        smem_set.fetch_or(bit, std::memory_order_release);
+    }
+    const int sms = sm_count();
+    if (sms < 1) return PA_ERR_CUDA;
+    const int ctas = sms < kAllHeadsMaxCtas ? sms : kAllHeadsMaxCtas;
+    CUtensorMap mk, mv;
+    int rc = cached_cache_map(&mk, prm.k_cache, prm.num_blocks, HKV, BS, D, 2, HKV * BS);
+    if (rc == PA_OK) rc = cached_cache_map(&mv, prm.v_cache, prm.num_blocks, HKV, BS, D, 2, HKV * BS);
+    if (rc != PA_OK) return rc;
+    const AllHeadsLayout lay = allheads_layout(num_seqs, prm.h_q, D);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    AllHeadsParams ap{};
+    ap.out = prm.out;
+    ap.q = prm.q;
+    ap.block_tables = prm.block_tables;
+    ap.context_lens = prm.context_lens;
+    ap.counters = reinterpret_cast<int *>(ws);
+    ap.part_ml = reinterpret_cast<float *>(ws + lay.ml);
+    ap.part_o = reinterpret_cast<float *>(ws + lay.o);
+    ap.max_blocks_per_seq = prm.max_blocks_per_seq;
+    ap.num_seqs = num_seqs;
+    ap.num_blocks = prm.num_blocks;
+    ap.num_ctas = ctas;
+    ap.qk_scale = prm.qk_scale;
+    ap.pdl_wait_last = prm.pdl_wait_last;
+    return launch_ex(paged_decode_allheads_kernel<D, BS, G, HKV>, dim3(ctas), dim3(AC::THREADS),
+                     (size_t)AC::smem_bytes(num_seqs), st, prm.pdl_wait_last != 0, ap, mk, mv);
+}
+
+template <int D, int BS>
+int dispatch_allheads_group(int g, const DecodeParams &prm, int n, void *ws, cudaStream_t st)
+{
+    return switch_group(g, [&](auto gc) {
+        constexpr int G = decltype(gc)::value;
+        return launch_allheads<D, BS, G>(prm, n, ws, st);
+    });
+}
+
+int dispatch_allheads(int d, int bs, int g, const DecodeParams &prm, int n, void *ws, cudaStream_t st)
+{
+    if (d == 64) {
+        if (bs == 16) return dispatch_allheads_group<64, 16>(g, prm, n, ws, st);
+        if (bs == 32) return dispatch_allheads_group<64, 32>(g, prm, n, ws, st);
+    } else if (d == 128) {
+        if (bs == 16) return dispatch_allheads_group<128, 16>(g, prm, n, ws, st);
+        if (bs == 32) return dispatch_allheads_group<128, 32>(g, prm, n, ws, st);
+    }
+    return PA_ERR_UNSUPPORTED;
+}
+
 // Shared argument checks of the decode calls.  Returns PA_OK and fills `prm`.
 int prepare_decode(DecodeParams &prm, void *out, const void *q, const void *k_cache, const void *v_cache,
                    const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
@@ -529,6 +626,9 @@ int decode_partitions_impl(void *out, const void *q, const void *k_cache, const 
                             workspace_bytes);
     if (rc != PA_OK || num_seqs == 0) return rc;
     prm.pdl_wait_last = after_append ? 1 : 0;
+    if (partition_size == PA_PARTITION_AUTO && allheads_applies(num_seqs, h_kv, head_dim, block_size, cache_dtype))
+        return dispatch_allheads(head_dim, block_size, h_q / h_kv, prm, num_seqs, workspace,
+                                 static_cast<cudaStream_t>(stream));
     if (partition_size == PA_PARTITION_AUTO && balanced_applies(num_seqs, h_q, h_kv, cache_dtype))
         return dispatch_balanced(head_dim, block_size, h_q / h_kv, prm, num_seqs, bal_layout(num_seqs, h_q, head_dim),
                                  workspace, static_cast<cudaStream_t>(stream));
@@ -676,18 +776,57 @@ static __device__ __align__(256) unsigned char g_pa_static_ws[PA_STATIC_WS_BYTES
 namespace {
 
 constexpr int kMaxDevices = 64;
-std::atomic<void *> g_static_ws_addr[kMaxDevices];
 
-// Device address of g_pa_static_ws on the current device (set up on first use).
+// The array's device address belongs to the CUDA context that was current when it was looked
+// up (the device's primary context).  After cudaDeviceReset the module is loaded again, in a
+// new context, possibly at another address; so the cache entry carries the context's id and
+// is looked up again when the current context's id differs.
+struct StaticWsEntry {
+    std::atomic<void *> addr{nullptr};
+    std::atomic<unsigned long long> ctx_id{0};
+};
+StaticWsEntry g_static_ws[kMaxDevices];
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+
+template <class Fn>
+Fn driver_fn(const char *name)
+{
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint(name, &ptr, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess)
+        return nullptr;
+    return reinterpret_cast<Fn>(ptr);
+}
+
+// Id of the CUDA context current on this thread (0 when none is current or it is unknown).
+unsigned long long current_ctx_id()
+{
+    static const CtxGetCurrentFn get_current = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+    static const CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+    if (!get_current || !get_id) return 0;
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
+
+// Device address of g_pa_static_ws on the current device, looked up on the first call on a
+// device (and again after the device's context was replaced).
 int static_ws_address(void **addr)
 {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return PA_ERR_UNSUPPORTED;
-    void *p = g_static_ws_addr[dev].load(std::memory_order_acquire);
-    if (p == nullptr) {
+    StaticWsEntry &e = g_static_ws[dev];
+    void *p = e.addr.load(std::memory_order_acquire);
+    const unsigned long long id = current_ctx_id();
+    if (p == nullptr || id == 0 || id != e.ctx_id.load(std::memory_order_acquire)) {
+        p = nullptr;
         if (cudaGetSymbolAddress(&p, g_pa_static_ws) != cudaSuccess || p == nullptr) return PA_ERR_CUDA;
-        g_static_ws_addr[dev].store(p, std::memory_order_release);
+        e.ctx_id.store(current_ctx_id(), std::memory_order_release);   // the lookup made a context current
+        e.addr.store(p, std::memory_order_release);
     }
     *addr = p;
     return PA_OK;
@@ -703,7 +842,7 @@ int pa_decode_static_ws(void *out, const void *q, const void *k_cache, const voi
                         int num_blocks, float scale, int cache_dtype, float k_scale, float v_scale,
                         int partition_size, void *stream)
 {
-    if (num_seqs < 0 || h_q <= 0 || head_dim <= 0 || max_context_len < 0 || partition_size < 0)
+    if (num_seqs < 0 || h_q <= 0 || head_dim <= 0 || max_context_len < 0 || partition_size < PA_PARTITION_AUTO)
         return PA_ERR_INVALID_ARG;
     const size_t need = pa_decode_workspace_size(num_seqs, h_q, head_dim, max_context_len, partition_size);
     if (need > PA_STATIC_WS_BYTES) return PA_ERR_WORKSPACE;           // beyond the static array
@@ -711,25 +850,37 @@ int pa_decode_static_ws(void *out, const void *q, const void *k_cache, const voi
     if (need > 0) {
         const int rc = static_ws_address(&ws);
         if (rc != PA_OK) return rc;
+    }
+    const size_t ws_bytes = need > 0 ? (size_t)PA_STATIC_WS_BYTES : 0;
+    // every argument check of pa_decode first, so that a rejected call queues nothing
+    DecodeParams chk{};
+    int rc = prepare_decode(chk, out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                            num_seqs, max_context_len, h_q, h_kv, head_dim, block_size, num_blocks, scale,
+                            cache_dtype, k_scale, v_scale, nullptr, nullptr, partition_size, ws, ws_bytes);
+    if (rc != PA_OK || num_seqs == 0) return rc;
+    if (need > 0) {
         // the group counters at the front of the scratch must start at zero (a launch that
-        // stopped early could have left counts behind); the rest needs no clearing
-        const size_t counters = ws_layout(num_seqs, h_q, head_dim,
-                                          grid_partitions(max_context_len, partition_size)).counters_bytes;
+        // stopped early could have left counts behind); both workspace layouts (fixed
+        // partitions and PA_PARTITION_AUTO) begin with the same num_seqs x h_q counters
+        const size_t counters = round256((size_t)num_seqs * h_q * sizeof(int));
         if (cudaMemsetAsync(ws, 0, counters, static_cast<cudaStream_t>(stream)) != cudaSuccess) return PA_ERR_CUDA;
     }
     return pa_decode(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
                      max_context_len, h_q, h_kv, head_dim, block_size, num_blocks, scale, cache_dtype, k_scale,
-                     v_scale, partition_size, ws, need > 0 ? (size_t)PA_STATIC_WS_BYTES : 0, stream);
+                     v_scale, partition_size, ws, ws_bytes, stream);
 }
 
 size_t pa_decode_workspace_size(int num_seqs, int h_q, int head_dim, int max_context_len, int partition_size)
 {
     if (num_seqs <= 0 || h_q <= 0 || head_dim <= 0) return 0;
     if (partition_size == PA_PARTITION_AUTO) {
-        const size_t bal = bal_layout(num_seqs, h_q, head_dim).total;
+        // the largest of the schedules AUTO can pick (h_kv is not an argument here)
+        size_t need = bal_layout(num_seqs, h_q, head_dim).total;
+        const size_t all = allheads_layout(num_seqs, h_q, head_dim).total;
         const size_t grid = pa_decode_workspace_size(num_seqs, h_q, head_dim, max_context_len,
                                                      auto_fallback_partition(max_context_len));
-        return bal > grid ? bal : grid;
+        if (all > need) need = all;
+        return grid > need ? grid : need;
     }
     if (partition_size <= 0) return 0;
     const int p_max = grid_partitions(max_context_len, partition_size);

@@ -50,6 +50,15 @@ def test_long_context_b8_sampled(orc):
     _full_parity(orc, case, rows=rows)
 
 
+def test_long_context_b8_full_size_all_rows(orc):
+    """The long-context workload at full size (8 sequences of U{32768..131072} tokens, 2.7 GB of
+    K/V, 512-token partitions: up to 256 per sequence, combined by the separate merge pass),
+    every (sequence, query head) row against the oracle, in the launch configuration
+    bench.py times."""
+    case = workloads.make_case("long_context_b8", 0, device=DEV)
+    _full_parity(orc, case)
+
+
 @pytest.mark.parametrize("seed", [0, 1])
 def test_long_context_reduced_all_rows(orc, seed):
     case = workloads.make_case("long_context_b8", seed, B=2, ctx_range=(20000, 40000))
@@ -77,6 +86,13 @@ def test_fp8_mha_b32_sampled_full_size(orc, bs):
     seqs = {0, 13, 31}
     rows = [(s, h) for s in sorted(seqs) for h in (0, 7, 19, 31)]
     _full_parity(orc, case, rows=rows, seqs=seqs)
+
+
+def test_fp8_mha_b32_bs16_full_size_all_rows(orc):
+    """The E4M3 MHA workload at full size (32 sequences x 4096 tokens x 32 KV heads, 1.07 GB of
+    codes), every row against the oracle evaluated on its own quantised cache."""
+    case = workloads.make_case("fp8_mha_b32_bs16", 0, device=DEV)
+    _full_parity(orc, case)
 
 
 @pytest.mark.parametrize("bs", [16, 32, 64])
@@ -270,13 +286,22 @@ def _mean_abs_v_under_softmax(case, kc, vc):
 
 
 def test_split_vs_unsplit_agree():
-    """Different partition sizes evaluate the same sums in a different order and round the
-    probabilities to bf16 (for p.V on the tensor cores) against different running maxima,
-    so results may differ by one output ulp plus 2 * 2^-9 * sum_t p_t |V_t| / sum_t p_t."""
+    """Split vs unsplit context: the same attention ("现代 AI 的“推理加速之谜”…" section 1,
+    softmax(q K^T / sqrt(d)) V) evaluated with different partition sizes.
+
+    Bound, derived from the kernel's arithmetic: p.V runs on the tensor cores with the
+    probabilities p_t rounded to the operand type of V (bf16, unit roundoff 2^-9), while the
+    normaliser l sums the unrounded fp32 p_t.  One evaluation's result therefore differs from
+    exact fp32 arithmetic by at most |sum_t (p~_t - p_t) V_t| / sum_t p_t <= 2^-9 * wbar, with
+    wbar = sum_t p_t |V_t| / sum_t p_t.  Two partitionings round against different running
+    maxima, so their fp32 results differ by at most 2 * 2^-9 * wbar (plus fp32 reordering, the
+    1e-6 term); each is then rounded to bf16 (half an ulp, at most 2^-8 |x|), giving
+    2^-7 * max(|a|, |b|) + 2^-8 * wbar.  The oracle tolerance (2e-2) is unchanged; this bound
+    is about 3e-3 at these magnitudes."""
     case = _with_appended(workloads.make_case("llama3_8b_b64", 2, device=DEV, B=24))
     ref = _decode(case, case.k_cache, case.v_cache, P=0).float()
     wbar = _mean_abs_v_under_softmax(case, case.k_cache, case.v_cache)
-    for P in (16, 64, 256, 512, 2048):
+    for P in (16, 64, 256, 512, 2048, AUTO):
         got = _decode(case, case.k_cache, case.v_cache, P=P).float()
         assert torch.isfinite(got).all()
         tol = 2.0 ** -7 * torch.maximum(ref.abs(), got.abs()) + 2.0 ** -8 * wbar + 1e-6
@@ -392,6 +417,17 @@ def test_auto_schedule_long_context_sampled(orc):
 def test_auto_schedule_every_variant(orc, d, bs, g):
     case = workloads.make_case("llama3_8b_b64", 11 * d + bs + g, B=7, h_q=2 * g, h_kv=2, d=d, bs=bs,
                                ctx_range=(1, 3000), pool_factor=1.2)
+    _full_parity(orc, case, partition_size=AUTO)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("bs", [16, 32])
+@pytest.mark.parametrize("g", [1, 2, 4, 8])
+def test_auto_whole_block_every_variant(orc, d, bs, g):
+    """8 KV heads: PA_PARTITION_AUTO runs the whole-block kernel (one CTA streams every head of
+    a block); every instantiated (head_dim, block size, group) against the oracle."""
+    case = workloads.make_case("llama3_8b_b64", 7 * d + bs + g, B=9, h_q=8 * g, h_kv=8, d=d, bs=bs,
+                               ctx_range=(1, 2500), pool_factor=1.2)
     _full_parity(orc, case, partition_size=AUTO)
 
 

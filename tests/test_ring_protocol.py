@@ -82,3 +82,53 @@ def test_library_stage_counts_are_multiples_of_consumer_warps():
     assert len(rows) == 6 * 7
     for stages, nw in rows:
         assert stages % nw == 0 and stages >= nw, (stages, nw)
+
+
+def _ring_all_heads(stages, nw, nunits, seed, count=None):
+    """The whole-block kernel's ring: unit k's K goes to use j = 2k and its V to j = 2k + 1,
+    stage j % stages; every consumer warp consumes every use in order and the stage's empty
+    barrier completes a phase after `count` (all nw) warps arrived."""
+    count = nw if count is None else count
+    rnd = random.Random(seed)
+    nuse = 2 * nunits
+    full_done, empty_done, arrivals = [0] * stages, [0] * stages, [0] * stages
+    landed, inflight = set(), []
+    prod, nxt = 0, [0] * nw
+    passes = lambda done, k: (done & 1) != (k & 1)
+    for _ in range(400000):
+        if all(n == nuse for n in nxt):
+            return "ok"
+        a = rnd.randrange(nw + 2)
+        if a == nw and prod < nuse:
+            s = prod % stages
+            if prod < stages or passes(empty_done[s], prod // stages - 1):
+                if any(n <= prod - stages for n in nxt):
+                    return "overwrite"                      # a warp still reads the stage's last use
+                inflight.append(prod)
+                prod += 1
+        elif a == nw + 1 and inflight:
+            j = inflight.pop(rnd.randrange(len(inflight)))
+            landed.add(j)
+            full_done[j % stages] += 1
+        elif a < nw:
+            j = nxt[a]
+            if j < nuse and passes(full_done[j % stages], j // stages):
+                if j not in landed:
+                    return "early"
+                s = j % stages
+                arrivals[s] += 1
+                if arrivals[s] == count:
+                    arrivals[s] = 0
+                    empty_done[s] += 1
+                nxt[a] += 1
+    return "stuck"
+
+
+def test_whole_block_ring_protocol_model():
+    """Every stage count the whole-block kernel instantiates (3, 6, 12: 64, 32 and 16 KB
+    stages in a 192 KB ring), with its 8 consumer warps: no early pass, no deadlock.  An
+    empty barrier initialised for one arrival instead of eight lets the producer refill a
+    stage a slower warp still reads, and the model sees it (an overwrite or an early pass)."""
+    assert any(_ring_all_heads(6, 8, 30, s, count=1) in ("early", "overwrite") for s in range(200))
+    for stages in (3, 6, 12):
+        assert all(_ring_all_heads(stages, 8, 30, s) == "ok" for s in range(60)), stages
