@@ -8,7 +8,7 @@ decode attention + partition merge) on the llama3_8b_b64 workload: 64 sequences,
 
 Prints ONE JSON line (rank 0).  `value` is KV GB/s of the whole job (algorithmic K+V bytes
 the step must read / device time of the step, CUDA events, inputs resident in HBM, L2
-flushed between steps).  `e2e` is the same metric through the binding's public calls with
+flushed between steps or inputs larger than L2).  `e2e` is the same metric through the binding's public calls with
 pinned host inputs copied in and the output copied back inside the timed region.
 `--impl reference` times the CPU oracle (the plain fp64 C implementation) on a bounded
 sample of the same workload, on the host cores.
@@ -54,7 +54,12 @@ def parse_args(argv=None):
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--warm-l2", action="store_true", help="do not flush L2 between steps")
+    ap.add_argument("--l2", choices=["auto", "write", "write+read", "none"], default="auto",
+                    help="between timed steps: write a 2x L2 buffer (write), then also read a second one so the "
+                         "flush's dirty lines are written back before the step (write+read), or nothing (none, "
+                         "for inputs larger than L2); auto = none when the step reads at least 4x L2 of distinct "
+                         "K/V, else write+read")
+    ap.add_argument("--warm-l2", action="store_true", help="same as --l2 none")
     return ap.parse_args(argv)
 
 
@@ -100,6 +105,38 @@ def shard_seeds(seed: int, world: int):
 # ------------------------------------------------------------------------------------- metrics
 def kv_bytes(case) -> int:
     return case.kv_bytes()
+
+
+def distinct_kv_bytes(case) -> int:
+    """K+V bytes of the step that are distinct in memory (shared prompt blocks counted once)."""
+    if "unique_tokens" in case.meta:
+        return case.meta["unique_tokens"] * case.h_kv * case.d * case.elem_bytes * 2
+    return kv_bytes(case)
+
+
+B200_L2_BYTES = 132120576          # what the device reports; used only where no GPU is visible
+
+
+def l2_size() -> int:
+    import torch
+    if torch.cuda.is_available():
+        return torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
+    return B200_L2_BYTES
+
+
+def l2_plan(args, distinct_bytes: int, l2: int):
+    """(mode, description) of what runs between timed steps; see L2Flush."""
+    mode = "none" if args.warm_l2 else args.l2
+    if mode == "auto":
+        mode = "none" if distinct_bytes >= 4 * l2 else "write+read"
+    desc = {
+        "none": "no flush: every step reads %d distinct bytes of K/V, %.1fx L2 (%d B)"
+                % (distinct_bytes, distinct_bytes / l2, l2),
+        "write": "flushed between steps (2x L2 write, outside the events)",
+        "write+read": "flushed between steps outside the events: 2x L2 written, then a second 2x L2 buffer "
+                      "read so that the flush's dirty lines are written back before the step",
+    }[mode]
+    return mode, desc
 
 
 def partition_kernel_bytes(case) -> int:
@@ -235,6 +272,21 @@ def cow_pairs(case):
     return torch.tensor(pairs, dtype=torch.int64).reshape(-1, 2)
 
 
+def step_config(args, case, P, world, l2_desc):
+    """The `config` object of the JSON line; both arms print the same one."""
+    per_head = case.per_head_scales
+    return {"workload": args.workload, "num_seqs": case.B, "h_q": case.h_q, "h_kv": case.h_kv, "head_dim": case.d,
+            "block_size": case.bs, "ctx": ctx_desc(case), "partition": P,
+            "num_blocks": case.num_blocks, "kv_bytes_per_step_per_gpu": kv_bytes(case),
+            "step": ("pa_decode_step: reshape_and_cache(%d new tokens) + split-context decode with in-kernel "
+                     "merge, the decode launched as a programmatic dependent of the write" % case.B
+                     if not per_head else
+                     "reshape_and_cache(%d new tokens) + split-context decode with in-kernel merge" % case.B),
+            "scales": ("per KV head" if per_head else "per tensor") if case.quantised else None,
+            "l2": l2_desc,
+            "parallelism": "replicas (weak scaling, no collective)" if world > 1 else "single GPU"}
+
+
 def percentiles_ms(xs):
     """p10 / median / p90 of per-step times (ms), nearest-rank."""
     if not xs:
@@ -242,6 +294,27 @@ def percentiles_ms(xs):
     v = sorted(xs)
     pick = lambda f: v[min(len(v) - 1, max(0, int(math.ceil(f * len(v))) - 1))]
     return {"p10": round(pick(0.10), 5), "p50": round(pick(0.50), 5), "p90": round(pick(0.90), 5)}
+
+
+class L2Flush:
+    """What runs between timed steps (outside the events).  Writing a buffer of 2x L2 evicts the
+    step's data but leaves up to a whole L2 of dirty lines, whose write-back the next step would
+    pay for (7 % of the 64-sequence decode); reading a second 2x L2 buffer after it leaves clean
+    lines.  A step whose K/V read is several times L2 needs no flush at all."""
+
+    def __init__(self, args, dev, distinct_bytes: int):
+        import torch
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+        self.mode, self.desc = l2_plan(args, distinct_bytes, l2)
+        self.wbuf = (torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+                     if self.mode in ("write", "write+read") else None)
+        self.rbuf = torch.ones(2 * l2 // 4, dtype=torch.float32, device=dev) if self.mode == "write+read" else None
+
+    def __call__(self):
+        if self.wbuf is not None:
+            self.wbuf.zero_()
+        if self.rbuf is not None:
+            self.rbuf.sum()
 
 
 def run_ours(args):
@@ -277,8 +350,7 @@ def run_ours(args):
     slots, tables, ctx = case.slot_mapping, case.block_tables, case.context_lens
     out = torch.empty((B, h_q, d), dtype=torch.bfloat16, device=dev)
     ws = pa.make_workspace(B, h_q, d, mcl, P, dev)
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+    flush = L2Flush(args, dev, distinct_kv_bytes(case))
     stream = torch.cuda.Stream(device=dev)
 
     # argument checks once; the timed loop calls the C ABI directly (which still validates),
@@ -329,8 +401,7 @@ def run_ours(args):
         torch.cuda.nvtx.range_push(nvtx)
         with torch.cuda.stream(stream):
             for i in range(args.steps):
-                if not args.warm_l2:
-                    flush.zero_()
+                flush()
                 body(evs[i])
         torch.cuda.synchronize(dev)
         torch.cuda.nvtx.range_pop()
@@ -342,7 +413,7 @@ def run_ours(args):
     per_step = []                      # the last timed() call's per-step intervals (ms)
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
-            flush.zero_()
+            flush()
             step()
     torch.cuda.synchronize(dev)
 
@@ -391,62 +462,8 @@ def run_ours(args):
     # end to end through the public calls: pinned host inputs in, result out, every step
     e2e = None
     if not args.no_e2e:
-        # one pinned host buffer holds every input of a step (q, new K/V rows, slot ids, block
-        # tables, context lengths): one host->device copy in, one device->host copy of out
-        parts = [("q", q), ("k_new", k_new), ("v_new", v_new), ("slots", slots), ("tables", tables), ("ctx", ctx)]
-        offs, total = {}, 0
-        for n, t in parts:
-            offs[n] = total
-            total += (t.numel() * t.element_size() + 255) // 256 * 256
-        host_buf = torch.empty(total, dtype=torch.uint8).pin_memory()
-        dev_buf = torch.empty(total, dtype=torch.uint8, device=dev)
-        view = lambda buf, n, t: buf[offs[n]: offs[n] + t.numel() * t.element_size()].view(t.dtype).view(t.shape)
-        for n, t in parts:
-            view(host_buf, n, t).copy_(t.cpu())
-        dv = {n: view(dev_buf, n, t) for n, t in parts}
-        out_host = torch.empty((B, h_q, d), dtype=torch.bfloat16).pin_memory()
-        h2d = sum(t.numel() * t.element_size() for _, t in parts)
-        d2h = out_host.numel() * out_host.element_size()
-        e_rargs = pa.reshape_call_args(dv["k_new"], dv["v_new"], kc, vc, dv["slots"], ks_arg, vs_arg)
-        e_dargs = pa.decode_call_args(out, dv["q"], kc, vc, dv["tables"], dv["ctx"], mcl, case.scale, P,
-                                      ks_arg, vs_arg, workspace=ws)
-
-        e_sargs = None if per_head else pa.step_call_args(dv["k_new"], dv["v_new"], dv["slots"], out, dv["q"], kc, vc,
-                                                          dv["tables"], dv["ctx"], mcl, case.scale, P, ks_arg, vs_arg,
-                                                          workspace=ws)
-
-        def e2e_step():
-            dev_buf.copy_(host_buf, non_blocking=True)
-            if e_sargs is not None:
-                rc = L.pa_decode_step(*e_sargs, sp)
-            else:
-                rc = write_call(e_rargs, sp)
-                rc |= decode_call(e_dargs, sp)
-            out_host.copy_(out, non_blocking=True)
-            if rc:
-                raise SystemExit("library call failed: %d" % rc)
-
-        with torch.cuda.stream(stream):
-            for _ in range(args.warmup):
-                flush.zero_()
-                e2e_step()
-        torch.cuda.synchronize(dev)
-        eev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize(dev)
-        torch.cuda.nvtx.range_push("timed_e2e")
-        with torch.cuda.stream(stream):
-            for i in range(args.steps):
-                if not args.warm_l2:
-                    flush.zero_()
-                eev[i][0].record(stream)
-                e2e_step()
-                eev[i][1].record(stream)
-        torch.cuda.synchronize(dev)
-        torch.cuda.nvtx.range_pop()
-        e2e_ms = sum(a.elapsed_time(b) for a, b in eev)
-        e2e = {"ms": e2e_ms, "h2d": h2d, "d2h": d2h}
+        e2e = run_e2e(args, pa, L, case, kc, vc, q, k_new, v_new, slots, tables, ctx, mcl, P, ks_arg, vs_arg,
+                      write_call, decode_call, per_head, stream, dev, world, dist, flush)
 
     errs = pa.pa_device_errors(clear=True)
     if errs:
@@ -491,17 +508,7 @@ def run_ours(args):
         "vs_baseline": None,
         "dtype": "bf16 q/out, %s KV, fp32 accumulate" % case.cache,
         "data": "synthetic",
-        "config": {"workload": args.workload, "num_seqs": B, "h_q": h_q, "h_kv": case.h_kv, "head_dim": d,
-                   "block_size": case.bs, "ctx": ctx_desc(case), "partition": P,
-                   "num_blocks": case.num_blocks, "kv_bytes_per_step_per_gpu": my_bytes,
-                   "step": ("pa_decode_step: reshape_and_cache(%d new tokens) + split-context decode with in-kernel "
-                            "merge, the decode launched as a programmatic dependent of the write" % B
-                            if not per_head else
-                            "reshape_and_cache(%d new tokens) + split-context decode with in-kernel merge" % B),
-                   "scales": ("per KV head" if case.per_head_scales else "per tensor") if case.quantised else None,
-                   "l2": ("warm: no flush between steps" if args.warm_l2 else
-                          "flushed between steps (2x L2 write, outside the events)"),
-                   "parallelism": "replicas (weak scaling, no collective)" if world > 1 else "single GPU"},
+        "config": step_config(args, case, P, world, flush.desc),
         "tokens_per_s": round(tot_seqs / per_step_s, 1),
         "tokens_per_s_32_layer_attention_only": round(tot_seqs / per_step_s / 32, 1),
         "step_ms_rank0": step_pct,
@@ -534,12 +541,114 @@ def run_ours(args):
     if e2e:
         line["e2e"] = {"value": round(tot_bytes / (e2e_ms / 1e3 / K) / 1e9, 2), "unit": "GB/s",
                        "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
-                       "ms_per_step": round(e2e_ms / K, 5)}
+                       "ms_per_step": round(e2e_ms / K, 5),
+                       "loop": "pa_decode_step through the C ABI; inputs copied in from pinned host memory and out "
+                               "copied back every step, double-buffered on two copy streams so that copies overlap "
+                               "the neighbouring steps' decode; timed from the first copy in to the last copy out; "
+                               + ("L2: " + flush.desc if flush.mode == "none" else
+                                  "L2 flushed (%s) on the compute stream before every decode, inside the timed loop"
+                                  % flush.mode)}
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(case)
     if world > 1:
         dist.destroy_process_group()
     return line
+
+
+def run_e2e(args, pa, L, case, kc, vc, q, k_new, v_new, slots, tables, ctx, mcl, P, ks_arg, vs_arg,
+            write_call, decode_call, per_head, stream, dev, world, dist, flush):
+    """The step end to end through the C ABI, as a decode loop runs it: each step's inputs (q, the
+    new K/V rows, slot ids, block tables, context lengths) are copied in from one pinned host
+    buffer, pa_decode_step runs, and `out` is copied back to pinned host memory.  Consecutive
+    steps are pipelined: two input buffers and two outputs, the host-to-device copies on one
+    stream and the device-to-host copies on another, ordered by events, so that step i+1's
+    inputs arrive and step i-1's output leaves while step i decodes.  When the step's distinct
+    K/V is several times L2 the loop runs without a flush (the `value` rule); otherwise the flush
+    runs on the compute stream before each decode, inside the timed loop.  Returns the time of
+    K steps (first copy in to last copy out)."""
+    import torch
+    B, h_q, d = case.B, case.h_q, case.d
+    parts = [("q", q), ("k_new", k_new), ("v_new", v_new), ("slots", slots), ("tables", tables), ("ctx", ctx)]
+    offs, total = {}, 0
+    for n, t in parts:
+        offs[n] = total
+        total += (t.numel() * t.element_size() + 255) // 256 * 256
+    view = lambda buf, n, t: buf[offs[n]: offs[n] + t.numel() * t.element_size()].view(t.dtype).view(t.shape)
+    host_in, dev_in, outs, out_host, sargs = [], [], [], [], []
+    for _ in range(2):
+        hb = torch.empty(total, dtype=torch.uint8).pin_memory()
+        for n, t in parts:
+            view(hb, n, t).copy_(t.cpu())
+        db = torch.empty(total, dtype=torch.uint8, device=dev)
+        dv = {n: view(db, n, t) for n, t in parts}
+        o = torch.empty((B, h_q, d), dtype=torch.bfloat16, device=dev)
+        ws = pa.make_workspace(B, h_q, d, mcl, P, dev)
+        if per_head:
+            ra = pa.reshape_call_args(dv["k_new"], dv["v_new"], kc, vc, dv["slots"], ks_arg, vs_arg)
+            da = pa.decode_call_args(o, dv["q"], kc, vc, dv["tables"], dv["ctx"], mcl, case.scale, P, ks_arg, vs_arg,
+                                     workspace=ws)
+            sargs.append(("split", ra, da, ws))
+        else:
+            sa = pa.step_call_args(dv["k_new"], dv["v_new"], dv["slots"], o, dv["q"], kc, vc, dv["tables"], dv["ctx"],
+                                   mcl, case.scale, P, ks_arg, vs_arg, workspace=ws)
+            sargs.append(("step", sa, None, ws))
+        host_in.append(hb)
+        dev_in.append(db)
+        outs.append(o)
+        out_host.append(torch.empty((B, h_q, d), dtype=torch.bfloat16).pin_memory())
+    h2d = sum(t.numel() * t.element_size() for _, t in parts)
+    d2h = out_host[0].numel() * out_host[0].element_size()
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    sp = stream.cuda_stream
+    ev_in = [torch.cuda.Event() for _ in range(2)]          # inputs of the buffer's step have landed
+    ev_dec = [torch.cuda.Event() for _ in range(2)]         # the buffer's step decoded (inputs read, out written)
+    ev_out = [torch.cuda.Event() for _ in range(2)]         # the buffer's output copied out
+
+    def loop(n):
+        for i in range(n):
+            b = i % 2
+            if i >= 2:
+                s_in.wait_event(ev_dec[b])                  # step i-2 has finished with this input buffer
+            with torch.cuda.stream(s_in):
+                dev_in[b].copy_(host_in[b], non_blocking=True)
+            ev_in[b].record(s_in)
+            stream.wait_event(ev_in[b])
+            if i >= 2:
+                stream.wait_event(ev_out[b])                # step i-2's output has left this buffer
+            if flush.mode != "none":
+                with torch.cuda.stream(stream):
+                    flush()
+            kind, a1, a2, _ = sargs[b]
+            if kind == "step":
+                rc = L.pa_decode_step(*a1, sp)
+            else:
+                rc = write_call(a1, sp)
+                rc |= decode_call(a2, sp)
+            if rc:
+                raise SystemExit("library call failed: %d" % rc)
+            ev_dec[b].record(stream)
+            s_out.wait_event(ev_dec[b])
+            with torch.cuda.stream(s_out):
+                out_host[b].copy_(outs[b], non_blocking=True)
+            ev_out[b].record(s_out)
+
+    loop(args.warmup)
+    torch.cuda.synchronize(dev)
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    torch.cuda.nvtx.range_push("timed_e2e")
+    t_start.record(s_in)
+    loop(args.steps)
+    s_out.wait_event(ev_out[(args.steps - 1) % 2])
+    t_end.record(s_out)
+    torch.cuda.synchronize(dev)
+    torch.cuda.nvtx.range_pop()
+    got = out_host[(args.steps - 1) % 2]
+    if not torch.equal(got.view(torch.int16), outs[(args.steps - 1) % 2].cpu().view(torch.int16)):
+        raise SystemExit("e2e: the copied-out result differs from the device result")
+    return {"ms": t_start.elapsed_time(t_end), "h2d": h2d, "d2h": d2h}
 
 
 def oracle_step_state(case, orc):
@@ -611,13 +720,16 @@ def run_reference(args):
     g = case.h_q // case.h_kv
     all_rows = [(s, h) for s in range(case.B) for h in range(case.h_q)]
     kw["scale"] = case.scale
-    t = time.perf_counter()
-    orc.paged_decode_rows(all_rows[:4], q, kc, vc, tab, ctx, **kw)
-    per_row = (time.perf_counter() - t) / 4
-    budget = 90.0 / max(1, args.steps + args.warmup)              # whole run within a few minutes
-    n_rows = int(max(1, min(len(all_rows), budget / max(per_row, 1e-6))))
-    pos = 0
     row_bytes = lambda r: int(ctx[r[0]]) * case.d * case.elem_bytes * 2 / g   # 1/g of the KV head's bytes
+    probe = all_rows[:case.h_q]                                    # sequence 0's rows: the cost per byte
+    t = time.perf_counter()
+    orc.paged_decode_rows(probe, q, kc, vc, tab, ctx, **kw)
+    per_byte = (time.perf_counter() - t) / max(1.0, sum(row_bytes(r) for r in probe))
+    step_s = per_byte * sum(row_bytes(r) for r in all_rows)        # the whole workload, estimated
+    budget = 150.0 / max(1, args.steps + args.warmup)             # whole run within a few minutes
+    # the whole workload per step when it fits the budget, else a rotating sample of its rows
+    n_rows = len(all_rows) if step_s <= budget else int(max(1, len(all_rows) * budget / step_s))
+    pos = 0
 
     def take():
         nonlocal pos
@@ -628,19 +740,28 @@ def run_reference(args):
     for _ in range(args.warmup):
         orc.paged_decode_rows(take(), q, kc, vc, tab, ctx, **kw)
     tot_s, tot_b = 0.0, 0.0
+    whole = n_rows == len(all_rows)
+    wkw = {k: v for k, v in kw.items() if k != "scale"}
     for _ in range(args.steps):
         rows = take()
         t = time.perf_counter()
+        if whole:                  # the whole step: the appended tokens' cache write, then every row
+            orc.reshape_and_cache(kn, vn, kc, vc, sl, d=case.d, num_blocks=case.num_blocks, **wkw)
         orc.paged_decode_rows(rows, q, kc, vc, tab, ctx, **kw)
         tot_s += time.perf_counter() - t
         tot_b += sum(row_bytes(r) for r in rows)
     value = tot_b / tot_s / 1e9
-    sample = "%d of %d (sequence, query head) decode rows per step, rotating through the batch" % (n_rows, len(all_rows))
+    if whole:
+        sample = ("the whole workload every step: cache write of the %d appended tokens and all %d (sequence, "
+                  "query head) decode rows, single-threaded fp64 C" % (case.B, len(all_rows)))
+    else:
+        sample = ("%d of %d (sequence, query head) decode rows per step, rotating through the batch"
+                  % (n_rows, len(all_rows)))
     return {"impl": "reference", "metric": METRIC, "value": round(value, 5), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(tot_s / args.steps * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": args.workload, "num_seqs": case.B, "h_q": case.h_q, "h_kv": case.h_kv,
-                       "head_dim": case.d, "block_size": case.bs, "ctx": ctx_desc(case), "kv_cache": case.cache},
+            "config": step_config(args, case, case.partition if args.partition is None else args.partition, world,
+                                  l2_plan(args, distinct_kv_bytes(case), l2_size())[1]),
             "cpu_baseline": {"value": round(value, 5), "unit": "GB/s", "cores": 1, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": round(value, 5), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -677,8 +798,7 @@ def run_prefill(args):
     case = workloads.make_prefill_case(args.workload, seed, device=dev)
     kc, vc = case.k_cache, case.v_cache
     out = torch.empty_like(case.q)
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+    flush = L2Flush(args, dev, int(case.context_lens.sum().item()) * case.h_kv * case.d * 2 * 2)
     stream = torch.cuda.Stream(device=dev)
     L, sp = pa.lib(), stream.cuda_stream
     rargs = pa.reshape_call_args(case.key_new, case.value_new, kc, vc, case.slot_mapping)
@@ -692,8 +812,7 @@ def run_prefill(args):
         torch.cuda.synchronize(dev)
         with torch.cuda.stream(stream):
             for i in range(n_steps):
-                if not args.warm_l2:
-                    flush.zero_()
+                flush()
                 evs[i][0].record(stream)
                 rc = 0
                 for fn, a in calls:
@@ -745,8 +864,7 @@ def run_prefill(args):
                    "cached_tokens": case.meta["cached"], "chunk_lens": case.meta["chunk"],
                    "attention_flops_per_step": int(flops),
                    "step": "reshape_and_cache(all chunk tokens) + pa_prefill",
-                   "l2": ("warm: no flush between steps" if args.warm_l2 else
-                          "flushed between steps (2x L2 write, outside the events)")},
+                   "l2": flush.desc},
         "tokens_per_s": round(tot_tok / (step_ms / 1e3 / K), 1),
         "step_ms_rank0": step_pct,
         "kernels_ms_alone": {"prefill": round(kern_ms / K, 5)},

@@ -260,10 +260,20 @@ __device__ __forceinline__ void cta_combine_and_write(const DecodeParams &p, con
         const int h = idx / (D / 4), d4 = idx % (D / 4);
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         const float *po = p.ws_o + (row0 + h) * p.p_max * D + 4 * d4;
-        for (int q = 0; q < n_part; ++q) {
-            const float w = mw[h * kFusedMergeMaxPartitions + q];
-            const float4 x = __ldcg(reinterpret_cast<const float4 *>(po + (size_t)q * D));
-            acc.x += w * x.x; acc.y += w * x.y; acc.z += w * x.z; acc.w += w * x.w;
+        // partials in rounds of four whose loads are issued together, summed in partition order
+        constexpr int R = 4;
+        for (int q0 = 0; q0 < n_part; q0 += R) {
+            float4 x[R];
+#pragma unroll
+            for (int u = 0; u < R; ++u)
+                if (q0 + u < n_part) x[u] = __ldcg(reinterpret_cast<const float4 *>(po + (size_t)(q0 + u) * D));
+#pragma unroll
+            for (int u = 0; u < R; ++u) {
+                if (q0 + u < n_part) {
+                    const float w = mw[h * kFusedMergeMaxPartitions + q0 + u];
+                    acc.x += w * x[u].x; acc.y += w * x[u].y; acc.z += w * x[u].z; acc.w += w * x[u].w;
+                }
+            }
         }
         __nv_bfloat16 *dst = p.out + (row0 + h) * D + 4 * d4;
         *reinterpret_cast<uint2 *>(dst) = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));

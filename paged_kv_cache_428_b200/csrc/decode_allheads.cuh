@@ -108,6 +108,103 @@ __device__ __forceinline__ UnitPos locate_unit(const int *prefix, int num_seqs, 
     return u;
 }
 
+// (m, l) <- the online-softmax combination of (m, l) and (m2, l2); m = -inf marks "nothing yet"
+// (a written partial always has a finite m: a failed one carries m = 0 and l = NaN, which the
+// combination passes on).
+__device__ __forceinline__ void ml_combine(float &m, float &l, float m2, float l2)
+{
+    if (m2 == -INFINITY) return;
+    if (m == -INFINITY) {
+        m = m2;
+        l = l2;
+        return;
+    }
+    const float mx = fmaxf(m, m2);
+    l = l * exp2f(m - mx) + l2 * exp2f(m2 - mx);
+    m = mx;
+}
+
+// The merge of one (sequence, KV head) split over CTAs c0..c1, by the warp that completed its
+// count: out = sum_c 2^(m_c - M) o_c / sum_c 2^(m_c - M) l_c for the G query heads.  Loads are
+// issued together rather than one after another: the (m, l) pairs one per lane (lane % G is the
+// head), combined across the lanes of each head; then the o rows, 8/G partials per round,
+// each lane owning D/32 dims of every head.
+template <int D, int G, int HQ>
+__device__ __forceinline__ void allheads_merge(const AllHeadsParams &p, int s, int kvh, int c0, int c1, int gstart,
+                                               int T, int Ce, int lane)
+{
+    constexpr unsigned FULL = 0xffffffffu;
+    constexpr int DPL = D / 32;
+    const int n = c1 - c0 + 1;
+    // CTA cc > c0 holds its partial in slot 0; c0 in slot 0 when the sequence starts its range,
+    // else in slot 1
+    const int slot0 = (gstart == (int)((long long)c0 * T / Ce)) ? 0 : 1;
+    auto prow = [&](int i, int h) -> size_t {
+        const int cc = c0 + i;
+        return ((size_t)cc * 2 + (i == 0 ? slot0 : 0)) * HQ + (size_t)kvh * G + h;
+    };
+    const int hl = lane % G;
+    float mm = -INFINITY, ll = 0.f;
+    for (int i = lane / G; i < n; i += 32 / G) {
+        const float2 ml = __ldcg(reinterpret_cast<const float2 *>(p.part_ml + prow(i, hl) * 2));
+        ml_combine(mm, ll, ml.x, ml.y);
+    }
+#pragma unroll
+    for (int off = 16; off >= G; off >>= 1) {
+        const float m2 = __shfl_xor_sync(FULL, mm, off), l2 = __shfl_xor_sync(FULL, ll, off);
+        ml_combine(mm, ll, m2, l2);
+    }
+    float Mx[G], invL[G], acc[G][DPL];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+        Mx[h] = __shfl_sync(FULL, mm, h);                   // lane h holds head h
+        invL[h] = 1.f / __shfl_sync(FULL, ll, h);
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) acc[h][e] = 0.f;
+    }
+    constexpr int UNR = cmax(1, 8 / G);                     // partials per round: 8 (head, partial) rows
+    for (int i0 = 0; i0 < n; i0 += UNR) {
+        float mv[UNR][G];
+        float ov[UNR][G][DPL];
+#pragma unroll
+        for (int u = 0; u < UNR; ++u) {
+            const int i = i0 + u < n ? i0 + u : n - 1;      // past the end: re-read the last one, weight 0
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                const size_t ps = prow(i, h);
+                mv[u][h] = __ldcg(p.part_ml + ps * 2);
+                const float *po = p.part_o + ps * D + DPL * lane;
+                if constexpr (DPL == 4) {
+                    const float4 v = __ldcg(reinterpret_cast<const float4 *>(po));
+                    ov[u][h][0] = v.x; ov[u][h][1] = v.y; ov[u][h][2] = v.z; ov[u][h][3] = v.w;
+                } else {
+                    const float2 v = __ldcg(reinterpret_cast<const float2 *>(po));
+                    ov[u][h][0] = v.x; ov[u][h][1] = v.y;
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < UNR; ++u) {
+            if (i0 + u < n) {
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    const float w = exp2f(mv[u][h] - Mx[h]) * invL[h];
+#pragma unroll
+                    for (int e = 0; e < DPL; ++e) acc[h][e] += w * ov[u][h][e];
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+        __nv_bfloat16 *dst = p.out + ((size_t)s * HQ + (size_t)kvh * G + h) * D + DPL * lane;
+        if constexpr (DPL == 4)
+            *reinterpret_cast<uint2 *>(dst) = make_uint2(pack_bf16x2(acc[h][0], acc[h][1]), pack_bf16x2(acc[h][2], acc[h][3]));
+        else
+            *reinterpret_cast<uint32_t *>(dst) = pack_bf16x2(acc[h][0], acc[h][1]);
+    }
+}
+
 template <int D, int BS, int G, int HKV>
 __global__ void __launch_bounds__(AllHeadsConfig<D, BS, G, HKV>::THREADS, 1)
     paged_decode_allheads_kernel(const AllHeadsParams p, const __grid_constant__ CUtensorMap tmap_k,
@@ -414,7 +511,7 @@ __global__ void __launch_bounds__(AllHeadsConfig<D, BS, G, HKV>::THREADS, 1)
                             po[16 * mt + r + 8] = failed ? __int_as_float(0x7fc00000) : o[mt][2 + j];
                         }
                         if (r == 0) {
-                            p.part_ml[ps * 2] = m_run[j];
+                            p.part_ml[ps * 2] = failed ? 0.f : m_run[j];
                             p.part_ml[ps * 2 + 1] = failed ? __int_as_float(0x7fc00000) : l_run[j];
                         }
                     }
@@ -436,53 +533,7 @@ __global__ void __launch_bounds__(AllHeadsConfig<D, BS, G, HKV>::THREADS, 1)
                     }
                 }
                 last = __shfl_sync(FULL, last, 0);
-                if (last) {
-                    // CTA cc > c0 holds the partial in slot 0; c0 in slot 0 when the sequence
-                    // starts its range, else in slot 1
-                    const int slot0 = (gstart == (int)((long long)c0 * T / Ce)) ? 0 : 1;
-                    for (int h = 0; h < G; ++h) {
-                        const size_t hrow = (size_t)kvh * G + h;
-                        float Mx = -INFINITY;
-                        for (int cc = c0 + lane; cc <= c1; cc += 32) {
-                            const size_t ps = ((size_t)cc * 2 + (cc == c0 ? slot0 : 0)) * HQ + hrow;
-                            Mx = fmaxf(Mx, __ldcg(p.part_ml + ps * 2));
-                        }
-#pragma unroll
-                        for (int off = 16; off > 0; off >>= 1) Mx = fmaxf(Mx, __shfl_xor_sync(FULL, Mx, off));
-                        float L = 0.f;
-                        for (int cc = c0 + lane; cc <= c1; cc += 32) {
-                            const size_t ps = ((size_t)cc * 2 + (cc == c0 ? slot0 : 0)) * HQ + hrow;
-                            const float2 ml = __ldcg(reinterpret_cast<const float2 *>(p.part_ml + ps * 2));
-                            L += exp2f(ml.x - Mx) * ml.y;
-                        }
-#pragma unroll
-                        for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(FULL, L, off);
-                        const float invL = 1.f / L;
-                        // lane owns D/32 consecutive dims
-                        constexpr int DPL = D / 32;
-                        float acc[DPL];
-#pragma unroll
-                        for (int i = 0; i < DPL; ++i) acc[i] = 0.f;
-                        for (int cc = c0; cc <= c1; ++cc) {
-                            const size_t ps = ((size_t)cc * 2 + (cc == c0 ? slot0 : 0)) * HQ + hrow;
-                            const float w = exp2f(__ldcg(p.part_ml + ps * 2) - Mx) * invL;
-                            const float *po = p.part_o + ps * D + DPL * lane;
-                            if constexpr (DPL == 4) {
-                                const float4 v = __ldcg(reinterpret_cast<const float4 *>(po));
-                                acc[0] += w * v.x; acc[1] += w * v.y; acc[2] += w * v.z; acc[3] += w * v.w;
-                            } else {
-                                const float2 v = __ldcg(reinterpret_cast<const float2 *>(po));
-                                acc[0] += w * v.x; acc[1] += w * v.y;
-                            }
-                        }
-                        __nv_bfloat16 *dst = p.out + ((size_t)cur.s * HQ + hrow) * D + DPL * lane;
-                        if constexpr (DPL == 4)
-                            *reinterpret_cast<uint2 *>(dst) =
-                                make_uint2(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]));
-                        else
-                            *reinterpret_cast<uint32_t *>(dst) = pack_bf16x2(acc[0], acc[1]);
-                    }
-                }
+                if (last) allheads_merge<D, G, HQ>(p, cur.s, kvh, c0, c1, gstart, T, Ce, lane);
             }
             // ---- next sequence ----
             x = seg_end;
