@@ -177,8 +177,9 @@ __device__ __forceinline__ void q8_consume_block(const uint8_t *ktile, int valid
         if (sub * 16 >= valid) break;
         // matrices of one x4 load: (tokens 0-7, chunk c), (tokens 8-15, chunk c), then chunk c + 1
         const int tok = sub * 16 + (mat & 1) * 8 + mrow;
-        // ---- S^T = K . Q^T for 16 tokens ----
-        float sT[4] = {0.f, 0.f, 0.f, 0.f};
+        // ---- S^T = K . Q^T for 16 tokens (even and odd k-steps in two accumulators: two
+        //      dependency chains of half the length) ----
+        float sA[4] = {0.f, 0.f, 0.f, 0.f}, sB[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int ks = 0; ks < C::KS; ks += 2) {
             uint32_t w[4];
@@ -186,11 +187,12 @@ __device__ __forceinline__ void q8_consume_block(const uint8_t *ktile, int valid
             uint32_t a0, a1, a2, a3;
             q8_quad_to_f16<QT>(w[0], a0, a2);
             q8_quad_to_f16<QT>(w[1], a1, a3);
-            mma_f16_16816(sT, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
+            mma_f16_16816(sA, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
             q8_quad_to_f16<QT>(w[2], a0, a2);
             q8_quad_to_f16<QT>(w[3], a1, a3);
-            mma_f16_16816(sT, a0, a1, a2, a3, qb[ks + 1][0], qb[ks + 1][1]);
+            mma_f16_16816(sB, a0, a1, a2, a3, qb[ks + 1][0], qb[ks + 1][1]);
         }
+        const float sT[4] = {sA[0] + sB[0], sA[1] + sB[1], sA[2] + sB[2], sA[3] + sB[3]};
         // ---- online softmax: tokens r and r + 8, heads 2tq and 2tq + 1 ----
         const int t0 = sub * 16 + r;
         const float x0 = t0 < valid ? sT[0] * qk_scale : -INFINITY;
