@@ -5,7 +5,8 @@
 // (decode_mma.cuh): one CTA per (context partition, KV head, sequence), a producer warp
 // streaming each physical block's K and V code tiles through an mbarrier ring, consumer warps
 // folding whole blocks into their own online-softmax state with mma.sync m16n8k16 (fp16 in,
-// fp32 accumulate).  Both code sets are exact in fp16.
+// fp32 accumulate).  Both code sets are exact in fp16.  INT8 K codes enter the scores as
+// c + 1152 (one byte permute each, no subtraction); 1152 * sum(q) is taken off every score.
 //
 // The code tiles arrive by 2-D TMA exactly as stored (one byte per element, rows of D bytes,
 // 128-byte swizzle for D = 128, 64-byte swizzle for D = 64) and are read with ldmatrix treating
@@ -68,7 +69,10 @@ __device__ __forceinline__ uint32_t swz_q8(int row, int chunk)
     else return static_cast<uint32_t>(row * 64 + ((chunk ^ ((row >> 1) & 3)) << 4));
 }
 
-// Four codes (byte 0 first) -> fp16 pairs (codes 0, 1) and (codes 2, 3).
+// Four K codes (byte 0 first) -> fp16 pairs (codes 0, 1) and (codes 2, 3).  E4M3: the values.
+// INT8: the values plus 1152 (the biased code c + 128 in the mantissa of 1024, exact), so the
+// subtraction is left out here; q . (k + 1152) - 1152 * sum(q) is taken from the scores instead
+// (q8_k_bias), one subtraction per score rather than two per four codes.
 template <int QT>
 __device__ __forceinline__ void q8_quad_to_f16(uint32_t w, uint32_t &lo, uint32_t &hi)
 {
@@ -76,7 +80,34 @@ __device__ __forceinline__ void q8_quad_to_f16(uint32_t w, uint32_t &lo, uint32_
         lo = e4m3x2_to_f16x2(w & 0xffffu);
         hi = e4m3x2_to_f16x2(w >> 16);
     } else {
-        s8x4_to_f16x2x2(w, lo, hi);
+        const uint32_t u = w ^ 0x80808080u;
+        asm("prmt.b32 %0, %1, %2, 0x4140;" : "=r"(lo) : "r"(u), "r"(0x64646464u));
+        asm("prmt.b32 %0, %1, %2, 0x4342;" : "=r"(hi) : "r"(u), "r"(0x64646464u));
+    }
+}
+
+// For INT8 K codes: 1152 * sum over d of the (fp16) q of each of this lane's two heads 2t, 2t+1
+// (t = lane % 4) -- what the scores of biased codes carry on top of q . k; 0 for E4M3.
+template <class C, int QT>
+__device__ __forceinline__ void q8_k_bias(const uint32_t (&qb)[C::KS][2], int lane, float (&bias)[2])
+{
+    bias[0] = bias[1] = 0.f;
+    if constexpr (QT == 2) {
+        float sum = 0.f;                              // this lane's dims of head lane / 4
+#pragma unroll
+        for (int ks = 0; ks < C::KS; ++ks) {
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const __half2 h = *reinterpret_cast<const __half2 *>(&qb[ks][j]);
+                const float2 f = __half22float2(h);
+                sum += f.x + f.y;
+            }
+        }
+        sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+        sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+        const int tq = lane & 3;
+        bias[0] = 1152.f * __shfl_sync(0xffffffffu, sum, 4 * (2 * tq));
+        bias[1] = 1152.f * __shfl_sync(0xffffffffu, sum, 4 * (2 * tq + 1));
     }
 }
 
@@ -164,8 +195,8 @@ __device__ __forceinline__ void q8_pv(uint32_t vbase, int tok, int mat, int u, i
 // o[mt][0..1] are dim 16 mt + 2 (T/4), o[mt][2..3] dim 16 mt + 2 (T/4) + 1 (heads 2t, 2t+1).
 template <class C, int D, int QT>
 __device__ __forceinline__ void q8_consume_block(const uint8_t *ktile, int valid, const uint32_t (&qb)[C::KS][2],
-                                                 float qk_scale, float (&m_run)[2], float (&l_run)[2],
-                                                 float (&o)[C::MT][4], int lane)
+                                                 const float (&kbias)[2], float qk_scale, float (&m_run)[2],
+                                                 float (&l_run)[2], float (&o)[C::MT][4], int lane)
 {
     constexpr unsigned FULL = 0xffffffffu;
     const uint32_t kbase = smem_addr(ktile);
@@ -192,7 +223,8 @@ __device__ __forceinline__ void q8_consume_block(const uint8_t *ktile, int valid
             q8_quad_to_f16<QT>(w[3], a1, a3);
             mma_f16_16816(sB, a0, a1, a2, a3, qb[ks + 1][0], qb[ks + 1][1]);
         }
-        const float sT[4] = {sA[0] + sB[0], sA[1] + sB[1], sA[2] + sB[2], sA[3] + sB[3]};
+        const float sT[4] = {sA[0] + sB[0] - kbias[0], sA[1] + sB[1] - kbias[1], sA[2] + sB[2] - kbias[0],
+                             sA[3] + sB[3] - kbias[1]};
         // ---- online softmax: tokens r and r + 8, heads 2tq and 2tq + 1 ----
         const int t0 = sub * 16 + r;
         const float x0 = t0 < valid ? sT[0] * qk_scale : -INFINITY;
@@ -339,6 +371,8 @@ __global__ void __maxnreg__(96)
         uint32_t qb[C::KS][2];
         const float qk_scale = p.qk_scale * head_k_factor(p, kvh) *
                                q8_load_q<C, G, D>(qb, p.q + ((size_t)seq * p.h_q + (size_t)kvh * G) * D, lane);
+        float kbias[2];
+        q8_k_bias<C, QT>(qb, lane, kbias);
         for (int i = warp; i < nblk; i += NW) {
             if (*abort_flag) break;
             const int st = i % STAGES;
@@ -354,7 +388,7 @@ __global__ void __maxnreg__(96)
                 if (lane == 0) *bad_flag = 1;
             } else {
                 q8_consume_block<C, D, QT>(stages + st * C::STAGE_BYTES, min(BS, tok_end - (tok_begin + i * BS)), qb,
-                                           qk_scale, m_run, l_run, o, lane);
+                                           kbias, qk_scale, m_run, l_run, o, lane);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty_bar[st]);
