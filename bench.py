@@ -2,7 +2,7 @@
 """Benchmark of one paged decode step (cache write of the appended tokens + split-context
 decode attention + partition merge) on the llama3_8b_b64 workload: 64 sequences, 32 query /
 8 KV heads, head_dim 128, bf16 KV in 16-token blocks drawn shuffled from a pool sized to
-1.1x demand, contexts ~ U{512..4096}.
+1.1x demand, contexts ~ U{512..4096}, 2048-token partitions.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -487,6 +487,8 @@ def run_ours(args):
         kernel = "paged_decode_partition_q8_kernel (%s codes converted in registers, tensor cores)" % case.cache.upper()
     elif os.environ.get("PA_DECODE_BF16_CUDA_CORES") == "1":
         kernel = "paged_decode_partition_kernel (bf16, CUDA cores)"
+    elif P == -1 and os.environ.get("PA_DECODE_AUTO_WHOLE_BLOCK") == "1" and case.h_kv == 8 and case.bs in (16, 32):
+        kernel = "paged_decode_allheads_kernel + paged_decode_allheads_merge_kernel"
     elif P == -1:
         kernel = "paged_decode_balanced_kernel"
     else:

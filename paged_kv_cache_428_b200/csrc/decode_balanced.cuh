@@ -141,7 +141,7 @@ __device__ __forceinline__ FlatPos locate_block(const int *prefix, int num_seqs,
 }
 
 // CTA whose range holds flat block x: the largest c with floor(c T / C) <= x (C <= T).
-__device__ __forceinline__ int cta_of_block(long long x, long long total, int num_ctas)
+__host__ __device__ __forceinline__ int cta_of_block(long long x, long long total, int num_ctas)
 {
     return (int)(((x + 1) * num_ctas - 1) / total);
 }

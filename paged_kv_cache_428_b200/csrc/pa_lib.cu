@@ -1,5 +1,6 @@
 // pa_lib.cu -- C-ABI entry points of the device calls (argument checks, dispatch, launch).
 // All device code of the library is in this one translation unit.
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
@@ -457,30 +458,36 @@ int dispatch_balanced(int d, int bs, int g, const DecodeParams &prm, int n, cons
 }
 
 // ---- whole-block schedule (PA_PARTITION_AUTO, 8 KV heads) ------------------------------------
-// Workspace: [group counters][partial (m, l): kAllHeadsMaxCtas x 2 x h_q x 2][partial o].
+// Workspace: [chunk pool: 16 ints][block prefix sums: num_seqs + 1 ints] (counters_bytes, zero
+// before the first launch; every launch leaves the pool zero) [partial (m, l): kAllHeadsSlots x
+// h_q x 2 floats][partial o: kAllHeadsSlots x h_q x head_dim floats].
 struct AllHeadsLayout {
-    size_t ml = 0, o = 0, total = 0;
+    size_t prefix = 0, ml = 0, o = 0, total = 0, counters_bytes = 0;
 };
 
 AllHeadsLayout allheads_layout(int num_seqs, int h_q, int head_dim)
 {
     AllHeadsLayout L;
-    L.ml = round256((size_t)num_seqs * h_q * sizeof(int));
-    L.o = L.ml + round256((size_t)kAllHeadsMaxCtas * 2 * h_q * 2 * sizeof(float));
-    L.total = L.o + (size_t)kAllHeadsMaxCtas * 2 * h_q * head_dim * sizeof(float);
+    L.prefix = 16 * sizeof(int);
+    L.counters_bytes = round256(L.prefix + ((size_t)num_seqs + 1) * sizeof(int));
+    L.ml = L.counters_bytes;
+    L.o = L.ml + round256((size_t)kAllHeadsSlots * h_q * 2 * sizeof(float));
+    L.total = L.o + (size_t)kAllHeadsSlots * h_q * head_dim * sizeof(float);
     return L;
 }
 
-// PA_DECODE_AUTO_PER_HEAD=1 keeps PA_PARTITION_AUTO on the per-KV-head balanced kernel (A/B runs).
-bool auto_per_head()
+// PA_DECODE_AUTO_WHOLE_BLOCK=1 runs PA_PARTITION_AUTO at 8 KV heads on the whole-block kernel
+// instead of the per-KV-head balanced kernel (A/B runs: measured slower on the 64-sequence
+// workload, 114.6 against 108.7 us, the streaming rate being the same and its merge a second launch).
+bool auto_whole_block()
 {
-    static const bool v = env_flag("PA_DECODE_AUTO_PER_HEAD");
+    static const bool v = env_flag("PA_DECODE_AUTO_WHOLE_BLOCK");
     return v;
 }
 
 bool allheads_applies(int num_seqs, int h_kv, int head_dim, int block_size, int cache_dtype)
 {
-    return cache_dtype == PA_CACHE_BF16 && !bf16_on_cuda_cores() && !auto_per_head() && h_kv == kAllHeadsHkv &&
+    return cache_dtype == PA_CACHE_BF16 && !bf16_on_cuda_cores() && auto_whole_block() && h_kv == kAllHeadsHkv &&
            num_seqs <= kAllHeadsMaxSeqs && (block_size == 16 || block_size == 32) &&
            (head_dim == 64 || head_dim == 128);
 }
@@ -515,7 +522,8 @@ int launch_allheads(const DecodeParams &prm, int num_seqs, void *workspace, cuda
     ap.q = prm.q;
     ap.block_tables = prm.block_tables;
     ap.context_lens = prm.context_lens;
-    ap.counters = reinterpret_cast<int *>(ws);
+    ap.pool = reinterpret_cast<int *>(ws);
+    ap.prefix_out = reinterpret_cast<int *>(ws + lay.prefix);
     ap.part_ml = reinterpret_cast<float *>(ws + lay.ml);
     ap.part_o = reinterpret_cast<float *>(ws + lay.o);
     ap.max_blocks_per_seq = prm.max_blocks_per_seq;
@@ -524,8 +532,21 @@ int launch_allheads(const DecodeParams &prm, int num_seqs, void *workspace, cuda
     ap.num_ctas = ctas;
     ap.qk_scale = prm.qk_scale;
     ap.pdl_wait_last = prm.pdl_wait_last;
-    return launch_ex(paged_decode_allheads_kernel<D, BS, G, HKV>, dim3(ctas), dim3(AC::THREADS),
-                     (size_t)AC::smem_bytes(num_seqs), st, prm.pdl_wait_last != 0, ap, mk, mv);
+    rc = launch_ex(paged_decode_allheads_kernel<D, BS, G, HKV>, dim3(ctas), dim3(AC::THREADS),
+                   (size_t)AC::smem_bytes(num_seqs), st, prm.pdl_wait_last != 0, ap, mk, mv);
+    if (rc != PA_OK) return rc;
+    // the split sequences' pieces, combined by a second launch that may start while the first
+    // one finishes (it waits for it before reading anything)
+    AllHeadsMergeParams mp{};
+    mp.out = prm.out;
+    mp.prefix = ap.prefix_out;
+    mp.part_ml = ap.part_ml;
+    mp.part_o = ap.part_o;
+    mp.num_seqs = num_seqs;
+    mp.h_q = prm.h_q;
+    mp.num_ctas = ctas;
+    return launch_ex(paged_decode_allheads_merge_kernel<D>, dim3(prm.h_q, num_seqs), dim3(kAllHeadsMergeWarps * 32), 0,
+                     st, true, mp);
 }
 
 template <int D, int BS>
@@ -859,10 +880,12 @@ int pa_decode_static_ws(void *out, const void *q, const void *k_cache, const voi
                             cache_dtype, k_scale, v_scale, nullptr, nullptr, partition_size, ws, ws_bytes);
     if (rc != PA_OK || num_seqs == 0) return rc;
     if (need > 0) {
-        // the group counters at the front of the scratch must start at zero (a launch that
-        // stopped early could have left counts behind); both workspace layouts (fixed
-        // partitions and PA_PARTITION_AUTO) begin with the same num_seqs x h_q counters
-        const size_t counters = round256((size_t)num_seqs * h_q * sizeof(int));
+        // the counters at the front of the scratch must start at zero (a launch that stopped
+        // early could have left counts behind): the largest counter area of the workspace
+        // layouts (fixed partitions, the PA_PARTITION_AUTO schedules), which every layout's
+        // size covers
+        const size_t counters = std::max(round256((size_t)num_seqs * h_q * sizeof(int)),
+                                         allheads_layout(num_seqs, h_q, head_dim).counters_bytes);
         if (cudaMemsetAsync(ws, 0, counters, static_cast<cudaStream_t>(stream)) != cudaSuccess) return PA_ERR_CUDA;
     }
     return pa_decode(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,

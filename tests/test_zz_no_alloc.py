@@ -82,8 +82,9 @@ def test_static_workspace_decode_matches_pa_decode_and_oracle(orc):
     case = workloads.make_case("llama3_8b_b64", 24, B=5, ctx_range=(20, 700))
     assert pa.pa_decode_workspace_size(case.B, case.h_q, case.d, case.max_context_len, 0) == 0
     _check_static(orc, case, 0, "bf16 P=0")
-    # 4. the balanced schedule (PA_PARTITION_AUTO) with its own partial layout
-    _check_static(orc, workloads.make_case("llama3_8b_b64", 25, B=12), pa.PA_PARTITION_AUTO, "bf16 AUTO")
+    # 4. PA_PARTITION_AUTO (the balanced schedule with its own partial layout; 16 query heads keep
+    #    the largest AUTO workspace inside the array)
+    _check_static(orc, workloads.make_case("llama3_8b_b64", 25, B=12, h_q=16), pa.PA_PARTITION_AUTO, "bf16 AUTO")
     # 5. a one-byte-code cache (INT8, per-tensor scales) on the tensor-core q8 kernel
     _check_static(orc, workloads.make_case("int8_mha_b32_bs16", 26, B=4, ctx_fixed=1500), 512, "int8 P=512")
     assert big > 0

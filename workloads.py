@@ -49,7 +49,7 @@ CONFIGS = {
     "tiny_gqa2_d64": dict(B=2, h_q=4, h_kv=2, d=64, bs=16, cache="bf16", ctx_cached=(37, 80),
                           num_blocks=16, partition=0),
     "llama3_8b_b64": dict(B=64, h_q=32, h_kv=8, d=128, bs=16, cache="bf16", ctx_range=(512, 4096),
-                          pool_factor=1.1, partition=512),
+                          pool_factor=1.1, partition=2048),
     "long_context_b8": dict(B=8, h_q=32, h_kv=8, d=128, bs=16, cache="bf16",
                             ctx_range=(32768, 131072), pool_factor=1.0, partition=512),
     "shared_prefix_4x8": dict(prompts=4, samples=8, prompt_len=2048, tail_range=(0, 256), h_q=32,
