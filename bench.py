@@ -284,6 +284,9 @@ def step_config(args, case, P, world, l2_desc):
                      "reshape_and_cache(%d new tokens) + split-context decode with in-kernel merge" % case.B),
             "scales": ("per KV head" if per_head else "per tensor") if case.quantised else None,
             "l2": l2_desc,
+            "timing": ("one CUDA-event pair around the K back-to-back steps; step_ms_rank0 percentiles from a "
+                       "second pass with an event pair per step" if l2_desc.startswith("no flush") else
+                       "an event pair per step, the L2 flush between steps outside the events"),
             "parallelism": "replicas (weak scaling, no collective)" if world > 1 else "single GPU"}
 
 
@@ -391,9 +394,28 @@ def run_ours(args):
         if rc:
             raise SystemExit("library call failed: %d" % rc)
 
-    def timed(body, n_ev, nvtx):
-        """Run `body` for args.steps steps, L2 flushed before each (outside the events);
-        returns the summed event intervals (ms).  Barrier + synchronize on both sides."""
+    def timed(body, n_ev, nvtx, per_step_events=False):
+        """Run `body` for args.steps steps; returns the time of the steps (ms; with n_ev > 2, the
+        summed intervals between consecutive events).  Barrier + synchronize on both sides.
+        Without an L2 flush the steps run back to back between one pair of events, as a decode
+        loop runs them; with a flush (or per_step_events) every step has its own event pair and
+        the flush runs outside them."""
+        if flush.mode == "none" and not per_step_events and n_ev == 2:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            if world > 1:
+                dist.barrier()
+            torch.cuda.synchronize(dev)
+            torch.cuda.nvtx.range_push(nvtx)
+            with torch.cuda.stream(stream):
+                e0.record(stream)
+                for i in range(args.steps):
+                    body(None)
+                e1.record(stream)
+            torch.cuda.synchronize(dev)
+            torch.cuda.nvtx.range_pop()
+            if world > 1:
+                dist.barrier()
+            return [e0.elapsed_time(e1)]
         evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
         if world > 1:
             dist.barrier()
@@ -421,18 +443,22 @@ def run_ours(args):
     sampler = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
     time.sleep(0.3)
     t0 = time.time()
-    # the timed region: K whole steps, each bracketed by two events
+    # the timed region: K whole steps
     step_ms = timed(step, 2, "timed")[0]
-    step_pct = percentiles_ms(per_step)
     t1 = time.time()
+    if flush.mode == "none":                 # per-step spread from a second pass, an event pair per step
+        timed(step, 2, "per_step", per_step_events=True)
+    step_pct = percentiles_ms(per_step)
 
     # each kernel alone over K launches (for the roofline and the per-kernel split); an event
     # pair itself reads about 2.7 us on this GPU, so these per-kernel times are slight overestimates
     def only(fn, args_):
         def body(evs):
-            evs[0].record(stream)
+            if evs:
+                evs[0].record(stream)
             rc = fn(*args_, sp)
-            evs[1].record(stream)
+            if evs:
+                evs[1].record(stream)
             if rc:
                 raise SystemExit("library call failed: %d" % rc)
         return body
@@ -448,9 +474,11 @@ def run_ours(args):
         kc_s, vc_s, cow_dev = kc.clone(), vc.clone(), cow.to(dev)
 
         def copy_body(evs):
-            evs[0].record(stream)
+            if evs:
+                evs[0].record(stream)
             pa.pa_copy_blocks([kc_s], [vc_s], cow_dev, stream=stream)
-            evs[1].record(stream)
+            if evs:
+                evs[1].record(stream)
         copy_ms = timed(copy_body, 2, "kernel_copy_blocks")[0]
         del kc_s, vc_s
     t2 = time.time()
@@ -518,8 +546,10 @@ def run_ours(args):
         "pct_of_nominal_8tbs": round(value / world / 8000.0, 4),
         "kernels_ms_alone": {"reshape_and_cache": round(write_ms / K, 5),
                              "decode (partitions + in-kernel merge)": round(part_ms / K, 5),
-                             "note": "each kernel timed alone over K launches after the timed steps; "
-                                     "an empty CUDA-event pair reads ~2.7 us and is included"},
+                             "note": ("each kernel timed alone over K back-to-back launches after the timed steps, "
+                                      "one CUDA-event pair around them" if flush.mode == "none" else
+                                      "each kernel timed alone over K launches after the timed steps, an event pair "
+                                      "per launch (an empty pair reads ~2.7 us and is included)")},
         "roofline": {"bound": "hbm", "kernel": kernel, "achieved": round(achieved, 1),
                      "peak": peak, "peak_kind": peak_kind + " (hbm_gbs copy bandwidth)", "unit": "GB/s",
                      "frac": round(achieved / peak, 4),
@@ -552,6 +582,7 @@ def run_ours(args):
                                   % flush.mode)}
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(case)
+        line["cpu_baseline_omp"] = cpu_baseline_omp(case)
     if world > 1:
         dist.destroy_process_group()
     return line
@@ -696,10 +727,35 @@ def cpu_baseline(case):
     orc.reshape_and_cache(kn, vn, kc, vc, sl, d=case.d, num_blocks=case.num_blocks, **kw)
     orc.paged_decode(q, kc, vc, tab, ctx, scale=case.scale, **kw)
     dt = time.perf_counter() - t0
-    return {"value": round(kv_bytes(case) / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+    line = {"value": round(kv_bytes(case) / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
             "seconds": round(dt, 2), "host_cpus": os.cpu_count(),
             "sample": "one full step of the workload (cache write of %d tokens + all %d x %d decode rows), "
                       "single-threaded fp64 C" % (case.B, case.B, case.h_q)}
+    return line
+
+
+def cpu_baseline_omp(case):
+    """The same oracle source built with OpenMP (rows shared out over the host's threads), on the
+    same whole step: a second, multi-core reference point."""
+    import numpy as np
+    import torch
+    import oracle
+    import workloads
+    orc = oracle.load(openmp=True)
+    u16 = lambda t: t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+    if case.quantised:
+        case = workloads.make_case(case.name, case.meta["seed"])
+    kc, vc, kw = oracle_step_state(case, orc)
+    q, kn, vn = u16(case.q), u16(case.key_new), u16(case.value_new)
+    tab, ctx, sl = case.block_tables.cpu().numpy(), case.context_lens.cpu().numpy(), case.slot_mapping.cpu().numpy()
+    t0 = time.perf_counter()
+    orc.reshape_and_cache(kn, vn, kc, vc, sl, d=case.d, num_blocks=case.num_blocks, **kw)
+    orc.paged_decode(q, kc, vc, tab, ctx, scale=case.scale, **kw)
+    dt = time.perf_counter() - t0
+    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return {"value": round(kv_bytes(case) / dt / 1e9, 4), "unit": "GB/s", "cores": threads,
+            "kind": "oracle, OpenMP build of the same source", "seconds": round(dt, 3),
+            "sample": "one full step of the workload, the decode rows over %d host threads" % threads}
 
 
 # ---------------------------------------------------------------------------- reference arm

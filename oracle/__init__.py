@@ -32,12 +32,23 @@ _LIB = _HERE / "liboracle.so"
 _c_double_p = ctypes.POINTER(ctypes.c_double)
 
 
-def build(src: Path = _SRC, out: Path = _LIB) -> Path:
-    """Compile the oracle with gcc (IEEE semantics: no fast-math, no FP contraction)."""
+_LIB_OMP = _HERE / "liboracle_omp.so"
+
+
+def build(src: Path = _SRC, out: Path = _LIB, openmp: bool = False) -> Path:
+    """Compile the oracle with gcc (IEEE semantics: no fast-math, no FP contraction).  With
+    `openmp`, the same source built with -fopenmp: the decode's independent rows run on all host
+    threads (the multi-core CPU baseline); the arithmetic of each row is unchanged."""
     cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared",
-           "-o", str(out), str(src), "-lm"]
+           *(["-fopenmp"] if openmp else []), "-o", str(out), str(src), "-lm"]
     subprocess.run(cmd, check=True)
     return out
+
+
+def build_all() -> None:
+    """Both libraries: the single-threaded oracle and its OpenMP build."""
+    build()
+    build(out=_LIB_OMP, openmp=True)
 
 
 def _stale(src: Path, out: Path) -> bool:
@@ -255,12 +266,18 @@ class Oracle:
         return out.reshape(T, h_q, d) if full else out
 
 
-def load(lib_path: os.PathLike | None = None) -> Oracle:
-    """The oracle compiled from oracle.c (built on demand), or a given library."""
+def load(lib_path: os.PathLike | None = None, openmp: bool = False) -> Oracle:
+    """The oracle compiled from oracle.c (built on demand), or a given library.  `openmp`
+    selects the OpenMP build of the same source (multi-core baseline timing only)."""
     if lib_path is None:
-        if _stale(_SRC, _LIB):
-            build()
-        lib_path = _LIB
+        if openmp:
+            if _stale(_SRC, _LIB_OMP):
+                build(out=_LIB_OMP, openmp=True)
+            lib_path = _LIB_OMP
+        else:
+            if _stale(_SRC, _LIB):
+                build()
+            lib_path = _LIB
     key = str(lib_path)
     if key not in _cache:
         _cache[key] = Oracle(Path(lib_path))

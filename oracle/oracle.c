@@ -309,14 +309,22 @@ int or_paged_decode(double *out, const uint16_t *q, const void *k_cache, const v
 {
     if (h_kv <= 0 || h_q % h_kv != 0) return -4;
     if (cache_dtype < 0 || cache_dtype > 2) return -5;
+    /* Rows are independent.  Built with -fopenmp (the second, multi-core baseline library)
+     * they are shared out over the host's threads; built without it the pragma is ignored and
+     * the loop runs in order on one thread.  Either way each row's arithmetic is the same. */
+    int err = 0;
+#pragma omp parallel for collapse(2) schedule(dynamic)
     for (int s = 0; s < B; ++s)
         for (int h = 0; h < h_q; ++h) {
             int rc = decode_one(out + ((size_t)s * h_q + h) * d, s, h, q, k_cache, v_cache,
                                 block_tables, max_blocks_per_seq, context_lens, h_q, h_kv, d, bs,
                                 num_blocks, scale, cache_dtype, k_scales, v_scales);
-            if (rc) return rc;
+            if (rc) {
+#pragma omp atomic write
+                err = rc;
+            }
         }
-    return 0;
+    return err;
 }
 
 /* Selected rows only: pairs[2*i] = sequence, pairs[2*i+1] = query head;
@@ -329,13 +337,18 @@ int or_paged_decode_rows(double *out, const int32_t *pairs, int npairs,
 {
     if (h_kv <= 0 || h_q % h_kv != 0) return -4;
     if (cache_dtype < 0 || cache_dtype > 2) return -5;
+    int err = 0;   /* as in or_paged_decode: rows over threads only in the -fopenmp build */
+#pragma omp parallel for schedule(dynamic)
     for (int i = 0; i < npairs; ++i) {
         int rc = decode_one(out + (size_t)i * d, pairs[2 * i], pairs[2 * i + 1], q, k_cache, v_cache,
                             block_tables, max_blocks_per_seq, context_lens, h_q, h_kv, d, bs,
                             num_blocks, scale, cache_dtype, k_scales, v_scales);
-        if (rc) return rc;
+        if (rc) {
+#pragma omp atomic write
+            err = rc;
+        }
     }
-    return 0;
+    return err;
 }
 
 /* ------------------------------------------------------------------------ */

@@ -62,19 +62,19 @@ CONFIGS = {
                                            h_kv=8, d=128, bs=16, cache="bf16", partition=512,
                                            order="interleaved"),
     "fp8_mha_b32_bs16": dict(B=32, h_q=32, h_kv=32, d=128, bs=16, cache="e4m3", ctx_fixed=4096,
-                             pool_factor=1.0, partition=512),
+                             pool_factor=1.0, partition=1024),
     "fp8_mha_b32_bs32": dict(B=32, h_q=32, h_kv=32, d=128, bs=32, cache="e4m3", ctx_fixed=4096,
-                             pool_factor=1.0, partition=512),
+                             pool_factor=1.0, partition=1024),
     "fp8_mha_b32_bs64": dict(B=32, h_q=32, h_kv=32, d=128, bs=64, cache="e4m3", ctx_fixed=4096,
-                             pool_factor=1.0, partition=512),
+                             pool_factor=1.0, partition=1024),
     "int8_mha_b32_bs16": dict(B=32, h_q=32, h_kv=32, d=128, bs=16, cache="int8", ctx_fixed=4096,
-                              pool_factor=1.0, partition=512),
+                              pool_factor=1.0, partition=1024),
     "int8_mha_b32_bs32": dict(B=32, h_q=32, h_kv=32, d=128, bs=32, cache="int8", ctx_fixed=4096,
-                              pool_factor=1.0, partition=512),
+                              pool_factor=1.0, partition=1024),
     "int8_mha_b32_bs64": dict(B=32, h_q=32, h_kv=32, d=128, bs=64, cache="int8", ctx_fixed=4096,
-                              pool_factor=1.0, partition=512),
+                              pool_factor=1.0, partition=1024),
     "int8_mha_b32_bs16_head": dict(B=32, h_q=32, h_kv=32, d=128, bs=16, cache="int8", ctx_fixed=4096,
-                                   pool_factor=1.0, partition=512, scales="head"),
+                                   pool_factor=1.0, partition=1024, scales="head"),
 }
 
 
