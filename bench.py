@@ -578,8 +578,8 @@ def run_ours(args):
                                "copied back every step, double-buffered on two copy streams so that copies overlap "
                                "the neighbouring steps' decode; timed from the first copy in to the last copy out; "
                                + ("L2: " + flush.desc if flush.mode == "none" else
-                                  "L2 flushed (%s) on the compute stream before every decode, inside the timed loop"
-                                  % flush.mode)}
+                                  "L2 not flushed between steps: the step's %d distinct bytes of K/V stay partly in "
+                                  "L2 (warm)" % distinct_kv_bytes(case))}
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(case)
         line["cpu_baseline_omp"] = cpu_baseline_omp(case)
@@ -595,10 +595,10 @@ def run_e2e(args, pa, L, case, kc, vc, q, k_new, v_new, slots, tables, ctx, mcl,
     buffer, pa_decode_step runs, and `out` is copied back to pinned host memory.  Consecutive
     steps are pipelined: two input buffers and two outputs, the host-to-device copies on one
     stream and the device-to-host copies on another, ordered by events, so that step i+1's
-    inputs arrive and step i-1's output leaves while step i decodes.  When the step's distinct
-    K/V is several times L2 the loop runs without a flush (the `value` rule); otherwise the flush
-    runs on the compute stream before each decode, inside the timed loop.  Returns the time of
-    K steps (first copy in to last copy out)."""
+    inputs arrive and step i-1's output leaves while step i decodes.  The loop never flushes L2
+    (a flush would be work of its own inside the loop); where the step's distinct K/V is smaller
+    than several L2s the line says so.  Returns the time of K steps (first copy in to last copy
+    out)."""
     import torch
     B, h_q, d = case.B, case.h_q, case.d
     parts = [("q", q), ("k_new", k_new), ("v_new", v_new), ("slots", slots), ("tables", tables), ("ctx", ctx)]
@@ -648,9 +648,6 @@ def run_e2e(args, pa, L, case, kc, vc, q, k_new, v_new, slots, tables, ctx, mcl,
             stream.wait_event(ev_in[b])
             if i >= 2:
                 stream.wait_event(ev_out[b])                # step i-2's output has left this buffer
-            if flush.mode != "none":
-                with torch.cuda.stream(stream):
-                    flush()
             kind, a1, a2, _ = sargs[b]
             if kind == "step":
                 rc = L.pa_decode_step(*a1, sp)
