@@ -35,3 +35,19 @@ def test_percentiles_nearest_rank():
     assert bench.percentiles_ms(xs) == {"p10": 10.0, "p50": 50.0, "p90": 90.0}
     assert bench.percentiles_ms([3.0]) == {"p10": 3.0, "p50": 3.0, "p90": 3.0}
     assert bench.percentiles_ms([]) is None
+
+
+def test_nvml_poller_summary_keeps_samples_inside_the_window():
+    """The NVML clock poller reports only samples taken inside the timed region, with the
+    clock-event reasons that were active in any of them (a fake NVML: no GPU here)."""
+    import types
+    import bench
+    p = bench.NvmlPoller.__new__(bench.NvmlPoller)
+    p.ok, p.max_sm = True, 1965
+    p.nv = types.SimpleNamespace(nvmlClocksEventReasonHwSlowdown=0x8, nvmlClocksEventReasonHwThermalSlowdown=0x40,
+                                 nvmlClocksEventReasonSwThermalSlowdown=0x20, nvmlClocksEventReasonSwPowerCap=0x4)
+    p.rows = [(0.5, 1200, 0x8, 300.0), (1.0, 1965, 0x0, 250.0), (1.2, 1965, 0x4, 260.0), (2.5, 900, 0x40, 100.0)]
+    s = p.summary(0.9, 2.0)
+    assert s["samples"] == 2 and s["sm_mhz"] == 1965 and s["reasons"] == ["sw_power_cap"]
+    assert s["power_w_max"] == 260.0 and s["sm_max_mhz"] == 1965
+    assert p.summary(3.0, 4.0) is None
