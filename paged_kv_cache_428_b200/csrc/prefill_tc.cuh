@@ -112,7 +112,7 @@ struct PrefillTcConfig {
     static constexpr int OFF_K = NQ * Q_BYTES;
     static constexpr int OFF_V = OFF_K + KST * KV_TILE;
     static constexpr int OFF_BARS = OFF_V + VST * KV_TILE;
-    static constexpr int NBARS = 2 * KST + 2 * VST + NQ * 7; // k, v full/empty; per tile s full, s free, p full x2, o done x2, drain
+    static constexpr int NBARS = 2 * KST + 2 * VST + NQ * 8; // k, v full/empty; per tile s full, s free, p full x2, o done x2, drain, q full
     static constexpr int OFF_MISC = OFF_BARS + NBARS * 8; // tensor-memory base, abort flag
     static constexpr int SMEM = OFF_MISC + 16 + 1024;
     static constexpr int TMEM_PER_Q = 256;                // S [0,64), P0 [64,96), P1 [96,128), O [128, 128 + D)
@@ -145,6 +145,7 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
     // per query tile q and buffer b: index 2 q + b
     uint64_t *s_full = bars + 2 * KST + 2 * VST, *s_free = s_full + NQ, *p_full = s_free + NQ, *o_done = p_full + 2 * NQ;
     uint64_t *drain = o_done + 2 * NQ;                          // one per query tile
+    uint64_t *q_full = drain + NQ;                              // one per query tile: Q in shared memory
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
 
@@ -191,26 +192,13 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
             mbar_init(&o_done[b], 1);
         }
         for (int q = 0; q < NQ; ++q) mbar_init(&drain[q], 1);
+        for (int q = 0; q < NQ; ++q) mbar_init(&q_full[q], 128);
         *abort_flag = 0;
         mbar_init_fence();
     }
     if (warp == C::MMA_WARP) {
         tmem_alloc(tmem_slot, C::TMEM_COLS);
         tmem_relinquish();
-    }
-    if (warp < 4 * NQ) {
-        // Q rows of query tile q into its swizzled shared tile (row t = token t / G, head t % G)
-        const int q = warp >> 2, t = threadIdx.x & 127;
-        const int tok = tok0_of(q) + t / G;
-        const bool ok = tok < chunk;
-        const uint4 *src = reinterpret_cast<const uint4 *>(
-            p.q + ((size_t)(q0 + (ok ? tok : 0)) * p.h_q + (size_t)kvh * G + t % G) * D);
-#pragma unroll
-        for (int c = 0; c < D / 8; ++c) {
-            const uint4 v = ok ? src[c] : make_uint4(0u, 0u, 0u, 0u);
-            *reinterpret_cast<uint4 *>(smem + C::OFF_Q + q * C::Q_BYTES + (c >> 3) * C::Q_HALF + swz128(t, c & 7)) = v;
-        }
-        fence_proxy_async_smem();
     }
     tc_fence_before_sync();
     __syncthreads();
@@ -317,7 +305,11 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
                 return true;
             };
             bool ok = true;
-            if (nkq > 0) ok = s_mma(0);
+            if (nkq > 0) {
+                // the tile's Q rows, written by its softmax warpgroup after the CTA barrier
+                ok = mbar_wait_or_abort(&q_full[q], 0, abort_flag) && !*abort_flag;
+                if (ok) ok = s_mma(0);
+            }
             for (int j = 0; j < nkq && ok; ++j) {
                 if (j + 1 < nkq) ok = s_mma(j + 1);
                 if (ok) ok = pv(j);
@@ -343,6 +335,22 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
         const int tok0 = tok0_of(q), nkv_q = nkv_of(q);
         const int tok = tok0 + t / G;
         const bool row_ok = tok < chunk;
+        {
+            // this thread's Q row into the tile's swizzled shared tile (row t = token t / G, head
+            // t % G), after the CTA barrier so that the loads overlap the producers' first K/V
+            // copies; the MMA warp waits for all 128 rows on q_full before the tile's first S
+            const uint4 *src = reinterpret_cast<const uint4 *>(
+                p.q + ((size_t)(q0 + (row_ok ? tok : 0)) * p.h_q + (size_t)kvh * G + t % G) * D);
+            uint4 v[D / 8];
+#pragma unroll
+            for (int c = 0; c < D / 8; ++c) v[c] = row_ok ? src[c] : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+            for (int c = 0; c < D / 8; ++c)
+                *reinterpret_cast<uint4 *>(smem + C::OFF_Q + q * C::Q_BYTES + (c >> 3) * C::Q_HALF + swz128(t, c & 7)) =
+                    v[c];
+            fence_proxy_async_smem();
+            mbar_arrive(&q_full[q]);
+        }
         const int pos = row_ok ? ctx - chunk + tok : 0;
         const int first_pos = ctx - chunk + tok0;
         const uint32_t lane_tm = tmem + q * C::TMEM_PER_Q + ((uint32_t)(32 * (warp & 3)) << 16);

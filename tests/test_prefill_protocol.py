@@ -7,7 +7,8 @@ Roles, as the kernel runs them for one CTA (two 128-row query tiles q = 0, 1):
     and p_full phase j >> 1 of buffer j & 1; completions arrive on s_full / k_empty and o_done /
     v_empty in issue order (tcgen05.commit); past its KV range the thread releases each K and V
     slot as its data lands;
-  * four softmax warps per query tile: wait s_full phase j, load S_j, arrive s_free; sometimes
+  * four softmax warps per query tile: first write the tile's Q rows to shared memory and
+    arrive q_full (the MMA thread waits for it before S_0); then wait s_full phase j, load S_j, arrive s_free; sometimes
     rescale O (wait o_done of P V_{j-1}); on the context's last tile wait V_j (zeroing rows);
     before storing P_j wait o_done of P V_{j-2}; arrive p_full; at the end wait o_done of the
     last P V and read O.
@@ -67,9 +68,11 @@ def run(nkv_q, KST, VST, seed, ctx_last_tile=True, rescale_p=0.2, abort_p=0.0, b
     s_free = [Bar(4) for _ in range(NQ)]
     p_full = [Bar(4) for _ in range(2 * NQ)]
     o_done = [Bar(1) for _ in range(2 * NQ)]
+    q_full = [Bar(4) for _ in range(NQ)]
     # data state
     kslot, vslot = [None] * KST, [None] * VST              # tile whose data sits in the slot
     kread, vread = [set() for _ in range(KST)], [set() for _ in range(VST)]   # pending MMA readers
+    qrows = [set() for _ in range(NQ)]                     # softmax warps whose Q rows are written
     sbuf = [None] * NQ                                     # tile of the completed S product
     s_pending = [False] * NQ                               # an S product is writing S
     sloaded = [[-1] * 4 for _ in range(NQ)]                # last S tile each softmax warp loaded
@@ -118,6 +121,7 @@ def run(nkv_q, KST, VST, seed, ctx_last_tile=True, rescale_p=0.2, abort_p=0.0, b
                 if not (yield (s_free[q], j - 1, True)) or abort[0]:
                     return False
                 check(all(x == j - 1 for x in sloaded[q]), "S_%d issued before every warp loaded S_%d" % (j, j - 1))
+            check(len(qrows[q]) == 4, "S_%d reads Q before every warp wrote its rows" % j)
             check(kslot[st] == j, "S_%d reads slot %d holding %s" % (j, st, kslot[st]))
             kread[st].add((q, j))
             s_pending[q] = True
@@ -154,7 +158,9 @@ def run(nkv_q, KST, VST, seed, ctx_last_tile=True, rescale_p=0.2, abort_p=0.0, b
 
         ok = True
         if nkq > 0:
-            ok = yield from s_mma(0)
+            ok = (yield (q_full[q], 0, True)) and not abort[0]
+            if ok:
+                ok = yield from s_mma(0)
         for j in range(nkq):
             if not ok:
                 break
@@ -178,6 +184,8 @@ def run(nkv_q, KST, VST, seed, ctx_last_tile=True, rescale_p=0.2, abort_p=0.0, b
 
     def softmax(q, w):
         n = nkv_q[q]
+        qrows[q].add(w)
+        q_full[q].arrive()
         for j in range(n):
             if not (yield (s_full[q], j, True)) or abort[0]:
                 return
@@ -258,7 +266,7 @@ def run(nkv_q, KST, VST, seed, ctx_last_tile=True, rescale_p=0.2, abort_p=0.0, b
             if not any(step(r) for r in sorted(alive)) and alive:
                 raise Violation("deadlock: %d roles blocked" % len(alive))
     if not abort[0]:
-        for b in k_empty + v_empty + s_free + p_full:
+        for b in k_empty + v_empty + s_free + p_full + q_full:
             check(b.pending == b.count, "a barrier was left with partial arrivals")
     return True
 
@@ -311,6 +319,8 @@ def _mutant(old, new):
      "yield (o_done[2 * q + (j & 1)], max(j - 2, 0) >> 1, True)"),
     # a K slot is released after one query tile's S instead of both
     ("k_empty = [Bar(NQ) for _ in range(KST)]", "k_empty = [Bar(1) for _ in range(KST)]"),
+    # S_0 issued without waiting for the softmax warps' Q rows
+    ("            ok = (yield (q_full[q], 0, True)) and not abort[0]\n", "            ok = True\n"),
     # S_{j+1} issued without waiting for the softmax to have loaded S_j
     ("            if j >= 1:\n                if not (yield (s_free[q], j - 1, True)) or abort[0]:\n                    return False\n",
      "            if False:\n                pass\n"),
