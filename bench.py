@@ -54,6 +54,9 @@ def parse_args(argv=None):
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prefill-schedule", choices=("queue", "grid"), default="queue",
+                    help="prefill workloads: pa_prefill_ws (one CTA per SM claiming work items) or "
+                         "pa_prefill (one CTA per work item)")
     ap.add_argument("--l2", choices=["auto", "write", "write+read", "none"], default="auto",
                     help="between timed steps: write a 2x L2 buffer (write), then also read a second one so the "
                          "flush's dirty lines are written back before the step (write+read), or nothing (none, "
@@ -887,11 +890,12 @@ def measured_bf16_peak():
     return 1590.0, "fallback"
 
 
-def prefill_kernel_name() -> str:
-    """The prefill kernel pa_prefill dispatches to (PA_PREFILL_MMA_SYNC=1 selects the mma.sync one)."""
+def prefill_kernel_name(schedule: str) -> str:
+    """The prefill kernel the call dispatches to (PA_PREFILL_MMA_SYNC=1 selects the mma.sync one)."""
     if os.environ.get("PA_PREFILL_MMA_SYNC") == "1":
         return "paged_prefill_kernel (mma.sync bf16)"
-    return "paged_prefill_tc_kernel (tcgen05.mma bf16, fp32 accumulators in tensor memory)"
+    how = "one CTA per SM claiming work items" if schedule == "queue" else "one CTA per work item"
+    return "paged_prefill_tc_kernel (tcgen05.mma bf16, fp32 accumulators in tensor memory; %s)" % how
 
 
 def run_prefill(args):
@@ -938,7 +942,12 @@ def run_prefill(args):
         return sum(per_step)
 
     per_step = []
-    step = [(L.pa_reshape_and_cache, rargs), (L.pa_prefill, pargs)]
+    if args.prefill_schedule == "queue":
+        ws = pa.make_prefill_workspace(dev)
+        pcall = (L.pa_prefill_ws, pargs + (ws.data_ptr(), ws.numel()))
+    else:
+        pcall = (L.pa_prefill, pargs)
+    step = [(L.pa_reshape_and_cache, rargs), pcall]
     timed(step, args.warmup)
     uuid = str(torch.cuda.get_device_properties(dev).uuid)
     sampler = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
@@ -948,7 +957,7 @@ def run_prefill(args):
     step_ms = timed(step, args.steps)
     step_pct = percentiles_ms(per_step)
     t1 = time.time()
-    kern_ms = timed([(L.pa_prefill, pargs)], args.steps)
+    kern_ms = timed([pcall], args.steps)
     t2 = time.time()
     time.sleep(0.1)
     sampler.stop()
@@ -976,12 +985,13 @@ def run_prefill(args):
                    "head_dim": case.d, "block_size": case.bs, "chunk_tokens": int(T),
                    "cached_tokens": case.meta["cached"], "chunk_lens": case.meta["chunk"],
                    "attention_flops_per_step": int(flops),
-                   "step": "reshape_and_cache(all chunk tokens) + pa_prefill",
+                   "step": "reshape_and_cache(all chunk tokens) + %s" % pcall[0].__name__,
+                   "schedule": args.prefill_schedule,
                    "l2": flush.desc},
         "tokens_per_s": round(tot_tok / (step_ms / 1e3 / K), 1),
         "step_ms_rank0": step_pct,
         "kernels_ms_alone": {"prefill": round(kern_ms / K, 5)},
-        "roofline": {"bound": "tensor", "kernel": prefill_kernel_name(), "achieved": round(achieved, 1),
+        "roofline": {"bound": "tensor", "kernel": prefill_kernel_name(args.prefill_schedule), "achieved": round(achieved, 1),
                      "peak": peak, "peak_kind": kind, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                      "traffic": None, "algorithmic_flops_per_launch": int(flops)},
         "gpu_launches": 2 * K,

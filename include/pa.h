@@ -249,11 +249,32 @@ int pa_decode_step(const void *key, const void *value, int64_t key_stride, int64
  * an mma.sync kernel instead); accuracy as pa_decode for bf16 caches (a quarter of the
  * softmax exponentials use a cubic with relative error < 1e-4, and terms below 2^-125 of the
  * row's running maximum come out as about that instead of 0).  Allocates nothing; needs no
- * workspace. */
+ * workspace.  One CTA per work item (a pair of 128-row query tiles of one sequence and KV
+ * head); pa_prefill_ws computes the same result with fewer, longer-lived CTAs. */
 int pa_prefill(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
                int max_blocks_per_seq, const int32_t *query_start, const int32_t *context_lens, int num_seqs,
                int max_query_len, int h_q, int h_kv, int head_dim, int block_size, int num_blocks, float scale,
                int cache_dtype, void *stream);
+
+/* Bytes of device workspace pa_prefill_ws needs (a constant: two int counters, padded). */
+size_t pa_prefill_workspace_size(void);
+
+/* pa_prefill with a work queue: the same arguments, result and errors, plus
+ *   workspace        device memory of at least pa_prefill_workspace_size() bytes, 16-byte
+ *                    aligned, all zero before the first call (e.g. cudaMemset once after
+ *                    allocating it); every call leaves it zero again.  Calls that share a
+ *                    workspace must not run at the same time (put them on one stream);
+ *   workspace_bytes  its size; NULL, too small or misaligned: PA_ERR_WORKSPACE, checked
+ *                    before anything else, nothing launched.
+ * The grid is one CTA per SM; each CTA claims work items from the counter in the workspace,
+ * sequences in order of context length, longest first (for up to 1024 sequences; beyond that
+ * in sequence order), and prepares the next item (block-table reads, K/V and Q copies) while it
+ * finishes the current one.  The caller's memory is not allocated, freed or resized. With
+ * PA_PREFILL_MMA_SYNC=1 the mma.sync kernel runs, which does not use the workspace. */
+int pa_prefill_ws(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
+                  int max_blocks_per_seq, const int32_t *query_start, const int32_t *context_lens, int num_seqs,
+                  int max_query_len, int h_q, int h_kv, int head_dim, int block_size, int num_blocks, float scale,
+                  int cache_dtype, void *workspace, size_t workspace_bytes, void *stream);
 
 /* ---- decode without any allocation (static scratch) ---------------------------
  * The pages have no counterpart for this call; it exists for callers that cannot

@@ -80,6 +80,9 @@ def _load() -> ctypes.CDLL:
         "pa_decode_step": (i32, [vp, vp, i64, i64, vp, vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32, i32, i32,
                                  f32, i32, f32, f32, i32, vp, sz, vp]),
         "pa_prefill": (i32, [vp, vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, i32, i32, i32, f32, i32, vp]),
+        "pa_prefill_workspace_size": (sz, []),
+        "pa_prefill_ws": (i32, [vp, vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, i32, i32, i32, f32, i32, vp, sz,
+                                vp]),
         "pa_device_errors": (i32, [ctypes.POINTER(ctypes.c_uint), i32]),
         "pa_validate_block_tables": (i32, [vp, i32, vp, i32, i32, i32]),
         "pa_validate_slots": (i32, [vp, i32, i32, i32]),
@@ -394,6 +397,25 @@ def pa_prefill(out, q, k_cache, v_cache, block_tables, query_start, context_lens
     """Causal attention of each sequence's chunk of query rows over the paged cache; returns out."""
     args = prefill_call_args(out, q, k_cache, v_cache, block_tables, query_start, context_lens, max_query_len, scale)
     _check(_lib.pa_prefill(*args, _stream_ptr(stream)), "pa_prefill")
+    return out
+
+
+def pa_prefill_workspace_size() -> int:
+    return int(_lib.pa_prefill_workspace_size())
+
+
+def make_prefill_workspace(device="cuda") -> torch.Tensor:
+    """A zero-filled workspace for pa_prefill_ws (each call leaves it zero again).  Calls that
+    share one must not run at the same time."""
+    return torch.zeros(pa_prefill_workspace_size(), dtype=torch.uint8, device=device)
+
+
+def pa_prefill_ws(out, q, k_cache, v_cache, block_tables, query_start, context_lens, max_query_len: int,
+                  workspace: torch.Tensor, scale: float = None, stream=None) -> torch.Tensor:
+    """pa_prefill on the work-queue schedule (one CTA per SM claiming work items); returns out."""
+    args = prefill_call_args(out, q, k_cache, v_cache, block_tables, query_start, context_lens, max_query_len, scale)
+    _need(workspace, "workspace", (torch.uint8,), 1)
+    _check(_lib.pa_prefill_ws(*args, workspace.data_ptr(), workspace.numel(), _stream_ptr(stream)), "pa_prefill_ws")
     return out
 
 

@@ -1,6 +1,7 @@
 // pa_lib.cu -- C-ABI entry points of the device calls (argument checks, dispatch, launch).
 // All device code of the library is in this one translation unit.
 #include <algorithm>
+#include <climits>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
@@ -26,6 +27,9 @@ namespace {
 constexpr float kLog2e = 1.4426950408889634f;
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// pa_prefill_ws: the claim counter and the finished-CTA counter, padded
+constexpr size_t kPrefillWorkspaceBytes = 256;
 
 int launch_status()
 {
@@ -733,7 +737,7 @@ int launch_prefill(const PrefillParams &pp, int num_seqs, int max_query_len, cud
 }
 
 template <int D, int BS, int G>
-int launch_prefill_tc(const PrefillParams &pp, int num_seqs, int max_query_len, cudaStream_t st)
+int launch_prefill_tc(const PrefillParams &pp, int num_seqs, int max_query_len, int *counters, cudaStream_t st)
 {
     using C = PrefillTcConfig<D, BS, G>;
     static std::atomic<unsigned long long> smem_set{0};
@@ -751,8 +755,20 @@ int launch_prefill_tc(const PrefillParams &pp, int num_seqs, int max_query_len, 
     if (rc == PA_OK) rc = cached_cache_map(&mv, pp.v_cache, pp.num_blocks, pp.h_kv, BS, D);
     if (rc != PA_OK) return rc;
     const int pairs = (prefill_tiles<C::TQ>(max_query_len) + C::NQ - 1) / C::NQ;
-    const dim3 grid(pairs, pp.h_kv, num_seqs);
-    paged_prefill_tc_kernel<D, BS, G><<<grid, C::THREADS, C::SMEM, st>>>(pp, mk, mv);
+    const long long items = (long long)pairs * pp.h_kv * num_seqs;
+    if (items > INT_MAX) return PA_ERR_UNSUPPORTED;
+    PrefillSched sc{};
+    sc.counters = counters;
+    sc.num_seqs = num_seqs;
+    sc.pairs_max = pairs;
+    sc.total_items = (int)items;
+    dim3 grid(pairs, pp.h_kv, num_seqs);                      // one CTA per item
+    if (counters) {
+        const int sms = sm_count();                              // one CTA per SM, claiming items
+        if (sms <= 0) return PA_ERR_CUDA;
+        grid = dim3((unsigned)std::min<long long>(sms, items));
+    }
+    paged_prefill_tc_kernel<D, BS, G><<<grid, C::THREADS, C::SMEM, st>>>(pp, sc, mk, mv);
     return launch_status();
 }
 
@@ -764,25 +780,25 @@ bool prefill_on_mma_sync()
 }
 
 template <int D, int BS>
-int dispatch_prefill_group(int g, const PrefillParams &pp, int n, int mql, cudaStream_t st)
+int dispatch_prefill_group(int g, const PrefillParams &pp, int n, int mql, int *counters, cudaStream_t st)
 {
     return switch_group(g, [&](auto gc) {
         constexpr int G = decltype(gc)::value;
         if (prefill_on_mma_sync()) return launch_prefill<D, BS, G>(pp, n, mql, st);
-        return launch_prefill_tc<D, BS, G>(pp, n, mql, st);
+        return launch_prefill_tc<D, BS, G>(pp, n, mql, counters, st);
     });
 }
 
-int dispatch_prefill(int d, int bs, int g, const PrefillParams &pp, int n, int mql, cudaStream_t st)
+int dispatch_prefill(int d, int bs, int g, const PrefillParams &pp, int n, int mql, int *counters, cudaStream_t st)
 {
     if (d == 64) {
-        if (bs == 16) return dispatch_prefill_group<64, 16>(g, pp, n, mql, st);
-        if (bs == 32) return dispatch_prefill_group<64, 32>(g, pp, n, mql, st);
-        if (bs == 64) return dispatch_prefill_group<64, 64>(g, pp, n, mql, st);
+        if (bs == 16) return dispatch_prefill_group<64, 16>(g, pp, n, mql, counters, st);
+        if (bs == 32) return dispatch_prefill_group<64, 32>(g, pp, n, mql, counters, st);
+        if (bs == 64) return dispatch_prefill_group<64, 64>(g, pp, n, mql, counters, st);
     } else if (d == 128) {
-        if (bs == 16) return dispatch_prefill_group<128, 16>(g, pp, n, mql, st);
-        if (bs == 32) return dispatch_prefill_group<128, 32>(g, pp, n, mql, st);
-        if (bs == 64) return dispatch_prefill_group<128, 64>(g, pp, n, mql, st);
+        if (bs == 16) return dispatch_prefill_group<128, 16>(g, pp, n, mql, counters, st);
+        if (bs == 32) return dispatch_prefill_group<128, 32>(g, pp, n, mql, counters, st);
+        if (bs == 64) return dispatch_prefill_group<128, 64>(g, pp, n, mql, counters, st);
     }
     return PA_ERR_UNSUPPORTED;
 }
@@ -1034,10 +1050,11 @@ int pa_reshape_and_cache_head_scales(const void *key, const void *value, int64_t
                         head_dim, block_size, num_blocks, cache_dtype, 1.f, 1.f, k_scales, v_scales, stream);
 }
 
-int pa_prefill(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
-               int max_blocks_per_seq, const int32_t *query_start, const int32_t *context_lens, int num_seqs,
-               int max_query_len, int h_q, int h_kv, int head_dim, int block_size, int num_blocks, float scale,
-               int cache_dtype, void *stream)
+namespace {
+int prefill_impl(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
+                 int max_blocks_per_seq, const int32_t *query_start, const int32_t *context_lens, int num_seqs,
+                 int max_query_len, int h_q, int h_kv, int head_dim, int block_size, int num_blocks, float scale,
+                 int cache_dtype, int *counters, void *stream)
 {
     if (num_seqs < 0 || max_query_len < 0 || h_q <= 0 || h_kv <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0)
         return PA_ERR_INVALID_ARG;
@@ -1065,9 +1082,35 @@ int pa_prefill(void *out, const void *q, const void *k_cache, const void *v_cach
     pp.h_kv = h_kv;
     pp.num_blocks = num_blocks;
     pp.qk_scale = scale * kLog2e;
-    return dispatch_prefill(head_dim, block_size, h_q / h_kv, pp, num_seqs, max_query_len,
+    return dispatch_prefill(head_dim, block_size, h_q / h_kv, pp, num_seqs, max_query_len, counters,
                             static_cast<cudaStream_t>(stream));
 }
+}  // namespace
+
+int pa_prefill(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
+               int max_blocks_per_seq, const int32_t *query_start, const int32_t *context_lens, int num_seqs,
+               int max_query_len, int h_q, int h_kv, int head_dim, int block_size, int num_blocks, float scale,
+               int cache_dtype, void *stream)
+{
+    return prefill_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, query_start, context_lens,
+                        num_seqs, max_query_len, h_q, h_kv, head_dim, block_size, num_blocks, scale, cache_dtype,
+                        nullptr, stream);
+}
+
+size_t pa_prefill_workspace_size(void) { return kPrefillWorkspaceBytes; }
+
+int pa_prefill_ws(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
+                  int max_blocks_per_seq, const int32_t *query_start, const int32_t *context_lens, int num_seqs,
+                  int max_query_len, int h_q, int h_kv, int head_dim, int block_size, int num_blocks, float scale,
+                  int cache_dtype, void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (workspace == nullptr || workspace_bytes < kPrefillWorkspaceBytes || !aligned16(workspace))
+        return PA_ERR_WORKSPACE;
+    return prefill_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, query_start, context_lens,
+                        num_seqs, max_query_len, h_q, h_kv, head_dim, block_size, num_blocks, scale, cache_dtype,
+                        static_cast<int *>(workspace), stream);
+}
+
 
 int pa_copy_blocks(void *const *k_caches, void *const *v_caches, int num_layers, const int64_t *block_pairs,
                    int num_pairs, size_t block_bytes, int num_blocks, void *stream)

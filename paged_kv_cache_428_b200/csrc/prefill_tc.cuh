@@ -1,35 +1,50 @@
 // prefill_tc.cuh -- chunked-prefill attention over the paged bf16 KV cache on the
 // 5th-generation tensor cores (tcgen05.mma, accumulators in tensor memory).
 //
-// Same computation and masking rules as paged_prefill_kernel (prefill.cuh).  One CTA per (pair
-// of query tiles, KV head, sequence); a query tile is 128 rows = 128 / G tokens x the G heads of
-// the KV head, and both tiles of a CTA share every K/V tile it streams.  Tensor memory per query
-// tile (256 of the 512 columns): S [0,64) fp32, P0 / P1 [64,128) bf16 pairs, O [128,128+D) fp32.
+// Same computation and masking rules as paged_prefill_kernel (prefill.cuh).  A work item is
+// (pair of query tiles, KV head, sequence); a query tile is 128 rows = 128 / G tokens x the G
+// heads of the KV head, and both tiles of an item share every K/V tile it streams.  Tensor
+// memory per query tile (256 of the 512 columns): S [0,64) fp32, P0 / P1 [64,128) bf16 pairs,
+// O [128,128+D) fp32.
+//
+// Scheduling.  With a claim counter (pa_prefill_ws) the grid is one CTA per SM and every CTA
+// claims items one after another from a global atomic counter, sequences in order of context
+// length, longest first, and the items of one (sequence, KV head) next to each other so that
+// CTAs running at the same time share their K/V tiles through L2.  Without one (pa_prefill) the
+// grid has one CTA per item.  In both cases the next item is known before the current one ends:
+// the producers start its block-table reads and K/V copies while the current item's last tiles
+// are in use, and its Q tiles are copied as soon as the current item's last S products are done,
+// so an item costs its KV tiles plus a short epilogue instead of a chain of dependent loads.
+//
 // Roles:
 //   warps 0-7  two softmax warpgroups, one per query tile: thread t of a warpgroup owns row t of
 //              its tile (= tensor-memory lane t).  It loads its row of S_j from tensor memory
 //              (which frees S for S_{j+1}), applies the causal / context mask, keeps the running
 //              max and sum (log2 domain; a quarter of the exponentials by a polynomial on
 //              the FMA pipe, beside the MUFU unit), stores its row of P_j (bf16) into tensor memory,
-//              rescales its row of O when its max moved, and finally normalises O and writes the
-//              output row.
+//              rescales its row of O when its max moved, and at the end of the item normalises O
+//              and writes the output row.
 //   warps 8-9  one MMA warp per query tile: lane 0 issues S_{j+1} = Q K_{j+1}^T (M 128, N 64,
 //              K = D, both operands in shared memory) as soon as the softmax has loaded S_j, and
 //              O += P_j V_j (M 128, N = D, K 64) with P read from tensor memory and V read N-major
 //              from shared memory; tcgen05.commit signals each step.  With one issuing thread per
 //              tile, one tile's barrier waits overlap the other tile's MMAs on the tensor core.
-//              Warp 8 also allocates the 512 tensor-memory columns.
+//              Warp 8 also allocates the 512 tensor-memory columns, once per CTA.
 //   warps 10-11 K and V producers: 2-D TMA copies per physical block (the decode tensor maps,
 //              128-byte swizzle), so the tiles are the MMA operands as they land.  Each warp
 //              reads the block table 32 entries at a time, the next 32 in flight meanwhile, and
-//              its lanes issue the copies of one tile.  K and V have rings of their own; a slot
-//              is free when both query tiles have released it (their MMAs that read it finished,
-//              or the tile's KV range ended before it).
-// Q is copied into a swizzled shared tile once.  V rows past the context are zeroed in shared
-// memory before the P V step (an unwritten NaN slot times a zero probability would poison O).
-// Every wait is bounded and also ends when another role has stopped the CTA; on a timeout or a
-// bad block the CTA records the error, stops, waits for its copies and MMAs in flight and frees
-// its tensor memory; its rows come out NaN.
+//              its lanes issue the copies of one tile.  K and V have rings of their own, indexed
+//              across items; a slot is free when both query tiles have released it (their MMAs
+//              that read it finished, or the tile's KV range ended before it).  V rows past the
+//              context in an item's last tile are zeroed by the V producer once the copy has
+//              landed and before the tile is marked full (an unwritten NaN slot times a zero
+//              probability would poison O).
+//   warp 12    scheduler: claims items, publishes each through a two-entry ring in shared memory,
+//              and copies each item's Q rows (cp.async, zero-filled past the chunk) into the
+//              swizzled Q tiles once the previous item's S products no longer read them.
+// Every wait on the data path is bounded and also ends when another role has stopped the CTA; on
+// a timeout or a bad block the CTA records the error, stops claiming, writes NaN into the rows
+// of the items it holds, waits for its copies and MMAs in flight and frees its tensor memory.
 #pragma once
 
 #include "prefill.cuh"
@@ -92,11 +107,51 @@ __device__ __forceinline__ float max3f(float a, float b, float c)
     return r;
 }
 
+
+// 16-byte cp.async into shared memory; zero-fill instead of reading when !ok.
+__device__ __forceinline__ void cp_async_16_zfill(void *dst, const void *src, bool ok)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)), "l"(src), "r"(ok ? 16 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// Non-blocking test of an mbarrier phase (test_wait never suspends the thread).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity)
+{
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// Sequence tables (query_start, context_lens) and the claim order are kept in shared memory for
+// up to this many sequences; beyond it the scheduler reads them from global memory and claims in
+// sequence order.
+constexpr int kPrefillSeqsInSmem = 1024;
+
+// Work distribution of one launch.
+struct PrefillSched {
+    int *counters;      // device [2]: next item to claim, CTAs finished (zero between launches);
+                        // nullptr: one CTA per item, item = blockIdx
+    int num_seqs;
+    int pairs_max;      // query-tile pairs of the longest chunk = items per (sequence, KV head)
+    int total_items;    // num_seqs * h_kv * pairs_max
+};
+
 template <int D, int BS, int G, int NQ_ = 2, int KST_ = 4, int VST_ = 4>
 struct PrefillTcConfig {
-    static constexpr int NQ = NQ_;                        // 128-row query tiles per CTA
-    static constexpr int THREADS = 128 * NQ + 32 * NQ + 64; // softmax warpgroups, one MMA warp per query tile, K and V TMA warps
+    static constexpr int NQ = NQ_;                        // 128-row query tiles per item
+    // softmax warpgroups, one MMA warp per query tile, K and V TMA warps (the K warp also claims
+    // and publishes the work items)
+    static constexpr int THREADS = 128 * NQ + 32 * NQ + 64;
     static constexpr int MMA_WARP = 4 * NQ, TMA_WARP = 5 * NQ;
+    static constexpr int ITEM_READERS = 4 * NQ + NQ + 1;  // warps that read each published item
     static constexpr int BM = 128;                        // rows per query tile = tensor-memory lanes
     static constexpr int TQ = BM / G;                     // query tokens per query tile
     static constexpr int BN = 64;                         // KV tokens per tile
@@ -112,9 +167,13 @@ struct PrefillTcConfig {
     static constexpr int OFF_K = NQ * Q_BYTES;
     static constexpr int OFF_V = OFF_K + KST * KV_TILE;
     static constexpr int OFF_BARS = OFF_V + VST * KV_TILE;
-    static constexpr int NBARS = 2 * KST + 2 * VST + NQ * 8; // k, v full/empty; per tile s full, s free, p full x2, o done x2, drain, q full
-    static constexpr int OFF_MISC = OFF_BARS + NBARS * 8; // tensor-memory base, abort flag
-    static constexpr int SMEM = OFF_MISC + 16 + 1024;
+    // k, v full/empty; per tile: s full, s free, p full x2, o done x2, drain, q full; item ring
+    // full x2 / empty x2; the V tail copy
+    static constexpr int NBARS = 2 * KST + 2 * VST + NQ * 8 + 5;
+    static constexpr int OFF_ITEMS = OFF_BARS + NBARS * 8;   // item ring: 2 x 8 ints
+    static constexpr int OFF_MISC = OFF_ITEMS + 64;       // tensor-memory base, abort flag
+    static constexpr int OFF_SEQ = OFF_MISC + 16;         // query_start, context_lens, claim order
+    static constexpr int SMEM = OFF_SEQ + (3 * kPrefillSeqsInSmem + 1) * 4 + 1024;
     static constexpr int TMEM_PER_Q = 256;                // S [0,64), P0 [64,96), P1 [96,128), O [128, 128 + D)
     static constexpr int COL_P = 64;
     static constexpr int POLY_PAIRS = 2;                  // of every 8 pairs of P, on the FMA pipe
@@ -129,9 +188,13 @@ struct PrefillTcConfig {
     static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
+// Item layout in the ring: seq (< 0: no more items), KV head, pair, first query row, chunk
+// length, context length, KV tiles of query tile 0 and of query tile 1.
+enum { IT_SEQ, IT_KVH, IT_PAIR, IT_Q0, IT_CHUNK, IT_CTX, IT_NKV0, IT_NKV1, IT_N };
+
 template <int D, int BS, int G, int NQ_ = 2, int KST_ = 4, int VST_ = 4>
 __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::THREADS, 1)
-    paged_prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmap_k,
+    paged_prefill_tc_kernel(const PrefillParams p, const PrefillSched sc, const __grid_constant__ CUtensorMap tmap_k,
                             const __grid_constant__ CUtensorMap tmap_v)
 {
     using C = PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>;
@@ -145,34 +208,17 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
     // per query tile q and buffer b: index 2 q + b
     uint64_t *s_full = bars + 2 * KST + 2 * VST, *s_free = s_full + NQ, *p_full = s_free + NQ, *o_done = p_full + 2 * NQ;
     uint64_t *drain = o_done + 2 * NQ;                          // one per query tile
-    uint64_t *q_full = drain + NQ;                              // one per query tile: Q in shared memory
+    uint64_t *q_full = drain + NQ;                              // one per query tile: Q copied
+    uint64_t *item_full = q_full + NQ, *item_empty = item_full + 2, *v_tail = item_empty + 2;
+    volatile int *items = reinterpret_cast<volatile int *>(smem + C::OFF_ITEMS);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
+    int *seq_qs = reinterpret_cast<int *>(smem + C::OFF_SEQ);
+    int *seq_ctx = seq_qs + kPrefillSeqsInSmem + 1, *seq_order = seq_ctx + kPrefillSeqsInSmem;
 
-    const int kvh = blockIdx.y, seq = blockIdx.z;
-    const int q0 = p.query_start[seq], q1 = p.query_start[seq + 1];
-    const int chunk = q1 - q0;
-    const int ctx = p.context_lens[seq];
-    const int ntiles = prefill_tiles<C::TQ>(chunk);
-    const int npairs = (ntiles + NQ - 1) / NQ;
-    const int pair = npairs - 1 - (int)blockIdx.x;             // longest KV ranges first
-    if (chunk > ctx) {                                         // rows left unwritten, flagged
-        if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0) record_error(PA_DEVERR_BAD_CHUNK);
-        return;
-    }
-    if (pair < 0 || chunk <= 0) return;                        // uniform over the CTA
-    // query tile q of this CTA: tokens [tok0(q), tok_end(q)); it reads KV tiles 0 .. nkv(q) - 1
-    auto tok0_of = [&](int q) { return (pair * NQ + q) * C::TQ; };
-    auto nkv_of = [&](int q) {
-        const int t0 = tok0_of(q);
-        if (t0 >= chunk) return 0;
-        return ceil_div(ctx - chunk + min(chunk, t0 + C::TQ), BN);
-    };
-    int nkv = 0;
-#pragma unroll
-    for (int q = 0; q < NQ; ++q) nkv = max(nkv, nkv_of(q));
-    const int nblk_seq = ceil_div(ctx, BS);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const bool claiming = sc.counters != nullptr;
+    const bool tables = claiming && sc.num_seqs <= kPrefillSeqsInSmem;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < KST; ++i) {
@@ -186,13 +232,18 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
         for (int q = 0; q < NQ; ++q) {
             mbar_init(&s_full[q], 1);
             mbar_init(&s_free[q], 4);
+            mbar_init(&drain[q], 1);
+            mbar_init(&q_full[q], 4);
         }
         for (int b = 0; b < 2 * NQ; ++b) {
             mbar_init(&p_full[b], 4);
             mbar_init(&o_done[b], 1);
         }
-        for (int q = 0; q < NQ; ++q) mbar_init(&drain[q], 1);
-        for (int q = 0; q < NQ; ++q) mbar_init(&q_full[q], 128);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&item_full[s], 1);
+            mbar_init(&item_empty[s], C::ITEM_READERS);
+        }
+        mbar_init(v_tail, 1);
         *abort_flag = 0;
         mbar_init_fence();
     }
@@ -200,16 +251,58 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
         tmem_alloc(tmem_slot, C::TMEM_COLS);
         tmem_relinquish();
     }
+    if (tables)
+        for (int i = threadIdx.x; i <= sc.num_seqs; i += C::THREADS) {
+            seq_qs[i] = __ldg(p.query_start + i);
+            if (i < sc.num_seqs) seq_ctx[i] = __ldg(p.context_lens + i);
+        }
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
+    if (tables) {
+        // claim order: sequences by context length, longest first (ties by index)
+        for (int s = threadIdx.x; s < sc.num_seqs; s += C::THREADS) {
+            const int c = seq_ctx[s];
+            int r = 0;
+            for (int u = 0; u < sc.num_seqs; ++u) {
+                const int cu = seq_ctx[u];
+                r += (cu > c) || (cu == c && u < s);
+            }
+            seq_order[r] = s;
+        }
+        __syncthreads();
+    }
+
+    // the n-th published item of this CTA, read by a whole warp; every reading warp arrives once
+    auto read_item = [&](int n, int (&it)[IT_N]) {
+        const int slot = n & 1;
+        const bool ok = mbar_wait_bounded(&item_full[slot], (n >> 1) & 1);
+#pragma unroll
+        for (int i = 0; i < IT_N; ++i) it[i] = items[slot * IT_N + i];
+        if (!ok) {
+            it[IT_SEQ] = -1;                                   // no item came: stop
+            if (lane == 0) {
+                record_error(PA_DEVERR_TIMEOUT);
+                *abort_flag = 1;
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&item_empty[slot]);
+    };
+    auto nkv_tile = [&](int chunk, int ctx, int pair, int q) {
+        const int t0 = (pair * NQ + q) * C::TQ;
+        return t0 >= chunk ? 0 : ceil_div(ctx - chunk + min(chunk, t0 + C::TQ), BN);
+    };
+
 
     if (warp == C::TMA_WARP || warp == C::TMA_WARP + 1) {
         // ------------------------------ TMA producers ------------------------------
         // one warp per operand: the warp reads the block table 32 entries at a time (the next
         // 32 are in flight meanwhile), lane 0 waits for the ring slot, and lane l issues the copy
-        // of block l / HALVES, half l % HALVES of the tile
+        // of block l / HALVES, half l % HALVES of the tile.  The K warp also claims the work
+        // items and publishes them through the two-entry ring; it claims the next item once it
+        // has filled its ring with the current one, so that claim latency is hidden.
         const bool is_v = warp != C::TMA_WARP;
         const int nst = is_v ? VST : KST;
         uint64_t *full = is_v ? v_full : k_full;
@@ -217,45 +310,161 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
         const CUtensorMap *map = is_v ? &tmap_v : &tmap_k;
         if (lane == 0) prefetch_tensormap(map);
         const uint64_t pol = l2_policy_evict_last();
-        const int32_t *trow = p.block_tables + (size_t)seq * p.max_blocks_per_seq;
         constexpr int BPT = C::BLOCKS_PER_TILE, TPB = 32 / BPT;
-        auto entry = [&](int lb) -> int {
-            return (lb < nblk_seq && lb < p.max_blocks_per_seq) ? __ldg(trow + lb) : -1;
-        };
-        int cur = entry(lane), nxt = entry(32 + lane);
         const int k = lane / C::HALVES, hf = lane % C::HALVES;
-        int issued = 0;                                        // tiles whose copies were issued
-        for (int it = 0; it < nkv; ++it) {
-            if (it > 0 && it % TPB == 0) {
-                cur = nxt;
-                nxt = entry((it / TPB + 1) * 32 + lane);
-            }
-            const int st = it % nst;
-            int go = 1;
+        int issued = 0, ntail = 0;                             // tiles whose copies were issued (all items)
+
+        // ---- claiming and publishing (K warp) ----
+        int published = 0;
+        bool more = true;                                      // lane 0: claims may continue
+        auto seq_q0 = [&](int s) { return tables ? seq_qs[s] : __ldg(p.query_start + s); };
+        auto seq_cx = [&](int s) { return tables ? seq_ctx[s] : __ldg(p.context_lens + s); };
+        // the next item with work, or the end (lane 0 claims, the warp gets it)
+        auto claim = [&](int (&it)[IT_N]) {
+#pragma unroll
+            for (int i = 0; i < IT_N; ++i) it[i] = -1;
             if (lane == 0) {
-                if (it >= nst && !mbar_wait_or_abort(&empty[st], ((it / nst) - 1) & 1, abort_flag)) {
-                    if (!*abort_flag) record_error(PA_DEVERR_TIMEOUT);
+                while (more) {
+                    int kk;
+                    if (claiming) {
+                        if (*abort_flag) {
+                            more = false;
+                            break;
+                        }
+                        kk = atomicAdd(sc.counters, 1);
+                        if (kk >= sc.total_items) {
+                            more = false;
+                            break;
+                        }
+                    } else {
+                        kk = blockIdx.x + sc.pairs_max * (blockIdx.y + p.h_kv * blockIdx.z);
+                        more = false;                          // one item per CTA
+                    }
+                    const int x = kk % sc.pairs_max, r = kk / sc.pairs_max;
+                    const int kvh = r % p.h_kv, zi = r / p.h_kv;
+                    const int seq = tables ? seq_order[zi] : zi;
+                    const int q0 = seq_q0(seq), chunk = seq_q0(seq + 1) - q0, ctx = seq_cx(seq);
+                    if (chunk > ctx) {                         // rows left unwritten, flagged
+                        if (x == 0 && kvh == 0) record_error(PA_DEVERR_BAD_CHUNK);
+                        continue;
+                    }
+                    const int pair = ceil_div(prefill_tiles<C::TQ>(chunk), NQ) - 1 - x;   // x = 0: longest KV range
+                    if (pair < 0 || chunk <= 0) continue;
+                    it[IT_SEQ] = seq;
+                    it[IT_KVH] = kvh;
+                    it[IT_PAIR] = pair;
+                    it[IT_Q0] = q0;
+                    it[IT_CHUNK] = chunk;
+                    it[IT_CTX] = ctx;
+                    it[IT_NKV0] = nkv_tile(chunk, ctx, pair, 0);
+                    it[IT_NKV1] = NQ > 1 ? nkv_tile(chunk, ctx, pair, 1) : 0;
+                    break;
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < IT_N; ++i) it[i] = __shfl_sync(FULL, it[i], 0);
+        };
+        auto publish = [&](const int (&it)[IT_N]) {
+            const int slot = published & 1;
+            if (lane == 0) {
+                // the slot's previous item has been read by every reader (bounded; on a timeout
+                // the CTA is stopped and the item is written all the same, so readers see the end)
+                if (published >= 2 && !mbar_wait_bounded(&item_empty[slot], ((published >> 1) - 1) & 1)) {
+                    record_error(PA_DEVERR_TIMEOUT);
                     *abort_flag = 1;
                 }
-                go = *abort_flag ? 0 : 1;
+#pragma unroll
+                for (int i = 0; i < IT_N; ++i) items[slot * IT_N + i] = it[i];
+                mbar_arrive(&item_full[slot]);
             }
-            if (!__shfl_sync(FULL, go, 0)) break;
-            const int nb = min(BPT, nblk_seq - it * BPT);
-            const int phys = __shfl_sync(FULL, cur, (it % TPB) * BPT + min(k, BPT - 1));
-            const bool mine = lane < nb * C::HALVES;
-            if (__any_sync(FULL, mine && (phys < 0 || phys >= p.num_blocks))) {
-                if (lane == 0) {
-                    record_error(PA_DEVERR_BAD_BLOCK);
-                    *abort_flag = 1;                           // the MMA warps' waits see it
-                }
-                break;
-            }
-            if (lane == 0) mbar_arrive_expect_tx(&full[st], (uint32_t)(nb * C::HALVES * BS * 128));
             __syncwarp();
-            if (mine)
-                tma_load_2d(smem + (is_v ? C::OFF_V : C::OFF_K) + st * C::KV_TILE + hf * C::KV_HALF + k * BS * 128, map,
-                            hf * 64, (phys * p.h_kv + kvh) * BS, &full[st], pol);
-            ++issued;
+            ++published;
+        };
+
+        int cur[IT_N], nxt[IT_N];
+        if (!is_v) {
+            claim(cur);
+            publish(cur);
+        } else {
+            read_item(0, cur);
+        }
+        for (int n = 0; cur[IT_SEQ] >= 0; ++n) {
+            const int ctx = cur[IT_CTX], nkv = max(cur[IT_NKV0], cur[IT_NKV1]);
+            const int nblk_seq = ceil_div(ctx, BS);
+            const int32_t *trow = p.block_tables + (size_t)cur[IT_SEQ] * p.max_blocks_per_seq;
+            auto entry = [&](int lb) -> int {
+                return (lb < nblk_seq && lb < p.max_blocks_per_seq) ? __ldg(trow + lb) : -1;
+            };
+            int ecur = entry(lane), enxt = entry(32 + lane);
+            const int row_kvh = cur[IT_KVH];
+            bool next_known = is_v;                            // K warp: next item claimed and published
+            for (int t = 0; t < nkv; ++t) {
+                if (t > 0 && t % TPB == 0) {
+                    ecur = enxt;
+                    enxt = entry((t / TPB + 1) * 32 + lane);
+                }
+                const int st = issued % nst;
+                int go = 1;
+                if (lane == 0) {
+                    if (issued >= nst && !mbar_wait_or_abort(&empty[st], ((issued / nst) - 1) & 1, abort_flag)) {
+                        if (!*abort_flag) record_error(PA_DEVERR_TIMEOUT);
+                        *abort_flag = 1;
+                    }
+                    go = *abort_flag ? 0 : 1;
+                }
+                if (!__shfl_sync(FULL, go, 0)) break;
+                const int nb = min(BPT, nblk_seq - t * BPT);
+                const int phys = __shfl_sync(FULL, ecur, (t % TPB) * BPT + min(k, BPT - 1));
+                const bool mine = lane < nb * C::HALVES;
+                if (__any_sync(FULL, mine && (phys < 0 || phys >= p.num_blocks))) {
+                    if (lane == 0) {
+                        record_error(PA_DEVERR_BAD_BLOCK);
+                        *abort_flag = 1;                       // the other roles' waits see it
+                    }
+                    break;
+                }
+                // V tile holding rows past the context: the copy lands on v_tail, the rows past
+                // the context are zeroed, and only then is the tile marked full
+                const bool tail = is_v && (t + 1) * BN > ctx;
+                uint64_t *bar = tail ? v_tail : &full[st];
+                uint8_t *dst = smem + (is_v ? C::OFF_V : C::OFF_K) + st * C::KV_TILE;
+                if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)(nb * C::HALVES * BS * 128));
+                __syncwarp();
+                if (mine)
+                    tma_load_2d(dst + hf * C::KV_HALF + k * BS * 128, map, hf * 64, (phys * p.h_kv + row_kvh) * BS, bar, pol);
+                ++issued;
+                if (tail) {
+                    // our own copy: wait for it whatever the abort flag says (bounded)
+                    const int landed = __shfl_sync(FULL, lane == 0 ? (int)mbar_wait_bounded(v_tail, ntail & 1) : 0, 0);
+                    ++ntail;
+                    if (landed) {
+                        const int r0 = ctx - t * BN, per_half = (BN - r0) * 8;
+                        for (int idx = lane; idx < C::HALVES * per_half; idx += 32) {
+                            const int h = idx / per_half, rem = idx % per_half;
+                            *reinterpret_cast<uint4 *>(dst + h * C::KV_HALF + (r0 + rem / 8) * 128 + (rem % 8) * 16) =
+                                make_uint4(0u, 0u, 0u, 0u);
+                        }
+                        fence_proxy_async_smem();
+                    } else if (lane == 0) {
+                        record_error(PA_DEVERR_TIMEOUT);
+                        *abort_flag = 1;
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&full[st]);     // completes the phase (no bytes expected)
+                }
+                if (!next_known && (t == nst - 1 || t == nkv - 1)) {
+                    claim(nxt);
+                    publish(nxt);
+                    next_known = true;
+                }
+            }
+            if (!next_known) {                                 // stopped early: publish the end
+                claim(nxt);
+                publish(nxt);
+            }
+            if (is_v) read_item(n + 1, nxt);
+#pragma unroll
+            for (int i = 0; i < IT_N; ++i) cur[i] = nxt[i];
         }
         // Every copy this warp issued has landed before the CTA can exit, also when it stopped
         // early and nobody consumed the last tiles: wait (bounded) for each of the last nst
@@ -269,62 +478,79 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
         // Lane 0 issues S_j = Q K_j^T and O += P_j V_j for its tile.  Every query tile releases
         // every K and V slot once per KV tile: a tile that reads the slot commits after its MMAs,
         // a tile whose range ended arrives as soon as the slot's data has landed (so the
-        // arrival falls into that tile's phase of the empty barrier).
+        // arrival falls into that tile's phase of the empty barrier).  Ring slots and the S / P
+        // / O barriers are counted across items (gk: KV tiles so far, gs: this tile's steps so far).
         const int q = warp - C::MMA_WARP;
+        const uint32_t d_s = tmem + q * C::TMEM_PER_Q, d_o = d_s + C::COL_O, d_p = d_s + C::COL_P;
+        const uint64_t qdesc = umma_desc_sw128(smem_addr(smem + C::OFF_Q + q * C::Q_BYTES), 16, 1024);
+        const uint64_t kdesc = umma_desc_sw128(smem_addr(smem + C::OFF_K), 16, 1024);
+        const uint64_t vdesc = umma_desc_sw128(smem_addr(smem + C::OFF_V), C::KV_HALF, 1024);
+        int gk = 0, gs = 0, nq = 0;                            // nq: items with work for this tile so far
+        bool ok = true;
+        for (int n = 0;; ++n) {
+            int it[IT_N];
+            read_item(n, it);
+            if (it[IT_SEQ] < 0) break;
+            if (lane == 0) {
+                const int nkq = (q == 0 ? it[IT_NKV0] : it[IT_NKV1]), nkv = max(it[IT_NKV0], it[IT_NKV1]);
+                auto s_mma = [&](int j) -> bool {
+                    const int gt = gk + j, st = gt % KST, gj = gs + j;
+                    if (!mbar_wait_or_abort(&k_full[st], (gt / KST) & 1, abort_flag) || *abort_flag) return false;
+                    if (gj >= 1 && (!mbar_wait_or_abort(&s_free[q], (gj - 1) & 1, abort_flag) || *abort_flag)) return false;
+                    tc_fence_after_sync();
+                    const uint64_t kd = kdesc + (uint64_t)((st * C::KV_TILE) >> 4);
+#pragma unroll
+                    for (int ks = 0; ks < D / 16; ++ks)
+                        umma_bf16_ss(d_s, qdesc + (uint64_t)(((ks >> 2) * C::Q_HALF + (ks & 3) * 32) >> 4),
+                                     kd + (uint64_t)(((ks >> 2) * C::KV_HALF + (ks & 3) * 32) >> 4), C::IDESC_S, ks > 0);
+                    umma_commit(&s_full[q]);
+                    umma_commit(&k_empty[st]);
+                    return true;
+                };
+                auto pv = [&](int i) -> bool {
+                    const int gt = gk + i, gi = gs + i;
+                    if (!mbar_wait_or_abort(&v_full[gt % VST], (gt / VST) & 1, abort_flag) || *abort_flag) return false;
+                    if (!mbar_wait_or_abort(&p_full[2 * q + (gi & 1)], (gi >> 1) & 1, abort_flag) || *abort_flag) return false;
+                    tc_fence_after_sync();
+                    const uint64_t vd = vdesc + (uint64_t)(((gt % VST) * C::KV_TILE) >> 4);
+                    const uint32_t pt = d_p + 32 * (gi & 1);
+#pragma unroll
+                    for (int kk = 0; kk < BN / 16; ++kk)
+                        umma_bf16_ts(d_o, pt + 8 * kk, vd + (uint64_t)((kk * 2048) >> 4), C::IDESC_O, i > 0 || kk > 0);
+                    umma_commit(&o_done[2 * q + (gi & 1)]);
+                    umma_commit(&v_empty[gt % VST]);
+                    return true;
+                };
+                // the item's Q tile, copied by the tile's softmax warps.  Only items with work for
+                // the tile use the barrier, on both sides: the softmax cannot finish such an item
+                // before its S products, so it never runs a phase ahead of this wait
+                if (nkq > 0) {
+                    if (ok) ok = mbar_wait_or_abort(&q_full[q], nq & 1, abort_flag) && !*abort_flag;
+                    ++nq;
+                    if (ok) ok = s_mma(0);
+                }
+                for (int j = 0; j < nkq && ok; ++j) {
+                    if (j + 1 < nkq) ok = s_mma(j + 1);
+                    if (ok) ok = pv(j);
+                }
+                // the KV tiles past this query tile's range: release their slots as they land
+                for (int j = nkq; j < nkv && ok; ++j) {
+                    const int gt = gk + j;
+                    ok = mbar_wait_or_abort(&k_full[gt % KST], (gt / KST) & 1, abort_flag) && !*abort_flag;
+                    if (ok) mbar_arrive(&k_empty[gt % KST]);
+                    ok = ok && mbar_wait_or_abort(&v_full[gt % VST], (gt / VST) & 1, abort_flag) && !*abort_flag;
+                    if (ok) mbar_arrive(&v_empty[gt % VST]);
+                }
+                if (!ok) {
+                    if (!*abort_flag) record_error(PA_DEVERR_TIMEOUT);
+                    *abort_flag = 1;
+                }
+                gk += nkv;
+                gs += nkq;
+            }
+            __syncwarp();
+        }
         if (lane == 0) {
-            const int nkq = nkv_of(q);
-            const uint32_t d_s = tmem + q * C::TMEM_PER_Q, d_o = d_s + C::COL_O, d_p = d_s + C::COL_P;
-            const uint64_t qdesc = umma_desc_sw128(smem_addr(smem + C::OFF_Q + q * C::Q_BYTES), 16, 1024);
-            const uint64_t kdesc = umma_desc_sw128(smem_addr(smem + C::OFF_K), 16, 1024);
-            const uint64_t vdesc = umma_desc_sw128(smem_addr(smem + C::OFF_V), C::KV_HALF, 1024);
-            auto s_mma = [&](int j) -> bool {
-                const int st = j % KST;
-                if (!mbar_wait_or_abort(&k_full[st], (j / KST) & 1, abort_flag) || *abort_flag) return false;
-                if (j >= 1 && (!mbar_wait_or_abort(&s_free[q], (j - 1) & 1, abort_flag) || *abort_flag)) return false;
-                tc_fence_after_sync();
-                const uint64_t kd = kdesc + (uint64_t)((st * C::KV_TILE) >> 4);
-#pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks)
-                    umma_bf16_ss(d_s, qdesc + (uint64_t)(((ks >> 2) * C::Q_HALF + (ks & 3) * 32) >> 4),
-                                 kd + (uint64_t)(((ks >> 2) * C::KV_HALF + (ks & 3) * 32) >> 4), C::IDESC_S, ks > 0);
-                umma_commit(&s_full[q]);
-                umma_commit(&k_empty[st]);
-                return true;
-            };
-            auto pv = [&](int i) -> bool {
-                if (!mbar_wait_or_abort(&v_full[i % VST], (i / VST) & 1, abort_flag) || *abort_flag) return false;
-                if (!mbar_wait_or_abort(&p_full[2 * q + (i & 1)], (i >> 1) & 1, abort_flag) || *abort_flag) return false;
-                tc_fence_after_sync();
-                const uint64_t vd = vdesc + (uint64_t)(((i % VST) * C::KV_TILE) >> 4);
-                const uint32_t pt = d_p + 32 * (i & 1);
-#pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk)
-                    umma_bf16_ts(d_o, pt + 8 * kk, vd + (uint64_t)((kk * 2048) >> 4), C::IDESC_O, i > 0 || kk > 0);
-                umma_commit(&o_done[2 * q + (i & 1)]);
-                umma_commit(&v_empty[i % VST]);
-                return true;
-            };
-            bool ok = true;
-            if (nkq > 0) {
-                // the tile's Q rows, written by its softmax warpgroup after the CTA barrier
-                ok = mbar_wait_or_abort(&q_full[q], 0, abort_flag) && !*abort_flag;
-                if (ok) ok = s_mma(0);
-            }
-            for (int j = 0; j < nkq && ok; ++j) {
-                if (j + 1 < nkq) ok = s_mma(j + 1);
-                if (ok) ok = pv(j);
-            }
-            // the KV tiles past this query tile's range: release their slots as they land
-            for (int j = nkq; j < nkv && ok; ++j) {
-                ok = mbar_wait_or_abort(&k_full[j % KST], (j / KST) & 1, abort_flag) && !*abort_flag;
-                if (ok) mbar_arrive(&k_empty[j % KST]);
-                ok = ok && mbar_wait_or_abort(&v_full[j % VST], (j / VST) & 1, abort_flag) && !*abort_flag;
-                if (ok) mbar_arrive(&v_empty[j % VST]);
-            }
-            if (!ok) {
-                if (!*abort_flag) record_error(PA_DEVERR_TIMEOUT);
-                *abort_flag = 1;
-            }
             umma_commit(&drain[q]);                             // every MMA this thread issued has finished
             mbar_wait_bounded(&drain[q], 0);
         }
@@ -332,184 +558,210 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
     } else {
         // ------------------------------ softmax warpgroups ------------------------------
         const int q = warp >> 2, t = threadIdx.x & 127;
-        const int tok0 = tok0_of(q), nkv_q = nkv_of(q);
-        const int tok = tok0 + t / G;
-        const bool row_ok = tok < chunk;
-        {
-            // this thread's Q row into the tile's swizzled shared tile (row t = token t / G, head
-            // t % G), after the CTA barrier so that the loads overlap the producers' first K/V
-            // copies; the MMA warp waits for all 128 rows on q_full before the tile's first S
-            const uint4 *src = reinterpret_cast<const uint4 *>(
-                p.q + ((size_t)(q0 + (row_ok ? tok : 0)) * p.h_q + (size_t)kvh * G + t % G) * D);
-            uint4 v[D / 8];
-#pragma unroll
-            for (int c = 0; c < D / 8; ++c) v[c] = row_ok ? src[c] : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-            for (int c = 0; c < D / 8; ++c)
-                *reinterpret_cast<uint4 *>(smem + C::OFF_Q + q * C::Q_BYTES + (c >> 3) * C::Q_HALF + swz128(t, c & 7)) =
-                    v[c];
-            fence_proxy_async_smem();
-            mbar_arrive(&q_full[q]);
-        }
-        const int pos = row_ok ? ctx - chunk + tok : 0;
-        const int first_pos = ctx - chunk + tok0;
         const uint32_t lane_tm = tmem + q * C::TMEM_PER_Q + ((uint32_t)(32 * (warp & 3)) << 16);
         uint64_t *my_s_full = s_full + q, *my_s_free = s_free + q;
         uint64_t *my_p_full = p_full + 2 * q, *my_o_done = o_done + 2 * q;
-        float m_run = -INFINITY, l_run = 0.f;
-        bool failed = false;
-        for (int j = 0; j < nkv_q; ++j) {
-            bool ok = __all_sync(FULL, mbar_wait_or_abort(my_s_full, j & 1, abort_flag));
-            if (!ok || *abort_flag) {
-                failed = true;
-                break;
-            }
-            tc_fence_after_sync();
-            uint32_t sr[2][32];
-            tmem_ld32(lane_tm, sr[0]);
-            tmem_ld32(lane_tm + 32u, sr[1]);
-            tmem_wait_ld();
-            tc_fence_before_sync();
+        // this thread's Q row of the tile into its swizzled shared tile (row t = token t / G, head
+        // t % G), zero-filled past the chunk; cp.async, completed by q_ready
+        auto copy_q = [&](int pair, int q0, int chunk, int kvh) {
+            const int tq = (pair * NQ + q) * C::TQ + t / G;
+            const bool ok = tq < chunk;
+            const __nv_bfloat16 *src = p.q + ((size_t)(q0 + (ok ? tq : 0)) * p.h_q + (size_t)kvh * G + t % G) * D;
+            uint8_t *qt = smem + C::OFF_Q + q * C::Q_BYTES;
+#pragma unroll
+            for (int c = 0; c < D / 8; ++c) cp_async_16_zfill(qt + (c >> 3) * C::Q_HALF + swz128(t, c & 7), src + 8 * c, ok);
+        };
+        // this thread's copies landed; once all four warps arrive the MMA warp may read the tile
+        auto q_ready = [&]() {
+            cp_async_wait_all();
+            fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(my_s_free);
-
-            // raw scores s; the log2-domain logit is s * qk_scale (qk_scale > 0, so the max of
-            // the logits is the scaled max of the scores), p = 2^(s * qk_scale - m) by one FMA
-            const int kv0 = j * BN;
-            if (kv0 + BN - 1 > first_pos) {
-#pragma unroll
-                for (int h = 0; h < 2; ++h)
-#pragma unroll
-                    for (int c = 0; c < 32; ++c)
-                        if (kv0 + 32 * h + c > pos) sr[h][c] = 0xff800000u;        // -inf
+            if (lane == 0) mbar_arrive(&q_full[q]);
+        };
+        int gs = 0;                                            // this tile's steps so far (all items)
+        bool q_copying = false;                                // the next item's Q copy is in flight
+        for (int n = 0;; ++n) {
+            int it[IT_N];
+            read_item(n, it);
+            if (it[IT_SEQ] < 0) break;
+            const int chunk = it[IT_CHUNK], ctx = it[IT_CTX], nkv_q = (q == 0 ? it[IT_NKV0] : it[IT_NKV1]);
+            if (nkv_q > 0) {                                   // only items with work use q_full
+                if (!q_copying && !*abort_flag) copy_q(it[IT_PAIR], it[IT_Q0], chunk, it[IT_KVH]);
+                q_ready();
             }
-            // pair i of the row tile = columns 2i, 2i + 1
-            auto pair_of = [&](int i) {
-                return make_float2(__uint_as_float(sr[i >> 4][2 * (i & 15)]), __uint_as_float(sr[i >> 4][2 * (i & 15) + 1]));
-            };
-            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const float2 s2 = pair_of(i);
-                m4[i & 3] = max3f(m4[i & 3], s2.x, s2.y);
-            }
-            const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-            // m_run is the reference the exponentials are taken against.  It moves (and O and
-            // l are rescaled) only when the tile's max exceeds it by more than 8, so p <= 2^8;
-            // O / l does not depend on the reference, and rescaling becomes rare, which keeps
-            // the softmax from waiting for the previous P V.
-            const float m_tile = mx * p.qk_scale;
-            float alpha = 1.f;
-            bool moved = false;
-            if (j == 0) {
-                m_run = m_tile;
-            } else if (m_tile > m_run + 8.f) {
-                alpha = ex2_approx(m_run - m_tile);
-                m_run = m_tile;
-                moved = true;
-            }
-            const float mn = m_run;
-            // p = 2^(s * qk_scale - m) in pairs: one packed FMA, then the MUFU unit for most pairs
-            // and the FMA-pipe polynomial for POLY_PAIRS of every 8 (the two units run side by
-            // side); the row sum in two packed partial sums
-            uint32_t pk[32];
-            const float2 sc2 = make_float2(p.qk_scale, p.qk_scale), nm2 = make_float2(-mn, -mn);
-            float2 rsa = make_float2(0.f, 0.f), rsb = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const float2 x2 = __ffma2_rn(pair_of(i), sc2, nm2);
-                const float2 e2 = (i & 7) < C::POLY_PAIRS ? ex2_poly2(x2) : make_float2(ex2_approx(x2.x), ex2_approx(x2.y));
-                if (i & 1) rsb = __fadd2_rn(rsb, e2);
-                else rsa = __fadd2_rn(rsa, e2);
-                pk[i] = pack_bf16x2(e2.x, e2.y);
-            }
-            const float rs = (rsa.x + rsb.x) + (rsa.y + rsb.y);
-            l_run = l_run * alpha + rs;
-            // rescale this warp's rows of O when any of their maxima moved (PV_{j-1} must be done)
-            if (__any_sync(FULL, moved)) {
-                ok = __all_sync(FULL, mbar_wait_or_abort(&my_o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag));
+            q_copying = false;
+            const int tok0 = (it[IT_PAIR] * NQ + q) * C::TQ;
+            const int tok = tok0 + t / G;
+            const bool row_ok = tok < chunk;
+            const int pos = row_ok ? ctx - chunk + tok : 0;
+            const int first_pos = ctx - chunk + tok0;
+            float m_run = -INFINITY, l_run = 0.f;
+            bool failed = *abort_flag != 0;                    // a stopped CTA writes NaN rows
+            for (int j = 0; j < nkv_q && !failed; ++j) {
+                const int gj = gs + j;
+                bool ok = __all_sync(FULL, mbar_wait_or_abort(my_s_full, gj & 1, abort_flag));
                 if (!ok || *abort_flag) {
                     failed = true;
                     break;
                 }
                 tc_fence_after_sync();
+                uint32_t sr[2][32];
+                tmem_ld32(lane_tm, sr[0]);
+                tmem_ld32(lane_tm + 32u, sr[1]);
+                tmem_wait_ld();
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(my_s_free);
+
+                // raw scores s; the log2-domain logit is s * qk_scale (qk_scale > 0, so the max of
+                // the logits is the scaled max of the scores), p = 2^(s * qk_scale - m) by one FMA
+                const int kv0 = j * BN;
+                if (kv0 + BN - 1 > first_pos) {
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+#pragma unroll
+                        for (int c = 0; c < 32; ++c)
+                            if (kv0 + 32 * h + c > pos) sr[h][c] = 0xff800000u;        // -inf
+                }
+                // pair i of the row tile = columns 2i, 2i + 1
+                auto pair_of = [&](int i) {
+                    return make_float2(__uint_as_float(sr[i >> 4][2 * (i & 15)]), __uint_as_float(sr[i >> 4][2 * (i & 15) + 1]));
+                };
+                float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float2 s2 = pair_of(i);
+                    m4[i & 3] = max3f(m4[i & 3], s2.x, s2.y);
+                }
+                const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+                // m_run is the reference the exponentials are taken against.  It moves (and O and
+                // l are rescaled) only when the tile's max exceeds it by more than 8, so p <= 2^8;
+                // O / l does not depend on the reference, and rescaling becomes rare, which keeps
+                // the softmax from waiting for the previous P V.
+                const float m_tile = mx * p.qk_scale;
+                float alpha = 1.f;
+                bool moved = false;
+                if (j == 0) {
+                    m_run = m_tile;
+                } else if (m_tile > m_run + 8.f) {
+                    alpha = ex2_approx(m_run - m_tile);
+                    m_run = m_tile;
+                    moved = true;
+                }
+                const float mn = m_run;
+                // p = 2^(s * qk_scale - m) in pairs: one packed FMA, then the MUFU unit for most pairs
+                // and the FMA-pipe polynomial for POLY_PAIRS of every 8 (the two units run side by
+                // side); the row sum in two packed partial sums
+                uint32_t pk[32];
+                const float2 sc2 = make_float2(p.qk_scale, p.qk_scale), nm2 = make_float2(-mn, -mn);
+                float2 rsa = make_float2(0.f, 0.f), rsb = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float2 x2 = __ffma2_rn(pair_of(i), sc2, nm2);
+                    const float2 e2 = (i & 7) < C::POLY_PAIRS ? ex2_poly2(x2) : make_float2(ex2_approx(x2.x), ex2_approx(x2.y));
+                    if (i & 1) rsb = __fadd2_rn(rsb, e2);
+                    else rsa = __fadd2_rn(rsa, e2);
+                    pk[i] = pack_bf16x2(e2.x, e2.y);
+                }
+                const float rs = (rsa.x + rsb.x) + (rsa.y + rsb.y);
+                l_run = l_run * alpha + rs;
+                // rescale this warp's rows of O when any of their maxima moved (P V_{j-1} must be done)
+                if (__any_sync(FULL, moved)) {
+                    ok = __all_sync(FULL, mbar_wait_or_abort(&my_o_done[(gj - 1) & 1], ((gj - 1) >> 1) & 1, abort_flag));
+                    if (!ok || *abort_flag) {
+                        failed = true;
+                        break;
+                    }
+                    tc_fence_after_sync();
+#pragma unroll
+                    for (int cb = 0; cb < D / 32; ++cb) {
+                        uint32_t o[32];
+                        tmem_ld32(lane_tm + C::COL_O + 32 * cb, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+                        tmem_st32(lane_tm + C::COL_O + 32 * cb, o);
+                    }
+                    tmem_wait_st();
+                }
+                // P buffer gj % 2 is free once P V_{gj-2} has finished
+                if (gj >= 2) {
+                    ok = __all_sync(FULL, mbar_wait_or_abort(&my_o_done[gj & 1], ((gj - 2) >> 1) & 1, abort_flag));
+                    if (!ok || *abort_flag) {
+                        failed = true;
+                        break;
+                    }
+                }
+                tmem_st32(lane_tm + (uint32_t)(C::COL_P + 32 * (gj & 1)), pk);
+                tmem_wait_st();
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&my_p_full[gj & 1]);
+            }
+            if (!failed && nkv_q > 0) {
+                // every S product of the item is done, so the tile's Q rows are no longer read:
+                // start copying the next item's rows (if it is published already) before the
+                // epilogue, which then overlaps the copy
+                const int ns = (n + 1) & 1;
+                if (mbar_test_wait(&item_full[ns], ((n + 1) >> 1) & 1)) {
+                    const volatile int *nx = items + ns * IT_N;
+                    if (nx[IT_SEQ] >= 0 && (q == 0 ? nx[IT_NKV0] : nx[IT_NKV1]) > 0 && !*abort_flag) {
+                        copy_q(nx[IT_PAIR], nx[IT_Q0], nx[IT_CHUNK], nx[IT_KVH]);
+                        q_copying = true;
+                    }
+                }
+            }
+            if (!failed && nkv_q > 0) {
+                const int gl = gs + nkv_q - 1;
+                const bool ok = __all_sync(FULL, mbar_wait_or_abort(&my_o_done[gl & 1], (gl >> 1) & 1, abort_flag));
+                failed = !ok || *abort_flag;
+            }
+            if (nkv_q > 0) {
+                if (!failed) tc_fence_after_sync();
+                // normalise and write this row
+                const float inv = (!failed && l_run > 0.f) ? 1.f / l_run : __int_as_float(0x7fc00000);
+                __nv_bfloat16 *orow =
+                    p.out + ((size_t)(it[IT_Q0] + (row_ok ? tok : 0)) * p.h_q + (size_t)it[IT_KVH] * G + t % G) * D;
 #pragma unroll
                 for (int cb = 0; cb < D / 32; ++cb) {
                     uint32_t o[32];
-                    tmem_ld32(lane_tm + C::COL_O + 32 * cb, o);
-                    tmem_wait_ld();
+                    if (!failed) {
+                        tmem_ld32(lane_tm + C::COL_O + 32 * cb, o);
+                        tmem_wait_ld();
+                    }
+                    if (row_ok) {
+                        uint32_t w[16];
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-                    tmem_st32(lane_tm + C::COL_O + 32 * cb, o);
+                        for (int c = 0; c < 16; ++c)
+                            w[c] = failed ? 0x7fc07fc0u
+                                          : pack_bf16x2(__uint_as_float(o[2 * c]) * inv, __uint_as_float(o[2 * c + 1]) * inv);
+#pragma unroll
+                        for (int v = 0; v < 4; ++v)
+                            reinterpret_cast<uint4 *>(orow + 32 * cb)[v] =
+                                make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+                    }
                 }
-                tmem_wait_st();
+                // the O reads are complete (tcgen05.wait::ld) before this warp arrives on the
+                // next item's first p_full, which lets the next item's first P V overwrite O
+                tc_fence_before_sync();
             }
-            // V rows past the context (last tile): zero them before the P V step reads the tile
-            if (kv0 + BN > ctx) {
-                ok = __all_sync(FULL, mbar_wait_or_abort(&v_full[j % VST], (j / VST) & 1, abort_flag));
-                if (!ok) {
-                    failed = true;
-                    break;
-                }
-                const int r0 = max(0, ctx - kv0);
-                uint8_t *vt = smem + C::OFF_V + (j % VST) * C::KV_TILE;
-                const int per_half = (BN - r0) * 8;
-                for (int idx = t; idx < C::HALVES * per_half; idx += 128) {
-                    const int hf = idx / per_half, rem = idx % per_half;
-                    *reinterpret_cast<uint4 *>(vt + hf * C::KV_HALF + (r0 + rem / 8) * 128 + (rem % 8) * 16) =
-                        make_uint4(0u, 0u, 0u, 0u);
-                }
-                fence_proxy_async_smem();
-            }
-            // P buffer j % 2 is free once P V_{j-2} has finished
-            if (j >= 2) {
-                ok = __all_sync(FULL, mbar_wait_or_abort(&my_o_done[j & 1], ((j - 2) >> 1) & 1, abort_flag));
-                if (!ok || *abort_flag) {
-                    failed = true;
-                    break;
-                }
-            }
-            tmem_st32(lane_tm + (uint32_t)(C::COL_P + 32 * (j & 1)), pk);
-            tmem_wait_st();
-            tc_fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&my_p_full[j & 1]);
+            gs += nkv_q;
         }
-        if (!failed && nkv_q > 0) {
-            const bool ok = __all_sync(FULL, mbar_wait_or_abort(&my_o_done[(nkv_q - 1) & 1], ((nkv_q - 1) >> 1) & 1, abort_flag));
-            failed = !ok || *abort_flag;
-        }
-        if (nkv_q > 0) {
-            if (!failed) tc_fence_after_sync();
-            // normalise and write this row
-            const float inv = (!failed && l_run > 0.f) ? 1.f / l_run : __int_as_float(0x7fc00000);
-            __nv_bfloat16 *orow = p.out + ((size_t)(q0 + (row_ok ? tok : 0)) * p.h_q + (size_t)kvh * G + t % G) * D;
-#pragma unroll
-            for (int cb = 0; cb < D / 32; ++cb) {
-                uint32_t o[32];
-                if (!failed) {
-                    tmem_ld32(lane_tm + C::COL_O + 32 * cb, o);
-                    tmem_wait_ld();
-                }
-                if (row_ok) {
-                    uint32_t w[16];
-#pragma unroll
-                    for (int c = 0; c < 16; ++c)
-                        w[c] = failed ? 0x7fc07fc0u
-                                      : pack_bf16x2(__uint_as_float(o[2 * c]) * inv, __uint_as_float(o[2 * c + 1]) * inv);
-#pragma unroll
-                    for (int v = 0; v < 4; ++v)
-                        reinterpret_cast<uint4 *>(orow + 32 * cb)[v] =
-                            make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
-                }
-            }
-        }
+        cp_async_wait_all();                                   // no copy in flight at exit
         tc_fence_before_sync();
     }
     __syncthreads();
     if (warp == C::MMA_WARP) {
         tc_fence_after_sync();
         tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+    if (claiming && threadIdx.x == 0) {
+        // the last CTA to finish leaves the counters at zero for the next launch
+        __threadfence();
+        if (atomicAdd(sc.counters + 1, 1) == (int)gridDim.x - 1) {
+            atomicExch(sc.counters, 0);
+            atomicExch(sc.counters + 1, 0);
+        }
     }
 }
 

@@ -141,6 +141,25 @@ def test_prefill_host_checks():
     assert rc(B=0) == 0 and rc(mql=0) == 0                  # nothing to do, nothing launched
 
 
+def test_prefill_ws_host_checks():
+    def rc(ws=FAKE, wsb=256, **kw):
+        a = dict(out=FAKE, q=FAKE, k=FAKE, v=FAKE, bt=FAKE, maxblk=8, qs=FAKE, ctx=FAKE, B=2, mql=64, hq=8, hkv=2,
+                 d=128, bs=16, nb=16, scale=0.088, dt=0)
+        a.update(kw)
+        return L.pa_prefill_ws(a["out"], a["q"], a["k"], a["v"], a["bt"], a["maxblk"], a["qs"], a["ctx"], a["B"],
+                               a["mql"], a["hq"], a["hkv"], a["d"], a["bs"], a["nb"], a["scale"], a["dt"], ws, wsb,
+                               None)
+    need = L.pa_prefill_workspace_size()
+    assert 8 <= need <= 4096
+    assert rc(ws=0) == -3                                   # no workspace
+    assert rc(wsb=need - 1) == -3                           # too small
+    assert rc(ws=FAKE + 8) == -3                            # misaligned
+    assert rc(ws=0, B=0) == -3                              # the workspace is checked first
+    assert rc(wsb=need, d=96) == -2                         # then pa_prefill's own checks
+    assert rc(wsb=need, hq=6, hkv=4) == -1
+    assert rc(wsb=need, B=0) == 0                           # nothing to do, nothing launched
+
+
 def test_decode_step_host_checks():
     def rc(**kw):
         a = dict(key=FAKE, val=FAKE, kst=0, vst=0, slots=FAKE, out=FAKE, q=FAKE, kc=FAKE, vc=FAKE, bt=FAKE, maxblk=8,
