@@ -13,8 +13,8 @@
 // CTAs running at the same time share their K/V tiles through L2.  Without one (pa_prefill) the
 // grid has one CTA per item.  In both cases the next item is known before the current one ends:
 // the producers start its block-table reads and K/V copies while the current item's last tiles
-// are in use, and its Q tiles are copied as soon as the current item's last S products are done,
-// so an item costs its KV tiles plus a short epilogue instead of a chain of dependent loads.
+// are in use, and the softmax warps start copying its Q rows once the current item's P V products
+// are done, so an item costs its KV tiles plus an epilogue instead of a chain of dependent loads.
 //
 // Roles:
 //   warps 0-7  two softmax warpgroups, one per query tile: thread t of a warpgroup owns row t of
@@ -23,7 +23,9 @@
 //              max and sum (log2 domain; one in eight of the exponentials by a polynomial on
 //              the FMA pipe, beside the MUFU unit), stores its row of P_j (bf16) into tensor memory,
 //              rescales its row of O when its max moved, and at the end of the item normalises O
-//              and writes the output row.
+//              and writes the output row.  It copies its Q row of each item (cp.async, zero-filled
+//              past the chunk) into the swizzled Q tile and arrives on the tile's q_full; the
+//              next item's copy starts before the epilogue when that item is published already.
 //   warps 8-9  one MMA warp per query tile: lane 0 issues S_{j+1} = Q K_{j+1}^T (M 128, N 64,
 //              K = D, both operands in shared memory) as soon as the softmax has loaded S_j, and
 //              O += P_j V_j (M 128, N = D, K 64) with P read from tensor memory and V read N-major
@@ -38,10 +40,9 @@
 //              that read it finished, or the tile's KV range ended before it).  V rows past the
 //              context in an item's last tile are zeroed by the V producer once the copy has
 //              landed and before the tile is marked full (an unwritten NaN slot times a zero
-//              probability would poison O).
-//   warp 12    scheduler: claims items, publishes each through a two-entry ring in shared memory,
-//              and copies each item's Q rows (cp.async, zero-filled past the chunk) into the
-//              swizzled Q tiles once the previous item's S products no longer read them.
+//              probability would poison O).  The K warp also claims the work items and
+//              publishes each through a two-entry ring in shared memory that every other warp
+//              reads; it claims the next item once the current one's first tiles are issued.
 // Every wait on the data path is bounded and also ends when another role has stopped the CTA; on
 // a timeout or a bad block the CTA records the error, stops claiming, writes NaN into the rows
 // of the items it holds, waits for its copies and MMAs in flight and frees its tensor memory.
@@ -131,7 +132,7 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity)
 }
 
 // Sequence tables (query_start, context_lens) and the claim order are kept in shared memory for
-// up to this many sequences; beyond it the scheduler reads them from global memory and claims in
+// up to this many sequences; beyond it the K producer reads them from global memory and claims in
 // sequence order.
 constexpr int kPrefillSeqsInSmem = 1024;
 
