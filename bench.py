@@ -40,6 +40,9 @@ METRIC = "paged decode attention KV GB/s & % of B200 HBM peak; decode tokens/s"
 FALLBACK_HBM_GBS = 6650.0
 KERNEL_SOURCES = [os.path.join(ROOT, "paged_kv_cache_428_b200", "csrc", f)
                   for f in ("common.cuh", "decode.cuh", "decode_mma.cuh", "decode_q8.cuh", "decode_balanced.cuh")]
+# the tcgen05 prefill kernel and every header it includes
+PREFILL_SOURCES = [os.path.join(ROOT, "paged_kv_cache_428_b200", "csrc", f)
+                   for f in ("common.cuh", "decode.cuh", "decode_mma.cuh", "prefill.cuh", "tc.cuh", "prefill_tc.cuh")]
 PROFILES = os.path.join(ROOT, "profiles")
 
 
@@ -176,31 +179,38 @@ def measured_peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(sources=None) -> str:
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
+    for f in sources or KERNEL_SOURCES:
         with open(f, "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
-def ncu_traffic_per_launch(workload: str, partition: int):
-    """DRAM bytes (read + write) of one decode-kernel launch from a committed ncu summary under
-    profiles/ that names this workload and partition size, or None when there is none or the
-    kernel sources changed since the counters were taken."""
+def ncu_traffic_per_launch(workload: str, partition=None, schedule=None, sources=None):
+    """DRAM bytes (read + write) of one launch of the workload's kernel from a committed ncu
+    summary under profiles/ that names this workload and partition size (decode) or schedule
+    (prefill), or None when there is none or the kernel sources changed since the counters were
+    taken."""
     if not os.path.isdir(PROFILES):
         return None
-    want = kernel_source_hash()
+    want = kernel_source_hash(sources)
     for name in sorted(os.listdir(PROFILES)):
         if not name.endswith(".md"):
             continue
         text = open(os.path.join(PROFILES, name)).read()
         w = re.search(r"^workload:\s*(\S+)", text, re.M)
         p = re.search(r"^partition:\s*(-?[0-9]+)", text, re.M)
+        sc = re.search(r"^schedule:\s*(\S+)", text, re.M)
         m = re.search(r"^traffic_bytes_per_launch:\s*([0-9]+)", text, re.M)
         h = re.search(r"^kernel_source_sha256_16:\s*([0-9a-f]+)", text, re.M)
-        if w and p and m and h and w.group(1) == workload and int(p.group(1)) == partition and h.group(1) == want:
-            return int(m.group(1))
+        if not (w and m and h) or w.group(1) != workload or h.group(1) != want:
+            continue
+        if partition is not None and not (p and int(p.group(1)) == partition):
+            continue
+        if schedule is not None and not (sc and sc.group(1) == schedule):
+            continue
+        return int(m.group(1))
     return None
 
 
@@ -993,7 +1003,9 @@ def run_prefill(args):
         "kernels_ms_alone": {"prefill": round(kern_ms / K, 5)},
         "roofline": {"bound": "tensor", "kernel": prefill_kernel_name(args.prefill_schedule), "achieved": round(achieved, 1),
                      "peak": peak, "peak_kind": kind, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                     "traffic": None, "algorithmic_flops_per_launch": int(flops)},
+                     "traffic": ncu_traffic_per_launch(args.workload, schedule=args.prefill_schedule,
+                                                       sources=PREFILL_SOURCES),
+                     "algorithmic_flops_per_launch": int(flops)},
         "gpu_launches": 2 * K,
         "clocks": poller.summary(t0, t1) or sampler.summary(t0, t1),
         "clocks_kernel_loops": poller.summary(t1, t2) or sampler.summary(t1, t2),
