@@ -109,6 +109,20 @@ def test_full_size_sampled(orc, name, queue):
     _parity(orc, case, queue, rows=rows)
 
 
+@pytest.mark.parametrize("queue", QUEUE)
+def test_empty_chunks_between_sequences(orc, queue):
+    """Sequences with no query rows (query_start repeats a value) among others: they have no work
+    items and their neighbours' rows are unaffected; also sequences with no tokens at all."""
+    case = workloads.make_prefill_case("prefill_llama3_8b_b8_chunk512", 45, B=9, h_q=8, h_kv=2, cached=(0, 100),
+                                       chunk=(0, 5))
+    assert case.meta["chunk"].count(0) >= 2
+    _parity(orc, case, queue)
+    case = workloads.make_prefill_case("prefill_llama3_8b_b8_chunk512", 59, B=7, h_q=8, h_kv=2, cached=(0, 0),
+                                       chunk=(0, 40))
+    assert 0 in case.meta["chunk"]
+    _parity(orc, case, queue)
+
+
 def test_queue_with_more_sequences_than_kept_in_shared_memory(orc):
     """1100 sequences (beyond the 1024 whose tables and claim order the kernel keeps in shared
     memory: it reads them from global memory and claims in sequence order), short chunks after
