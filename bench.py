@@ -38,6 +38,7 @@ if ROOT not in sys.path:
 
 METRIC = "paged decode attention KV GB/s & % of B200 HBM peak; decode tokens/s"
 FALLBACK_HBM_GBS = 6650.0
+DEFAULT_WORKLOAD = "llama3_8b_b64"
 KERNEL_SOURCES = [os.path.join(ROOT, "paged_kv_cache_428_b200", "csrc", f)
                   for f in ("common.cuh", "decode.cuh", "decode_mma.cuh", "decode_q8.cuh", "decode_balanced.cuh")]
 # the tcgen05 prefill kernel and every header it includes
@@ -52,11 +53,13 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="llama3_8b_b64")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--partition", type=int, default=None, help="tokens per split-context partition")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill-line", action="store_true",
+                    help="do not append the chunked-prefill measurement to the default decode line")
     ap.add_argument("--prefill-schedule", choices=("queue", "grid"), default="queue",
                     help="prefill workloads: pa_prefill_ws (one CTA per SM claiming work items) or "
                          "pa_prefill (one CTA per work item)")
@@ -1015,12 +1018,36 @@ def run_prefill(args):
     return line
 
 
+PREFILL_SIDE_WORKLOAD = "prefill_llama3_8b_b8_chunk512"
+
+
+def prefill_side_line(args) -> dict:
+    """The chunked-prefill row measured in the same run as the default decode line (one GPU):
+    the same method as `--workload prefill_llama3_8b_b8_chunk512`, fewer steps.  A failure here is
+    reported in the object and never costs the decode line."""
+    try:
+        pargs = parse_args(["--workload", PREFILL_SIDE_WORKLOAD, "--steps", "10", "--warmup", "3", "--no-cpu-baseline",
+                            "--no-e2e", "--seed", str(args.seed)])
+        pl = run_prefill(pargs)
+        keep = ("metric", "value", "unit", "steps", "warmup", "ms_per_step", "tokens_per_s", "kernels_ms_alone",
+                "roofline", "clocks")
+        out = {k: pl[k] for k in keep if k in pl}
+        out["config"] = {k: pl["config"][k] for k in ("workload", "schedule", "step", "attention_flops_per_step", "l2")
+                         if k in pl["config"]}
+        return out
+    except Exception as e:                                      # pragma: no cover - reported, not raised
+        return {"workload": PREFILL_SIDE_WORKLOAD, "error": repr(e)[:300]}
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl != "reference" and args.workload.startswith("prefill_"):
         line = run_prefill(args)
     else:
         line = run_reference(args) if args.impl == "reference" else run_ours(args)
+        if (line is not None and args.impl != "reference" and line.get("n_gpus") == 1 and not args.no_prefill_line
+                and args.workload == DEFAULT_WORKLOAD):
+            line["prefill"] = prefill_side_line(args)
     if line is not None:
         print(json.dumps(line), flush=True)
 
