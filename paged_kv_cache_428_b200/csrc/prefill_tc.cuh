@@ -581,16 +581,18 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
         };
         int gs = 0;                                            // this tile's steps so far (all items)
         bool q_copying = false;                                // the next item's Q copy is in flight
+        bool q_announced = false;                              // ... and already announced on q_full
         for (int n = 0;; ++n) {
             int it[IT_N];
             read_item(n, it);
             if (it[IT_SEQ] < 0) break;
             const int chunk = it[IT_CHUNK], ctx = it[IT_CTX], nkv_q = (q == 0 ? it[IT_NKV0] : it[IT_NKV1]);
-            if (nkv_q > 0) {                                   // only items with work use q_full
+            if (nkv_q > 0 && !q_announced) {                   // only items with work use q_full
                 if (!q_copying && !*abort_flag) copy_q(it[IT_PAIR], it[IT_Q0], chunk, it[IT_KVH]);
                 q_ready();
             }
             q_copying = false;
+            q_announced = false;
             const int tok0 = (it[IT_PAIR] * NQ + q) * C::TQ;
             const int tok = tok0 + t / G;
             const bool row_ok = tok < chunk;
@@ -716,6 +718,12 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
                 const int gl = gs + nkv_q - 1;
                 const bool ok = __all_sync(FULL, mbar_wait_or_abort(&my_o_done[gl & 1], (gl >> 1) & 1, abort_flag));
                 failed = !ok || *abort_flag;
+            }
+            if (q_copying) {
+                // the next item's Q rows have had the last P V to land: announce them now, so
+                // its first S product runs during this item's epilogue
+                q_ready();
+                q_announced = true;
             }
             if (nkv_q > 0) {
                 if (!failed) tc_fence_after_sync();

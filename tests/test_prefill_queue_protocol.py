@@ -9,9 +9,10 @@ Beyond the one-item protocol (tests/test_prefill_protocol.py) the queue adds:
   * a query tile's softmax warps copy its Q rows for each item that has work for the tile and
     arrive on q_full (four arrivals); the MMA thread waits q_full before that item's first S.
     Items without work for the tile use neither side of q_full;
-  * once an item's last P V of the tile has finished, each softmax warp checks (without
+  * once an item's last S product of the tile is done, each softmax warp checks (without
     waiting) whether the next item is published and, if it has work for the tile, starts
-    copying its Q rows before the epilogue reads O;
+    copying its Q rows, and after the item's last P V it arrives on q_full for that next item
+    before its epilogue reads O (the next item's first S product then overlaps the epilogue);
   * an item's first P V overwrites O (no accumulate), after the softmax warps read the previous
     item's O.
 The model runs random interleavings and checks that every parity wait is sound (the barrier has
@@ -203,6 +204,7 @@ def run_items(items, KST, VST, seed, rescale_p=0.2):
         gs = 0
         n = 0
         copying = None                                     # item whose Q copy this warp started early
+        announced = None                                   # ... and already arrived on q_full for
 
         def copy_q(item):
             check(q_reading[q] == 0, "Q rows of item %d copied while an S product reads the tile" % item)
@@ -213,11 +215,12 @@ def run_items(items, KST, VST, seed, rescale_p=0.2):
             if it is None:
                 break
             item, nk = it[0], it[1 + q]
-            if nk > 0:
+            if nk > 0 and announced != item:
                 if copying != item:
                     copy_q(item)
                 q_full[q].arrive()
             copying = None
+            announced = None
             for j in range(nk):
                 gj = gs + j
                 yield (s_full[q], gj, True)
@@ -242,6 +245,9 @@ def run_items(items, KST, VST, seed, rescale_p=0.2):
                         copying = nx[0]
                 gl = gs + nk - 1
                 yield (o_done[2 * q + (gl & 1)], gl >> 1, True)
+                if copying is not None:                    # the next item's Q announced before the epilogue
+                    q_full[q].arrive()
+                    announced = copying
                 check(pv_pending[q] == 0 and o_item[q] == item, "O of item %d read too early" % item)
                 o_read[q].add(w)
             gs += nk
@@ -336,8 +342,8 @@ def _mutant(old, new):
 
 @pytest.mark.parametrize("old,new", [
     # q_full used for every item (also without work): idle softmax warps run phases ahead
-    ("            if nk > 0:\n                if copying != item:\n                    copy_q(item)\n                q_full[q].arrive()\n",
-     "            if nk > 0 and copying != item:\n                copy_q(item)\n            q_full[q].arrive()\n"),
+    ("            if nk > 0 and announced != item:\n                if copying != item:\n                    copy_q(item)\n                q_full[q].arrive()\n",
+     "            if nk > 0 and announced != item and copying != item:\n                copy_q(item)\n            if announced != item:\n                q_full[q].arrive()\n"),
     # the next item's Q copy started before this item's S products are done
     ("            if nk > 0:\n                ns = (n + 1) & 1\n",
      "            if True:\n                ns = (n + 1) & 1\n"),
@@ -345,8 +351,10 @@ def _mutant(old, new):
     ("            if published >= 2:\n                yield (item_empty[slot], (published >> 1) - 1, False)\n",
      "            if False:\n                yield (item_empty[slot], (published >> 1) - 1, False)\n"),
     # the first P V of an item may start before the softmax read the previous item's O
-    ("                gl = gs + nk - 1\n                yield (o_done[2 * q + (gl & 1)], gl >> 1, True)\n                check(pv_pending[q] == 0 and o_item[q] == item, \"O of item %d read too early\" % item)\n                o_read[q].add(w)\n",
-     "                o_read[q].add(w)\n                gl = gs + nk - 1\n                yield (o_done[2 * q + (gl & 1)], gl >> 1, True)\n"),
+    # the epilogue reads O (and the next item's Q is announced) without waiting for the item's
+    # last P V
+    ("                gl = gs + nk - 1\n                yield (o_done[2 * q + (gl & 1)], gl >> 1, True)\n                if copying is not None:",
+     "                gl = gs + nk - 1\n                if copying is not None:"),
 ])
 def test_model_catches_planted_mistakes(old, new):
     bad = _mutant(old, new)
