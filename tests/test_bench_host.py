@@ -51,3 +51,30 @@ def test_nvml_poller_summary_keeps_samples_inside_the_window():
     assert s["samples"] == 2 and s["sm_mhz"] == 1965 and s["reasons"] == ["sw_power_cap"]
     assert s["power_w_max"] == 260.0 and s["sm_max_mhz"] == 1965
     assert p.summary(3.0, 4.0) is None
+
+
+def test_ncu_traffic_lookup_by_workload_schedule_and_source_hash(tmp_path, monkeypatch):
+    """A committed summary names its workload, partition (decode) or schedule (prefill), its
+    traffic per launch and the hash of the kernel sources it was taken on; a stale hash or a
+    different schedule finds nothing."""
+    monkeypatch.setattr(bench, "PROFILES", str(tmp_path))
+    h = bench.kernel_source_hash(bench.PREFILL_SOURCES)
+    (tmp_path / "a.md").write_text("workload: w1\nschedule: queue\ntraffic_bytes_per_launch: 123\n"
+                                   "kernel_source_sha256_16: %s\n" % h)
+    (tmp_path / "b.md").write_text("workload: w1\nschedule: grid\ntraffic_bytes_per_launch: 456\n"
+                                   "kernel_source_sha256_16: 0000000000000000\n")
+    (tmp_path / "c.md").write_text("workload: w2\npartition: 512\ntraffic_bytes_per_launch: 789\n"
+                                   "kernel_source_sha256_16: %s\n" % bench.kernel_source_hash())
+    assert bench.ncu_traffic_per_launch("w1", schedule="queue", sources=bench.PREFILL_SOURCES) == 123
+    assert bench.ncu_traffic_per_launch("w1", schedule="grid", sources=bench.PREFILL_SOURCES) is None   # stale
+    assert bench.ncu_traffic_per_launch("w2", 512) == 789
+    assert bench.ncu_traffic_per_launch("w2", 1024) is None
+    assert bench.ncu_traffic_per_launch("w1", schedule="queue") is None       # decode sources' hash differs
+
+
+def test_prefill_row_failure_is_reported_not_raised(monkeypatch):
+    def boom(args):
+        raise RuntimeError("no GPU here")
+    monkeypatch.setattr(bench, "run_prefill", boom)
+    row = bench.prefill_side_line(bench.parse_args([]))
+    assert row["workload"] == bench.PREFILL_SIDE_WORKLOAD and "no GPU here" in row["error"]
