@@ -4,8 +4,8 @@
 // Same computation and masking rules as paged_prefill_kernel (prefill.cuh).  A work item is
 // (pair of query tiles, KV head, sequence); a query tile is 128 rows = 128 / G tokens x the G
 // heads of the KV head, and both tiles of an item share every K/V tile it streams.  Tensor
-// memory per query tile (256 of the 512 columns): S [0,64) fp32, P0 / P1 [64,128) bf16 pairs,
-// O [128,128+D) fp32.
+// memory per query tile (256 of the 512 columns): S [0,64) fp32, P [64,96) bf16 pairs, Q dims
+// 0-63 [96,128) bf16 pairs, O [128,128+D) fp32.
 //
 // Scheduling.  With a claim counter (pa_prefill_ws) the grid is one CTA per SM and every CTA
 // claims items one after another from a global atomic counter, sequences in order of context
@@ -24,10 +24,14 @@
 //              the FMA pipe, beside the MUFU unit), stores its row of P_j (bf16) into tensor memory,
 //              rescales its row of O when its max moved, and at the end of the item normalises O
 //              and writes the output row.  It copies its Q row of each item (cp.async, zero-filled
-//              past the chunk) into the swizzled Q tile and arrives on the tile's q_full; the
-//              next item's copy starts before the epilogue when that item is published already.
+//              past the chunk) into the swizzled Q tile, puts the row's first 64 dims into
+//              tensor memory as well, and arrives on the tile's q_full; the next item's copy
+//              starts before the epilogue when that item is published already.  P has one
+//              buffer: P_j is stored once P V_{j-1} has finished (seen on o_done).
 //   warps 8-9  one MMA warp per query tile: lane 0 issues S_{j+1} = Q K_{j+1}^T (M 128, N 64,
-//              K = D, both operands in shared memory) as soon as the softmax has loaded S_j, and
+//              K = D; K from shared memory, Q dims 0-63 from tensor memory and the rest from
+//              shared memory, which leaves the N = 64 products less bound by shared-memory
+//              operand reads) as soon as the softmax has loaded S_j, and
 //              O += P_j V_j (M 128, N = D, K 64) with P read from tensor memory and V read N-major
 //              from shared memory; tcgen05.commit signals each step.  With one issuing thread per
 //              tile, one tile's barrier waits overlap the other tile's MMAs on the tensor core.
@@ -175,8 +179,9 @@ struct PrefillTcConfig {
     static constexpr int OFF_MISC = OFF_ITEMS + 64;       // tensor-memory base, abort flag
     static constexpr int OFF_SEQ = OFF_MISC + 16;         // query_start, context_lens, claim order
     static constexpr int SMEM = OFF_SEQ + (3 * kPrefillSeqsInSmem + 1) * 4 + 1024;
-    static constexpr int TMEM_PER_Q = 256;                // S [0,64), P0 [64,96), P1 [96,128), O [128, 128 + D)
+    static constexpr int TMEM_PER_Q = 256;                // S [0,64), P [64,96), Q dims 0-63 [96,128), O [128, 128 + D)
     static constexpr int COL_P = 64;
+    static constexpr int COL_QT = 96;
     static constexpr int POLY_PAIRS = 1;                  // of every 8 pairs of P, on the FMA pipe
     static constexpr int TMEM_COLS = NQ * TMEM_PER_Q;
     static constexpr int COL_O = 128;
@@ -206,7 +211,8 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BARS);
     uint64_t *k_full = bars, *k_empty = bars + KST, *v_full = bars + 2 * KST, *v_empty = v_full + VST;
-    // per query tile q and buffer b: index 2 q + b
+    // p_full / o_done: two per query tile q, used by alternate steps g (index 2 q + g % 2), so a
+    // parity wait never meets a barrier more than one phase ahead
     uint64_t *s_full = bars + 2 * KST + 2 * VST, *s_free = s_full + NQ, *p_full = s_free + NQ, *o_done = p_full + 2 * NQ;
     uint64_t *drain = o_done + 2 * NQ;                          // one per query tile
     uint64_t *q_full = drain + NQ;                              // one per query tile: Q copied
@@ -482,7 +488,8 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
         // arrival falls into that tile's phase of the empty barrier).  Ring slots and the S / P
         // / O barriers are counted across items (gk: KV tiles so far, gs: this tile's steps so far).
         const int q = warp - C::MMA_WARP;
-        const uint32_t d_s = tmem + q * C::TMEM_PER_Q, d_o = d_s + C::COL_O, d_p = d_s + C::COL_P;
+        const uint32_t d_s = tmem + q * C::TMEM_PER_Q, d_o = d_s + C::COL_O, d_p = d_s + C::COL_P,
+                       d_qt = d_s + C::COL_QT;
         const uint64_t qdesc = umma_desc_sw128(smem_addr(smem + C::OFF_Q + q * C::Q_BYTES), 16, 1024);
         const uint64_t kdesc = umma_desc_sw128(smem_addr(smem + C::OFF_K), 16, 1024);
         const uint64_t vdesc = umma_desc_sw128(smem_addr(smem + C::OFF_V), C::KV_HALF, 1024);
@@ -501,9 +508,14 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
                     tc_fence_after_sync();
                     const uint64_t kd = kdesc + (uint64_t)((st * C::KV_TILE) >> 4);
 #pragma unroll
-                    for (int ks = 0; ks < D / 16; ++ks)
-                        umma_bf16_ss(d_s, qdesc + (uint64_t)(((ks >> 2) * C::Q_HALF + (ks & 3) * 32) >> 4),
-                                     kd + (uint64_t)(((ks >> 2) * C::KV_HALF + (ks & 3) * 32) >> 4), C::IDESC_S, ks > 0);
+                    for (int ks = 0; ks < D / 16; ++ks) {
+                        const uint64_t kb = kd + (uint64_t)(((ks >> 2) * C::KV_HALF + (ks & 3) * 32) >> 4);
+                        if (ks < 4)         // dims 0-63 of Q from tensor memory: only K is read from shared memory
+                            umma_bf16_ts(d_s, d_qt + 8 * ks, kb, C::IDESC_S, ks > 0);
+                        else
+                            umma_bf16_ss(d_s, qdesc + (uint64_t)(((ks >> 2) * C::Q_HALF + (ks & 3) * 32) >> 4), kb,
+                                         C::IDESC_S, ks > 0);
+                    }
                     umma_commit(&s_full[q]);
                     umma_commit(&k_empty[st]);
                     return true;
@@ -514,7 +526,7 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
                     if (!mbar_wait_or_abort(&p_full[2 * q + (gi & 1)], (gi >> 1) & 1, abort_flag) || *abort_flag) return false;
                     tc_fence_after_sync();
                     const uint64_t vd = vdesc + (uint64_t)(((gt % VST) * C::KV_TILE) >> 4);
-                    const uint32_t pt = d_p + 32 * (gi & 1);
+                    const uint32_t pt = d_p;
 #pragma unroll
                     for (int kk = 0; kk < BN / 16; ++kk)
                         umma_bf16_ts(d_o, pt + 8 * kk, vd + (uint64_t)((kk * 2048) >> 4), C::IDESC_O, i > 0 || kk > 0);
@@ -575,7 +587,21 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
         // this thread's copies landed; once all four warps arrive the MMA warp may read the tile
         auto q_ready = [&]() {
             cp_async_wait_all();
+            {
+                // dims 0-63 of this row also into tensor memory (lane t, two dims per column), the
+                // A operand of the first four k-steps of S
+                const uint8_t *qt = smem + C::OFF_Q + q * C::Q_BYTES;
+#pragma unroll 1
+                for (int c = 0; c < 8; c += 2) {
+                    const uint4 a = *reinterpret_cast<const uint4 *>(qt + swz128(t, c));
+                    const uint4 b = *reinterpret_cast<const uint4 *>(qt + swz128(t, c + 1));
+                    const uint32_t r[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+                    tmem_st8(lane_tm + (uint32_t)(C::COL_QT + 4 * c), r);
+                }
+                tmem_wait_st();
+            }
             fence_proxy_async_smem();
+            tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(&q_full[q]);
         };
@@ -687,15 +713,15 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
                     }
                     tmem_wait_st();
                 }
-                // P buffer gj % 2 is free once P V_{gj-2} has finished
-                if (gj >= 2) {
-                    ok = __all_sync(FULL, mbar_wait_or_abort(&my_o_done[gj & 1], ((gj - 2) >> 1) & 1, abort_flag));
+                // the P columns are free once P V_{gj-1} has finished
+                if (gj >= 1) {
+                    ok = __all_sync(FULL, mbar_wait_or_abort(&my_o_done[(gj - 1) & 1], ((gj - 1) >> 1) & 1, abort_flag));
                     if (!ok || *abort_flag) {
                         failed = true;
                         break;
                     }
                 }
-                tmem_st32(lane_tm + (uint32_t)(C::COL_P + 32 * (gj & 1)), pk);
+                tmem_st32(lane_tm + (uint32_t)C::COL_P, pk);
                 tmem_wait_st();
                 tc_fence_before_sync();
                 __syncwarp();

@@ -4,25 +4,26 @@ Roles, as the kernel runs them for one CTA (two 128-row query tiles q = 0, 1):
   * K producer / V producer warps: tile it goes to slot it % ST after the slot's empty barrier
     completed phase it / ST - 1; its data lands later (the full barrier completes then);
   * one MMA thread per query tile: S_j needs K_j and (j > 0) s_free phase j - 1; P V_j needs V_j
-    and p_full phase j >> 1 of buffer j & 1; completions arrive on s_full / k_empty and o_done /
+    and p_full phase j >> 1 of barrier j & 1 (two barriers, one P buffer); completions arrive on s_full / k_empty and o_done /
     v_empty in issue order (tcgen05.commit); past its KV range the thread releases each K and V
     slot as its data lands;
-  * four softmax warps per query tile: first write the tile's Q rows to shared memory and
-    arrive q_full (the MMA thread waits for it before S_0); then wait s_full phase j, load S_j, arrive s_free; sometimes
+  * four softmax warps per query tile: first write the tile's Q rows to shared memory (and the
+    first 64 dims of them to tensor memory) and arrive q_full (the MMA thread waits for it before
+    S_0); then wait s_full phase j, load S_j, arrive s_free; sometimes
     rescale O (wait o_done of P V_{j-1}); on the context's last tile wait V_j (zeroing rows);
-    before storing P_j wait o_done of P V_{j-2}; arrive p_full; at the end wait o_done of the
+    before storing P_j wait o_done of P V_{j-1}; arrive p_full; at the end wait o_done of the
     last P V and read O.
 An mbarrier parity wait for phase k passes when the number of completed phases has a parity
 other than k's, so it is only sound if that number is k or k + 1 whenever the wait is tried:
 k - 1 would pass early, k + 2 would never pass.  The model runs random interleavings and checks
 that every wait respects this, that every role finishes without deadlock, and that no shared
 buffer is overwritten while an operation still reads it or read before it holds the right tile
-(K / V slots, S, the two P buffers, O).
+(K / V slots, S, the P buffer, O).
 
-One finding: the wait before storing P_j (for P V_{j-2}) is implied by the others.  S_j's
-commit is issued after P V_{j-2}'s on the same MMA thread and tcgen05.commit arrives only when
-all of that thread's earlier operations have finished, so a softmax that has S_j sees P V_{j-2}
-done; the kernel keeps the wait, which passes at once.
+The wait before storing P_j (for P V_{j-1}) is not implied by the others: S_j's commit is issued
+before P V_{j-1} on the MMA thread (S_j overlaps softmax j - 1), so a softmax that has S_j knows
+nothing of P V_{j-1}; a planted mistake that drops the wait is caught.  (With two P buffers the
+wait was for P V_{j-2}, which S_j's commit did imply.)
 """
 import inspect
 import random
@@ -76,8 +77,8 @@ def run(nkv_q, KST, VST, seed, ctx_last_tile=True, rescale_p=0.2, abort_p=0.0, b
     sbuf = [None] * NQ                                     # tile of the completed S product
     s_pending = [False] * NQ                               # an S product is writing S
     sloaded = [[-1] * 4 for _ in range(NQ)]                # last S tile each softmax warp loaded
-    pbuf = [[[None] * 4 for _ in range(2)] for _ in range(NQ)]   # tile of P per buffer and warp
-    pread = [[0, 0] for _ in range(NQ)]                    # pending P V reading each P buffer
+    pbuf = [[None] * 4 for _ in range(NQ)]                 # tile of P each warp stored (one buffer)
+    pread = [0] * NQ                                       # pending P V reading the P buffer
     pv_pending = [0] * NQ                                  # pending P V (writes O)
     inflight = []                                          # (kind, slot, tile) still landing
     tc_queue = [[] for _ in range(NQ)]                     # per MMA thread: completions in order
@@ -142,14 +143,14 @@ def run(nkv_q, KST, VST, seed, ctx_last_tile=True, rescale_p=0.2, abort_p=0.0, b
             if not (yield (p_full[2 * q + b], i >> 1, True)) or abort[0]:
                 return False
             check(vslot[st] == i, "P V_%d reads V slot %d holding %s" % (i, st, vslot[st]))
-            check(all(x == i for x in pbuf[q][b]), "P V_%d reads P buffer %d holding %s" % (i, b, pbuf[q][b]))
+            check(all(x == i for x in pbuf[q]), "P V_%d reads P holding %s" % (i, pbuf[q]))
             vread[st].add((q, i))
-            pread[q][b] += 1
+            pread[q] += 1
             pv_pending[q] += 1
 
             def done():
                 vread[st].discard((q, i))
-                pread[q][b] -= 1
+                pread[q] -= 1
                 pv_pending[q] -= 1
                 o_done[2 * q + b].arrive()
                 v_empty[st].arrive()
@@ -201,11 +202,11 @@ def run(nkv_q, KST, VST, seed, ctx_last_tile=True, rescale_p=0.2, abort_p=0.0, b
                     return
                 check(vslot[j % VST] == j, "zeroing rows of V_%d in the wrong slot contents" % j)
             b = j & 1
-            if j >= 2:
-                if not (yield (o_done[2 * q + b], (j - 2) >> 1, True)) or abort[0]:
+            if j >= 1:
+                if not (yield (o_done[2 * q + ((j - 1) & 1)], (j - 1) >> 1, True)) or abort[0]:
                     return
-            check(pread[q][b] == 0, "P_%d stored into buffer %d while a P V reads it" % (j, b))
-            pbuf[q][b][w] = j
+            check(pread[q] == 0, "P_%d stored while a P V reads the P buffer" % j)
+            pbuf[q][w] = j
             p_full[2 * q + b].arrive()
         if n > 0:
             if (yield (o_done[2 * q + ((n - 1) & 1)], (n - 1) >> 1, True)) and not abort[0]:
@@ -312,11 +313,15 @@ def _mutant(old, new):
 
 
 @pytest.mark.parametrize("old,new", [
-    # the softmax stores P_j after waiting for P V_{j-1}'s buffer phase instead of P V_{j-2}'s
-    ("yield (o_done[2 * q + b], (j - 2) >> 1, True)", "yield (o_done[2 * q + b], (j - 0) >> 1, True)"),
+    # the softmax stores P_j without waiting for P V_{j-1}, which may still read the P buffer
+    ("            if j >= 1:\n                if not (yield (o_done[2 * q + ((j - 1) & 1)], (j - 1) >> 1, True)) or abort[0]:\n                    return\n            check(pread",
+     "            check(pread"),
+    # ... or after P V_{j-2} only (the rule for two P buffers)
+    ("            if j >= 1:\n                if not (yield (o_done[2 * q + ((j - 1) & 1)], (j - 1) >> 1, True)) or abort[0]:\n                    return\n            check(pread",
+     "            if j >= 2:\n                if not (yield (o_done[2 * q + b], (j - 2) >> 1, True)) or abort[0]:\n                    return\n            check(pread"),
     # O rescaled after waiting for P V_{j-2} instead of P V_{j-1} (P V_{j-1} may still be adding)
-    ("yield (o_done[2 * q + ((j - 1) & 1)], (j - 1) >> 1, True)",
-     "yield (o_done[2 * q + (j & 1)], max(j - 2, 0) >> 1, True)"),
+    ("            if j > 0 and rnd.random() < rescale_p:\n                if not (yield (o_done[2 * q + ((j - 1) & 1)], (j - 1) >> 1, True)) or abort[0]:",
+     "            if j > 0 and rnd.random() < rescale_p:\n                if not (yield (o_done[2 * q + (j & 1)], max(j - 2, 0) >> 1, True)) or abort[0]:"),
     # a K slot is released after one query tile's S instead of both
     ("k_empty = [Bar(NQ) for _ in range(KST)]", "k_empty = [Bar(1) for _ in range(KST)]"),
     # S_0 issued without waiting for the softmax warps' Q rows

@@ -9,6 +9,9 @@ Beyond the one-item protocol (tests/test_prefill_protocol.py) the queue adds:
   * a query tile's softmax warps copy its Q rows for each item that has work for the tile and
     arrive on q_full (four arrivals); the MMA thread waits q_full before that item's first S.
     Items without work for the tile use neither side of q_full;
+  * each softmax warp also writes its rows of Q's first 64 dims into tensor memory (the A
+    operand of the first four k-steps of S) right before it arrives on q_full;
+  * one P buffer per tile: before storing P of step g a softmax warp waits for P V of step g - 1;
   * once an item's last S product of the tile is done, each softmax warp checks (without
     waiting) whether the next item is published and, if it has work for the tile, starts
     copying its Q rows, and after the item's last P V it arrives on q_full for that next item
@@ -17,8 +20,9 @@ Beyond the one-item protocol (tests/test_prefill_protocol.py) the queue adds:
     item's O.
 The model runs random interleavings and checks that every parity wait is sound (the barrier has
 completed k or k + 1 phases when a wait for phase k is tried), that nothing deadlocks, that an
-S product reads Q holding its own item's rows from all four warps, that no Q copy starts while
-an S product still reads the tile, that the first P V of an item starts only after the previous
+S product reads Q holding its own item's rows from all four warps, that no Q copy starts and
+no Q row is written to tensor memory while an S product still reads the tile, that P is not
+overwritten while a P V reads it, that the first P V of an item starts only after the previous
 item's O was read by all four warps, and that the K / V slots hold the tile each MMA expects.
 """
 import inspect
@@ -56,8 +60,8 @@ def run_items(items, KST, VST, seed, rescale_p=0.2):
     sbuf = [None] * NQ
     s_pending = [False] * NQ
     sloaded = [[-1] * 4 for _ in range(NQ)]
-    pbuf = [[[None] * 4 for _ in range(2)] for _ in range(NQ)]
-    pread = [[0, 0] for _ in range(NQ)]
+    pbuf = [[None] * 4 for _ in range(NQ)]               # step whose P each warp stored (one P buffer)
+    pread = [0] * NQ                                       # pending P V reading the P columns
     pv_pending = [0] * NQ
     o_item = [None] * NQ                                   # item whose P V sums are in O
     o_read = [set() for _ in range(NQ)]                    # warps that read O of o_item
@@ -162,19 +166,19 @@ def run_items(items, KST, VST, seed, rescale_p=0.2):
                 yield (v_full[st], gt // VST, True)
                 yield (p_full[2 * q + b], gi >> 1, True)
                 check(vslot[st] == gt, "P V reads V slot %d holding %s, wants %d" % (st, vslot[st], gt))
-                check(all(x == gi for x in pbuf[q][b]), "P V %d reads P buffer %s" % (gi, pbuf[q][b]))
+                check(all(x == gi for x in pbuf[q]), "P V %d reads P holding %s" % (gi, pbuf[q]))
                 if i == 0:
                     check(o_item[q] is None or len(o_read[q]) == 4,
                           "item %d overwrites O before item %s's O was read" % (item, o_item[q]))
                     o_item[q] = item
                     o_read[q] = set()
                 vread[st].add((q, gi))
-                pread[q][b] += 1
+                pread[q] += 1
                 pv_pending[q] += 1
 
                 def done():
                     vread[st].discard((q, gi))
-                    pread[q][b] -= 1
+                    pread[q] -= 1
                     pv_pending[q] -= 1
                     o_done[2 * q + b].arrive()
                     v_empty[st].arrive()
@@ -210,6 +214,11 @@ def run_items(items, KST, VST, seed, rescale_p=0.2):
             check(q_reading[q] == 0, "Q rows of item %d copied while an S product reads the tile" % item)
             qrows[q][w] = item
 
+        def announce_q():
+            # the warp's rows of Q's first 64 dims go into tensor memory right before q_full
+            check(q_reading[q] == 0, "Q written to tensor memory while an S product reads it")
+            q_full[q].arrive()
+
         while True:
             it = yield from read_item(n)
             if it is None:
@@ -218,7 +227,7 @@ def run_items(items, KST, VST, seed, rescale_p=0.2):
             if nk > 0 and announced != item:
                 if copying != item:
                     copy_q(item)
-                q_full[q].arrive()
+                announce_q()
             copying = None
             announced = None
             for j in range(nk):
@@ -231,10 +240,10 @@ def run_items(items, KST, VST, seed, rescale_p=0.2):
                     yield (o_done[2 * q + ((gj - 1) & 1)], (gj - 1) >> 1, True)
                     check(pv_pending[q] == 0, "O rescaled while a P V is pending")
                 b = gj & 1
-                if gj >= 2:
-                    yield (o_done[2 * q + b], (gj - 2) >> 1, True)
-                check(pread[q][b] == 0, "P stored into buffer %d while a P V reads it" % b)
-                pbuf[q][b][w] = gj
+                if gj >= 1:
+                    yield (o_done[2 * q + ((gj - 1) & 1)], (gj - 1) >> 1, True)
+                check(pread[q] == 0, "P %d stored while a P V reads the P columns" % gj)
+                pbuf[q][w] = gj
                 p_full[2 * q + b].arrive()
             if nk > 0:
                 ns = (n + 1) & 1
@@ -246,7 +255,7 @@ def run_items(items, KST, VST, seed, rescale_p=0.2):
                 gl = gs + nk - 1
                 yield (o_done[2 * q + (gl & 1)], gl >> 1, True)
                 if copying is not None:                    # the next item's Q announced before the epilogue
-                    q_full[q].arrive()
+                    announce_q()
                     announced = copying
                 check(pv_pending[q] == 0 and o_item[q] == item, "O of item %d read too early" % item)
                 o_read[q].add(w)
@@ -342,15 +351,20 @@ def _mutant(old, new):
 
 @pytest.mark.parametrize("old,new", [
     # q_full used for every item (also without work): idle softmax warps run phases ahead
-    ("            if nk > 0 and announced != item:\n                if copying != item:\n                    copy_q(item)\n                q_full[q].arrive()\n",
-     "            if nk > 0 and announced != item and copying != item:\n                copy_q(item)\n            if announced != item:\n                q_full[q].arrive()\n"),
+    ("            if nk > 0 and announced != item:\n                if copying != item:\n                    copy_q(item)\n                announce_q()\n",
+     "            if nk > 0 and announced != item and copying != item:\n                copy_q(item)\n            if announced != item:\n                announce_q()\n"),
     # the next item's Q copy started before this item's S products are done
     ("            if nk > 0:\n                ns = (n + 1) & 1\n",
      "            if True:\n                ns = (n + 1) & 1\n"),
     # the next item published before the slot's previous item was read by every warp
     ("            if published >= 2:\n                yield (item_empty[slot], (published >> 1) - 1, False)\n",
      "            if False:\n                yield (item_empty[slot], (published >> 1) - 1, False)\n"),
-    # the first P V of an item may start before the softmax read the previous item's O
+    # P stored without waiting for the previous step's P V, which may still read the P columns
+    ("                if gj >= 1:\n                    yield (o_done[2 * q + ((gj - 1) & 1)], (gj - 1) >> 1, True)\n                check(pread",
+     "                check(pread"),
+    # the two-buffer rule (wait for P V of step g - 2) with one buffer
+    ("                if gj >= 1:\n                    yield (o_done[2 * q + ((gj - 1) & 1)], (gj - 1) >> 1, True)\n                check(pread",
+     "                if gj >= 2:\n                    yield (o_done[2 * q + b], (gj - 2) >> 1, True)\n                check(pread"),
     # the epilogue reads O (and the next item's Q is announced) without waiting for the item's
     # last P V
     ("                gl = gs + nk - 1\n                yield (o_done[2 * q + (gl & 1)], gl >> 1, True)\n                if copying is not None:",
