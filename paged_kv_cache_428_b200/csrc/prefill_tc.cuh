@@ -46,7 +46,7 @@
 //              landed and before the tile is marked full (an unwritten NaN slot times a zero
 //              probability would poison O).  The K warp also claims the work items and
 //              publishes each through a two-entry ring in shared memory that every other warp
-//              reads; it claims the next item once the current one's first tiles are issued.
+//              reads; it claims the next item once the current one's last K tile is issued.
 // Every wait on the data path is bounded and also ends when another role has stopped the CTA; on
 // a timeout or a bad block the CTA records the error, stops claiming, writes NaN into the rows
 // of the items it holds, waits for its copies and MMAs in flight and frees its tensor memory.
@@ -309,7 +309,9 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
         // 32 are in flight meanwhile), lane 0 waits for the ring slot, and lane l issues the copy
         // of block l / HALVES, half l % HALVES of the tile.  The K warp also claims the work
         // items and publishes them through the two-entry ring; it claims the next item once it
-        // has filled its ring with the current one, so that claim latency is hidden.
+        // has issued the current item's last K tile: the ring then still holds about KST tiles
+        // of the current item, which hides the claim and the next item's first table reads, and
+        // a CTA deep in a long item does not hold on to an item that an idle CTA could run.
         const bool is_v = warp != C::TMA_WARP;
         const int nst = is_v ? VST : KST;
         uint64_t *full = is_v ? v_full : k_full;
@@ -459,7 +461,7 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&full[st]);     // completes the phase (no bytes expected)
                 }
-                if (!next_known && (t == nst - 1 || t == nkv - 1)) {
+                if (!next_known && t == nkv - 1) {
                     claim(nxt);
                     publish(nxt);
                     next_known = true;

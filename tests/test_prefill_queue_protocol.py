@@ -4,7 +4,7 @@ one CTA processing a sequence of work items.
 Beyond the one-item protocol (tests/test_prefill_protocol.py) the queue adds:
   * the K producer warp publishes items through a two-entry ring (item_full / item_empty; every
     reading warp arrives on item_empty once per item) and publishes the next item once it has
-    issued the current item's first min(KST, nkv) tiles;
+    issued the current item's last K tile;
   * the K / V rings, the S, P and O barriers are counted across items;
   * a query tile's softmax warps copy its Q rows for each item that has work for the tile and
     arrive on q_full (four arrivals); the MMA thread waits q_full before that item's first S.
@@ -102,7 +102,7 @@ def run_items(items, KST, VST, seed, rescale_p=0.2):
                 kslot[st] = None
                 inflight.append((False, st, issued))
                 issued += 1
-                if not known and (t == KST - 1 or t == nkv - 1):
+                if not known and t == nkv - 1:
                     yield from publish(nxt)
                     known = True
             if not known:
