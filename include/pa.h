@@ -268,7 +268,8 @@ size_t pa_prefill_workspace_size(void);
  *                    before anything else, nothing launched.
  * The grid is one CTA per SM; each CTA claims work items from the counter in the workspace,
  * sequences in order of context length, longest first (for up to 1024 sequences; beyond that
- * in sequence order), and prepares the next item (block-table reads, K/V and Q copies) while it
+ * in sequence order), within a sequence the longest query-tile pairs first (each for every KV
+ * head), and prepares the next item (block-table reads, K/V and Q copies) while it
  * finishes the current one.  The caller's memory is not allocated, freed or resized. With
  * PA_PREFILL_MMA_SYNC=1 the mma.sync kernel runs, which does not use the workspace. */
 int pa_prefill_ws(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,

@@ -9,8 +9,9 @@
 //
 // Scheduling.  With a claim counter (pa_prefill_ws) the grid is one CTA per SM and every CTA
 // claims items one after another from a global atomic counter, sequences in order of context
-// length, longest first, and the items of one (sequence, KV head) next to each other so that
-// CTAs running at the same time share their K/V tiles through L2.  Without one (pa_prefill) the
+// length, longest first, and within a sequence pair by pair (longest KV range first), each pair
+// for every KV head: the items of a sequence run at about the same time, so they share their
+// K/V tiles through L2, and the last items claimed are the shortest.  Without one (pa_prefill) the
 // grid has one CTA per item.  In both cases the next item is known before the current one ends:
 // the producers start its block-table reads and K/V copies while the current item's last tiles
 // are in use, and the softmax warps start copying its Q rows once the current item's P V products
@@ -334,23 +335,28 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
             for (int i = 0; i < IT_N; ++i) it[i] = -1;
             if (lane == 0) {
                 while (more) {
-                    int kk;
+                    int x, kvh, zi;
                     if (claiming) {
                         if (*abort_flag) {
                             more = false;
                             break;
                         }
-                        kk = atomicAdd(sc.counters, 1);
+                        const int kk = atomicAdd(sc.counters, 1);
                         if (kk >= sc.total_items) {
                             more = false;
                             break;
                         }
+                        // within a sequence pair-major (every KV head's pair x, then pair x + 1):
+                        // the last items claimed are the shortest pairs of all heads
+                        kvh = kk % p.h_kv;
+                        x = (kk / p.h_kv) % sc.pairs_max;
+                        zi = kk / (p.h_kv * sc.pairs_max);
                     } else {
-                        kk = blockIdx.x + sc.pairs_max * (blockIdx.y + p.h_kv * blockIdx.z);
+                        x = blockIdx.x;
+                        kvh = blockIdx.y;
+                        zi = blockIdx.z;
                         more = false;                          // one item per CTA
                     }
-                    const int x = kk % sc.pairs_max, r = kk / sc.pairs_max;
-                    const int kvh = r % p.h_kv, zi = r / p.h_kv;
                     const int seq = tables ? seq_order[zi] : zi;
                     const int q0 = seq_q0(seq), chunk = seq_q0(seq + 1) - q0, ctx = seq_cx(seq);
                     if (chunk > ctx) {                         // rows left unwritten, flagged
