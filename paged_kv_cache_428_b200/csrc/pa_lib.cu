@@ -158,6 +158,25 @@ int make_cache_map(CUtensorMap *map, const void *cache, int num_blocks, int h_kv
     return r == CUDA_SUCCESS ? PA_OK : PA_ERR_CUDA;
 }
 
+// The prefill queries q [tokens][h_q][head_dim] as a 3-D map (head_dim, h_q, tokens) whose box is
+// one query tile: 64 elements (128 bytes, 128-byte swizzle) x g heads x 128 / g tokens, landing as
+// the swizzled Q tile the S products read.  `tokens` only bounds the coordinates: the kernel loads
+// only tiles that lie inside their sequence's chunk.  q must be 16-byte aligned with 16-byte
+// strides, else the encoding fails and the kernel copies every tile itself.
+int make_q_map(CUtensorMap *map, const void *q, int h_q, int head_dim, int g, long long tokens)
+{
+    EncodeTiledFn enc = encode_tiled();
+    if (!enc || tokens <= 0 || 128 % g != 0) return PA_ERR_CUDA;
+    const cuuint64_t dims[3] = {(cuuint64_t)head_dim, (cuuint64_t)h_q, (cuuint64_t)tokens};
+    const cuuint64_t strides[2] = {(cuuint64_t)head_dim * 2, (cuuint64_t)h_q * head_dim * 2};
+    const cuuint32_t box[3] = {64u, (cuuint32_t)g, (cuuint32_t)(128 / g)};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(q), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? PA_OK : PA_ERR_CUDA;
+}
+
 // Encoded maps of recently used caches (per host thread): a decode step reuses the same
 // cache tensors call after call, and encoding costs host time on every launch otherwise.
 struct CachedMap {
@@ -762,13 +781,16 @@ int launch_prefill_tc(const PrefillParams &pp, int num_seqs, int max_query_len, 
     sc.num_seqs = num_seqs;
     sc.pairs_max = pairs;
     sc.total_items = (int)items;
+    CUtensorMap mq;
+    sc.q_tma = make_q_map(&mq, pp.q, pp.h_q, D, G, (long long)num_seqs * max_query_len) == PA_OK;
+    if (!sc.q_tma) std::memset(&mq, 0, sizeof(mq));
     dim3 grid(pairs, pp.h_kv, num_seqs);                      // one CTA per item
     if (counters) {
         const int sms = sm_count();                              // one CTA per SM, claiming items
         if (sms <= 0) return PA_ERR_CUDA;
         grid = dim3((unsigned)std::min<long long>(sms, items));
     }
-    paged_prefill_tc_kernel<D, BS, G><<<grid, C::THREADS, C::SMEM, st>>>(pp, sc, mk, mv);
+    paged_prefill_tc_kernel<D, BS, G><<<grid, C::THREADS, C::SMEM, st>>>(pp, sc, mk, mv, mq);
     return launch_status();
 }
 

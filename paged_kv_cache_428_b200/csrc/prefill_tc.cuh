@@ -24,10 +24,11 @@
 //              max and sum (log2 domain; one in eight of the exponentials by a polynomial on
 //              the FMA pipe, beside the MUFU unit), stores its row of P_j (bf16) into tensor memory,
 //              rescales its row of O when its max moved, and at the end of the item normalises O
-//              and writes the output row.  It copies its Q row of each item (cp.async, zero-filled
-//              past the chunk) into the swizzled Q tile, puts the row's first 64 dims into
-//              tensor memory as well, and arrives on the tile's q_full; the next item's copy
-//              starts before the epilogue when that item is published already.  P has one
+//              and writes the output row.  A query tile wholly inside its chunk arrives in the
+//              swizzled Q tile by one TMA load from the K producer; otherwise each thread copies
+//              its Q row (cp.async, zero-filled past the chunk), starting before the epilogue
+//              when the next item is published already.  Either way the thread then puts the
+//              row's first 64 dims into tensor memory and arrives on the tile's q_full.  P has one
 //              buffer: P_j is stored once P V_{j-1} has finished (seen on o_done).
 //   warps 8-9  one MMA warp per query tile: lane 0 issues S_{j+1} = Q K_{j+1}^T (M 128, N 64,
 //              K = D; K from shared memory, Q dims 0-63 from tensor memory and the rest from
@@ -47,7 +48,10 @@
 //              landed and before the tile is marked full (an unwritten NaN slot times a zero
 //              probability would poison O).  The K warp also claims the work items and
 //              publishes each through a two-entry ring in shared memory that every other warp
-//              reads; it claims the next item once the current one's last K tile is issued.
+//              reads; it claims the next item once the current one's last K tile is issued.  At
+//              the start of an item it loads the item's whole query tiles (3-D TMA of q, one box
+//              per tile) once both tiles have released the previous item's last K tile, i.e. once
+//              every S product that read the Q tiles has finished.
 // Every wait on the data path is bounded and also ends when another role has stopped the CTA; on
 // a timeout or a bad block the CTA records the error, stops claiming, writes NaN into the rows
 // of the items it holds, waits for its copies and MMAs in flight and frees its tensor memory.
@@ -122,6 +126,16 @@ __device__ __forceinline__ void cp_async_16_zfill(void *dst, const void *src, bo
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
+// 3-D tiled TMA load global -> shared (no multicast), completing on an mbarrier.
+__device__ __forceinline__ void tma_load_3d(void *dst, const void *tmap, int x, int y, int z, uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar))
+        : "memory");
+}
+
 // Non-blocking test of an mbarrier phase (test_wait never suspends the thread).
 __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity)
 {
@@ -148,6 +162,7 @@ struct PrefillSched {
     int num_seqs;
     int pairs_max;      // query-tile pairs of the longest chunk = items per (sequence, KV head)
     int total_items;    // num_seqs * h_kv * pairs_max
+    int q_tma;          // the Q tensor map is valid: query tiles inside their chunk come by TMA
 };
 
 template <int D, int BS, int G, int NQ_ = 2, int KST_ = 4, int VST_ = 4>
@@ -174,8 +189,8 @@ struct PrefillTcConfig {
     static constexpr int OFF_V = OFF_K + KST * KV_TILE;
     static constexpr int OFF_BARS = OFF_V + VST * KV_TILE;
     // k, v full/empty; per tile: s full, s free, p full x2, o done x2, drain, q full; item ring
-    // full x2 / empty x2; the V tail copy
-    static constexpr int NBARS = 2 * KST + 2 * VST + NQ * 8 + 5;
+    // full x2 / empty x2; the V tail copy; per tile: Q landed (TMA)
+    static constexpr int NBARS = 2 * KST + 2 * VST + NQ * 9 + 5;
     static constexpr int OFF_ITEMS = OFF_BARS + NBARS * 8;   // item ring: 2 x 8 ints
     static constexpr int OFF_MISC = OFF_ITEMS + 64;       // tensor-memory base, abort flag
     static constexpr int OFF_SEQ = OFF_MISC + 16;         // query_start, context_lens, claim order
@@ -202,7 +217,7 @@ enum { IT_SEQ, IT_KVH, IT_PAIR, IT_Q0, IT_CHUNK, IT_CTX, IT_NKV0, IT_NKV1, IT_N 
 template <int D, int BS, int G, int NQ_ = 2, int KST_ = 4, int VST_ = 4>
 __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::THREADS, 1)
     paged_prefill_tc_kernel(const PrefillParams p, const PrefillSched sc, const __grid_constant__ CUtensorMap tmap_k,
-                            const __grid_constant__ CUtensorMap tmap_v)
+                            const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ CUtensorMap tmap_q)
 {
     using C = PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>;
     constexpr int KST = C::KST, VST = C::VST, BN = C::BN, NQ = C::NQ;
@@ -218,6 +233,7 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
     uint64_t *drain = o_done + 2 * NQ;                          // one per query tile
     uint64_t *q_full = drain + NQ;                              // one per query tile: Q copied
     uint64_t *item_full = q_full + NQ, *item_empty = item_full + 2, *v_tail = item_empty + 2;
+    uint64_t *q_land = v_tail + 1;                               // one per query tile: its Q tile landed (TMA)
     volatile int *items = reinterpret_cast<volatile int *>(smem + C::OFF_ITEMS);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
@@ -252,6 +268,7 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
             mbar_init(&item_empty[s], C::ITEM_READERS);
         }
         mbar_init(v_tail, 1);
+        for (int q = 0; q < NQ; ++q) mbar_init(&q_land[q], 1);
         *abort_flag = 0;
         mbar_init_fence();
     }
@@ -298,6 +315,8 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
         __syncwarp();
         if (lane == 0) mbar_arrive(&item_empty[slot]);
     };
+    // query tile q of a pair lies wholly inside the chunk: its Q tile comes by one TMA load
+    auto q_by_tma = [&](int pair, int chunk, int q) { return sc.q_tma && (pair * NQ + q + 1) * C::TQ <= chunk; };
     auto nkv_tile = [&](int chunk, int ctx, int pair, int q) {
         const int t0 = (pair * NQ + q) * C::TQ;
         return t0 >= chunk ? 0 : ceil_div(ctx - chunk + min(chunk, t0 + C::TQ), BN);
@@ -403,9 +422,38 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
         } else {
             read_item(0, cur);
         }
+        int q_tma_n[NQ];                                       // K warp, lane 0: Q tiles loaded by TMA
+#pragma unroll
+        for (int qq = 0; qq < NQ; ++qq) q_tma_n[qq] = 0;
         for (int n = 0; cur[IT_SEQ] >= 0; ++n) {
             const int ctx = cur[IT_CTX], nkv = max(cur[IT_NKV0], cur[IT_NKV1]);
             const int nblk_seq = ceil_div(ctx, BS);
+            if (!is_v && sc.q_tma && lane == 0) {
+                // the item's query tiles that lie inside the chunk: one TMA load each into the Q
+                // tile, once every S product of the previous item has finished (the release of its
+                // last K tile by both query tiles says so)
+                if (issued > 0 && !*abort_flag) {
+                    const int gl = issued - 1;
+                    if (!mbar_wait_or_abort(&empty[gl % nst], (gl / nst) & 1, abort_flag)) {
+                        if (!*abort_flag) record_error(PA_DEVERR_TIMEOUT);
+                        *abort_flag = 1;
+                    }
+                }
+#pragma unroll
+                for (int qq = 0; qq < NQ; ++qq) {
+                    if ((qq == 0 ? cur[IT_NKV0] : cur[IT_NKV1]) > 0 && q_by_tma(cur[IT_PAIR], cur[IT_CHUNK], qq) &&
+                        !*abort_flag) {
+                        uint8_t *dst = smem + C::OFF_Q + qq * C::Q_BYTES;
+                        mbar_arrive_expect_tx(&q_land[qq], (uint32_t)C::Q_BYTES);
+#pragma unroll
+                        for (int h = 0; h < C::HALVES; ++h)
+                            tma_load_3d(dst + h * C::Q_HALF, &tmap_q, 64 * h, cur[IT_KVH] * G,
+                                        cur[IT_Q0] + (cur[IT_PAIR] * NQ + qq) * C::TQ, &q_land[qq]);
+                        ++q_tma_n[qq];
+                    }
+                }
+            }
+            __syncwarp();
             const int32_t *trow = p.block_tables + (size_t)cur[IT_SEQ] * p.max_blocks_per_seq;
             auto entry = [&](int lb) -> int {
                 return (lb < nblk_seq && lb < p.max_blocks_per_seq) ? __ldg(trow + lb) : -1;
@@ -485,8 +533,12 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
         // early and nobody consumed the last tiles: wait (bounded) for each of the last nst
         // tiles.  The tile nst before each was consumed before the slot was refilled, so each
         // wait's phase is unambiguous; on the normal path these waits return at once.
-        if (lane == 0)
+        if (lane == 0) {
             for (int i = max(0, issued - nst); i < issued; ++i) mbar_wait_bounded(&full[i % nst], (i / nst) & 1);
+#pragma unroll
+            for (int qq = 0; qq < NQ; ++qq)                        // and every Q tile it loaded
+                if (!is_v && q_tma_n[qq] > 0) mbar_wait_bounded(&q_land[qq], (q_tma_n[qq] - 1) & 1);
+        }
         __syncwarp();
     } else if (warp >= C::MMA_WARP && warp < C::MMA_WARP + NQ) {
         // ------------------------------ MMA issue, one warp per query tile ------------------------------
@@ -592,9 +644,10 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
 #pragma unroll
             for (int c = 0; c < D / 8; ++c) cp_async_16_zfill(qt + (c >> 3) * C::Q_HALF + swz128(t, c & 7), src + 8 * c, ok);
         };
-        // this thread's copies landed; once all four warps arrive the MMA warp may read the tile
-        auto q_ready = [&]() {
-            cp_async_wait_all();
+        int nqt = 0;                                           // Q tiles of this query tile that came by TMA
+        // the row's first 64 dims into tensor memory, then q_full: once all four warps arrive the
+        // MMA warp may read the tile
+        auto q_to_tmem = [&]() {
             {
                 // dims 0-63 of this row also into tensor memory (lane t, two dims per column), the
                 // A operand of the first four k-steps of S
@@ -613,6 +666,20 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
             __syncwarp();
             if (lane == 0) mbar_arrive(&q_full[q]);
         };
+        // this thread's copies landed
+        auto q_ready = [&]() {
+            cp_async_wait_all();
+            q_to_tmem();
+        };
+        // the tile's TMA load landed (bounded; a stopped CTA goes on with NaN rows)
+        auto q_ready_tma = [&]() {
+            if (!__all_sync(FULL, mbar_wait_or_abort(&q_land[q], nqt & 1, abort_flag)) && lane == 0) {
+                if (!*abort_flag) record_error(PA_DEVERR_TIMEOUT);
+                *abort_flag = 1;
+            }
+            ++nqt;
+            q_to_tmem();
+        };
         int gs = 0;                                            // this tile's steps so far (all items)
         bool q_copying = false;                                // the next item's Q copy is in flight
         bool q_announced = false;                              // ... and already announced on q_full
@@ -622,8 +689,12 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
             if (it[IT_SEQ] < 0) break;
             const int chunk = it[IT_CHUNK], ctx = it[IT_CTX], nkv_q = (q == 0 ? it[IT_NKV0] : it[IT_NKV1]);
             if (nkv_q > 0 && !q_announced) {                   // only items with work use q_full
-                if (!q_copying && !*abort_flag) copy_q(it[IT_PAIR], it[IT_Q0], chunk, it[IT_KVH]);
-                q_ready();
+                if (q_by_tma(it[IT_PAIR], chunk, q)) {
+                    q_ready_tma();
+                } else {
+                    if (!q_copying && !*abort_flag) copy_q(it[IT_PAIR], it[IT_Q0], chunk, it[IT_KVH]);
+                    q_ready();
+                }
             }
             q_copying = false;
             q_announced = false;
@@ -742,7 +813,8 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
                 const int ns = (n + 1) & 1;
                 if (mbar_test_wait(&item_full[ns], ((n + 1) >> 1) & 1)) {
                     const volatile int *nx = items + ns * IT_N;
-                    if (nx[IT_SEQ] >= 0 && (q == 0 ? nx[IT_NKV0] : nx[IT_NKV1]) > 0 && !*abort_flag) {
+                    if (nx[IT_SEQ] >= 0 && (q == 0 ? nx[IT_NKV0] : nx[IT_NKV1]) > 0 &&
+                        !q_by_tma(nx[IT_PAIR], nx[IT_CHUNK], q) && !*abort_flag) {
                         copy_q(nx[IT_PAIR], nx[IT_Q0], nx[IT_CHUNK], nx[IT_KVH]);
                         q_copying = true;
                     }
@@ -758,6 +830,21 @@ __global__ void __launch_bounds__(PrefillTcConfig<D, BS, G, NQ_, KST_, VST_>::TH
                 // its first S product runs during this item's epilogue
                 q_ready();
                 q_announced = true;
+            } else if (sc.q_tma && !failed && nkv_q > 0) {
+                // likewise for a next-item tile that came by TMA, if it has landed already
+                int go = 0;
+                if (lane == 0) {
+                    const int ns = (n + 1) & 1;
+                    if (mbar_test_wait(&item_full[ns], ((n + 1) >> 1) & 1)) {
+                        const volatile int *nx = items + ns * IT_N;
+                        go = nx[IT_SEQ] >= 0 && (q == 0 ? nx[IT_NKV0] : nx[IT_NKV1]) > 0 &&
+                             q_by_tma(nx[IT_PAIR], nx[IT_CHUNK], q) && mbar_test_wait(&q_land[q], nqt & 1);
+                    }
+                }
+                if (__shfl_sync(FULL, go, 0)) {
+                    q_ready_tma();
+                    q_announced = true;
+                }
             }
             if (nkv_q > 0) {
                 if (!failed) tc_fence_after_sync();

@@ -11,6 +11,10 @@ Beyond the one-item protocol (tests/test_prefill_protocol.py) the queue adds:
     Items without work for the tile use neither side of q_full;
   * each softmax warp also writes its rows of Q's first 64 dims into tensor memory (the A
     operand of the first four k-steps of S) right before it arrives on q_full;
+  * a query tile that lies wholly inside its chunk is not copied by the softmax warps: the K
+    producer loads it with one TMA (landing on q_land) at the start of the item, once both query
+    tiles have released the previous item's last K tile, and the softmax warps wait for q_land
+    (also before the epilogue, without waiting, to announce the next item's tile early);
   * one P buffer per tile: before storing P of step g a softmax warp waits for P V of step g - 1;
   * once an item's last S product of the tile is done, each softmax warp checks (without
     waiting) whether the next item is published and, if it has work for the tile, starts
@@ -34,9 +38,14 @@ import pytest
 from test_prefill_protocol import Bar, Violation, check
 
 
-def run_items(items, KST, VST, seed, rescale_p=0.2):
-    """items: list of (nkv of query tile 0, nkv of query tile 1) for one CTA."""
+def run_items(items, KST, VST, seed, rescale_p=0.2, tma_p=0.6):
+    """items: list of (nkv of query tile 0, nkv of query tile 1) for one CTA.  Each query tile of
+    an item is, at random (tma_p), one that lies wholly inside its chunk (its Q tile comes by TMA
+    from the K producer) or a ragged one (copied by the softmax warps)."""
     rnd = random.Random(seed)
+    rfull = random.Random(seed * 31 + 7)
+    q_slow = rfull.random() < 0.5
+    full = [(rfull.random() < tma_p, rfull.random() < tma_p) for _ in items]
     NQ = 2
     READERS = 4 * NQ + NQ + 1
     k_full = [Bar(1) for _ in range(KST)]
@@ -48,6 +57,7 @@ def run_items(items, KST, VST, seed, rescale_p=0.2):
     p_full = [Bar(4) for _ in range(2 * NQ)]
     o_done = [Bar(1) for _ in range(2 * NQ)]
     q_full = [Bar(4) for _ in range(NQ)]
+    q_land = [Bar(1) for _ in range(NQ)]                   # a Q tile loaded by TMA landed
     item_full = [Bar(1) for _ in range(2)]
     item_empty = [Bar(READERS) for _ in range(2)]
     ring = [None, None]
@@ -94,6 +104,15 @@ def run_items(items, KST, VST, seed, rescale_p=0.2):
             nkv = max(a, b)
             nxt = (idx + 1,) + items[idx + 1] if idx + 1 < len(items) else None
             known = False
+            # the item's whole query tiles by TMA, once both tiles released the previous item's
+            # last K tile (every S product of that item has finished)
+            if issued > 0:
+                gl = issued - 1
+                yield (k_empty[gl % KST], gl // KST, True)
+            for q in range(NQ):
+                if (a, b)[q] > 0 and full[idx][q]:
+                    check(q_reading[q] == 0, "Q tile of item %d loaded while an S product reads the tile" % idx)
+                    inflight.append(("q", q, idx))
             for t in range(nkv):
                 st = issued % KST
                 if issued >= KST:
@@ -219,15 +238,27 @@ def run_items(items, KST, VST, seed, rescale_p=0.2):
             check(q_reading[q] == 0, "Q written to tensor memory while an S product reads it")
             q_full[q].arrive()
 
+        nqt = 0
+
+        def announce_tma():
+            # a whole tile: wait for its TMA load, then as announce_q
+            nonlocal nqt
+            yield (q_land[q], nqt, True)
+            nqt += 1
+            announce_q()
+
         while True:
             it = yield from read_item(n)
             if it is None:
                 break
             item, nk = it[0], it[1 + q]
             if nk > 0 and announced != item:
-                if copying != item:
-                    copy_q(item)
-                announce_q()
+                if full[item][q]:
+                    yield from announce_tma()
+                else:
+                    if copying != item:
+                        copy_q(item)
+                    announce_q()
             copying = None
             announced = None
             for j in range(nk):
@@ -249,7 +280,7 @@ def run_items(items, KST, VST, seed, rescale_p=0.2):
                 ns = (n + 1) & 1
                 if item_full[ns].done == ((n + 1) >> 1) + 1:        # published (test_wait, no waiting)
                     nx = ring[ns]
-                    if nx is not None and nx[1 + q] > 0:
+                    if nx is not None and nx[1 + q] > 0 and not full[nx[0]][q]:
                         copy_q(nx[0])
                         copying = nx[0]
                 gl = gs + nk - 1
@@ -257,6 +288,11 @@ def run_items(items, KST, VST, seed, rescale_p=0.2):
                 if copying is not None:                    # the next item's Q announced before the epilogue
                     announce_q()
                     announced = copying
+                elif item_full[ns].done == ((n + 1) >> 1) + 1:     # likewise a whole tile whose load landed
+                    nx = ring[ns]
+                    if nx is not None and nx[1 + q] > 0 and full[nx[0]][q] and q_land[q].done == nqt + 1:
+                        yield from announce_tma()
+                        announced = nx[0]
                 check(pv_pending[q] == 0 and o_item[q] == item, "O of item %d read too early" % item)
                 o_read[q].add(w)
             gs += nk
@@ -301,9 +337,16 @@ def run_items(items, KST, VST, seed, rescale_p=0.2):
         if kind == "role":
             step(arg)
         elif kind == "land":
-            is_v, st, tile = inflight.pop(rnd.randrange(len(inflight)))
-            (vslot if is_v else kslot)[st] = tile
-            (v_full if is_v else k_full)[st].arrive()
+            i = rnd.randrange(len(inflight))
+            if inflight[i][0] == "q" and q_slow and rnd.random() < 0.95:
+                continue                                   # in half the runs Q tiles land late
+            what, st, tile = inflight.pop(i)
+            if what == "q":                                # a Q tile: all four warps' rows
+                qrows[st] = [tile] * 4
+                q_land[st].arrive()
+            else:
+                (vslot if what else kslot)[st] = tile
+                (v_full if what else k_full)[st].arrive()
         else:
             tc_queue[arg].pop(0)()
         if not inflight and not any(tc_queue) and alive:
@@ -351,8 +394,8 @@ def _mutant(old, new):
 
 @pytest.mark.parametrize("old,new", [
     # q_full used for every item (also without work): idle softmax warps run phases ahead
-    ("            if nk > 0 and announced != item:\n                if copying != item:\n                    copy_q(item)\n                announce_q()\n",
-     "            if nk > 0 and announced != item and copying != item:\n                copy_q(item)\n            if announced != item:\n                announce_q()\n"),
+    ("            if nk > 0 and announced != item:\n                if full[item][q]:",
+     "            if announced != item:\n                if full[item][q] and nk > 0:"),
     # the next item's Q copy started before this item's S products are done
     ("            if nk > 0:\n                ns = (n + 1) & 1\n",
      "            if True:\n                ns = (n + 1) & 1\n"),
@@ -365,6 +408,10 @@ def _mutant(old, new):
     # the two-buffer rule (wait for P V of step g - 2) with one buffer
     ("                if gj >= 1:\n                    yield (o_done[2 * q + ((gj - 1) & 1)], (gj - 1) >> 1, True)\n                check(pread",
      "                if gj >= 2:\n                    yield (o_done[2 * q + b], (gj - 2) >> 1, True)\n                check(pread"),
+    # a whole Q tile loaded by the K producer before the previous item's S products finished
+    ("            if issued > 0:\n                gl = issued - 1\n                yield (k_empty[gl % KST], gl // KST, True)\n", ""),
+    # a whole Q tile announced without waiting for its load to land
+    ("            yield (q_land[q], nqt, True)\n", "            if False:\n                yield\n"),
     # the epilogue reads O (and the next item's Q is announced) without waiting for the item's
     # last P V
     ("                gl = gs + nk - 1\n                yield (o_done[2 * q + (gl & 1)], gl >> 1, True)\n                if copying is not None:",
