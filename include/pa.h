@@ -236,7 +236,8 @@ int pa_decode_step(const void *key, const void *value, int64_t key_stride, int64
  * with token t of sequence s read from block block_tables[s][t / bs] at offset t % bs and
  * query head h reading KV head h / (h_q / h_kv).  The chunk's own K/V rows must be in the cache
  * (pa_reshape_and_cache of the chunk's tokens, e.g. with slots from pa_alloc_append_n).
- *   out, q         device bf16 [T][h_q][head_dim], T = query_start[num_seqs]
+ *   out, q         device bf16 [T][h_q][head_dim], T = query_start[num_seqs], 16-byte
+ *                  aligned (else PA_ERR_INVALID_ARG); T <= num_seqs * max_query_len
  *   query_start    device int32 [num_seqs + 1], non-decreasing, query_start[0] = 0
  *   context_lens   device int32 [num_seqs], each including its chunk (>= the chunk length; a
  *                  longer chunk leaves its rows unwritten and flags PA_DEVERR_BAD_CHUNK)
