@@ -247,9 +247,8 @@ int pa_decode_step(const void *key, const void *value, int64_t key_stride, int64
  * A block-table entry outside the pool is never dereferenced: it flags PA_DEVERR_BAD_BLOCK
  * and turns the affected rows into NaN.  5th-generation tensor cores (tcgen05.mma, bf16 in,
  * fp32 accumulators in tensor memory; the environment variable PA_PREFILL_MMA_SYNC=1 selects
- * an mma.sync kernel instead); accuracy as pa_decode for bf16 caches (one in eight of
- * the softmax exponentials use a cubic with relative error < 1e-4, and there terms below
- * 2^-125 of the row's running maximum come out as about that instead of 0).  Allocates nothing; needs no
+ * an mma.sync kernel instead); accuracy as pa_decode for bf16 caches (the softmax
+ * exponentials by ex2.approx).  Allocates nothing; needs no
  * workspace.  One CTA per work item (a pair of 128-row query tiles of one sequence and KV
  * head); pa_prefill_ws computes the same result with fewer, longer-lived CTAs. */
 int pa_prefill(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,

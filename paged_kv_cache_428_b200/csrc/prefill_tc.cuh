@@ -21,8 +21,9 @@
 //   warps 0-7  two softmax warpgroups, one per query tile: thread t of a warpgroup owns row t of
 //              its tile (= tensor-memory lane t).  It loads its row of S_j from tensor memory
 //              (which frees S for S_{j+1}), applies the causal / context mask, keeps the running
-//              max and sum (log2 domain; one in eight of the exponentials by a polynomial on
-//              the FMA pipe, beside the MUFU unit), stores its row of P_j (bf16) into tensor memory,
+//              max and sum (log2 domain; the exponentials on the MUFU unit, with a polynomial on
+//              the FMA pipe for POLY_PAIRS of every 8 pairs, 0 as measured best), stores its row
+//              of P_j (bf16) into tensor memory,
 //              rescales its row of O when its max moved, and at the end of the item normalises O
 //              and writes the output row.  A query tile wholly inside its chunk arrives in the
 //              swizzled Q tile by one TMA load from the K producer; otherwise each thread copies
@@ -198,7 +199,7 @@ struct PrefillTcConfig {
     static constexpr int TMEM_PER_Q = 256;                // S [0,64), P [64,96), Q dims 0-63 [96,128), O [128, 128 + D)
     static constexpr int COL_P = 64;
     static constexpr int COL_QT = 96;
-    static constexpr int POLY_PAIRS = 1;                  // of every 8 pairs of P, on the FMA pipe
+    static constexpr int POLY_PAIRS = 0;                  // of every 8 pairs of P, on the FMA pipe
     static constexpr int TMEM_COLS = NQ * TMEM_PER_Q;
     static constexpr int COL_O = 128;
     static constexpr uint32_t IDESC_S = umma_idesc_bf16(BM, BN, false);
